@@ -1,0 +1,433 @@
+#!/usr/bin/env python
+"""Benchmark: exact attention forward + backward on B200 through libfa.so's C ABI.
+
+One step = one pass of the whole hot path over one batch: fa_fwd (tiled forward with online softmax) followed by
+fa_bwd (preprocess, recomputing backward, dQ conversion).  The workload is the GPT-2-small-shaped causal
+self-attention (B=8, H=12, N=1024, d=64, bf16); the long-context causal rows (B=1, H=16, d=128, N=4096/8192/16384)
+are measured in the same run under "targets".  FLOPs are algorithmic: forward 4*d per visible (query, key) pair,
+backward 2.5x forward (five GEMM-shaped products per visible tile pair), step 3.5x forward.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--no-targets]
+
+Multi-GPU (torchrun, one process per GPU): each rank runs its own independent batch of the same shape (attention
+heads are independent, so there is no data-path collective: weak scaling); value = all ranks' FLOPs / max time.
+--impl reference times the fp64 CPU oracle (the reference arm of this repository) on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd / fwd+bwd TFLOP/s on 1 B200 and % of dense BF16 tensor peak"
+L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
+
+
+# ---------------------------------------------------------------------------------------------- FLOP accounting
+def visible_pairs(B, H, N, causal, key_lens=None, block_mask=None, tile=128):
+    """Number of (query, key) pairs the method must compute (integer, exact)."""
+    import numpy as np
+    if block_mask is None and key_lens is None:
+        return B * H * (N * (N + 1) // 2 if causal else N * N)
+    if block_mask is None and not causal:
+        return H * N * int(np.sum(np.minimum(np.asarray(key_lens, dtype=np.int64), N)))
+    # general: count per tile (rows x visible keys)
+    nT = -(-N // tile)
+    total = 0
+    lens = [N] * B if key_lens is None else [min(int(x), N) for x in key_lens]
+    for b in range(B):
+        for i in range(nT):
+            r0, r1 = i * tile, min(N, (i + 1) * tile)
+            for j in range(nT):
+                if block_mask is not None and not block_mask[i, j]:
+                    continue
+                c0, c1 = j * tile, min(N, (j + 1) * tile, lens[b])
+                if c1 <= c0:
+                    continue
+                for r in range(r0, r1):
+                    hi = min(c1, r + 1) if causal else c1
+                    total += max(0, hi - c0)
+    return total * H
+
+
+def fwd_flops(d, pairs):
+    return 4.0 * d * pairs
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), \
+            float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+# ---------------------------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while the timed region runs."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
+        "sync_boost": 0x10, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, device_index, period_s=0.002):
+        self.samples, self.reasons = [], 0
+        self.period = period_s
+        self._stop = threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # pragma: no cover - depends on the box
+            self.err = str(e)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        names = [n for n, bit in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
+                "samples": len(self.samples), "reasons": names}
+
+
+# ---------------------------------------------------------------------------------------------- GPU arm
+class Problem:
+    """Device-resident inputs, outputs and workspace for one attention workload; step() = fa_fwd + fa_bwd."""
+
+    def __init__(self, w, seed_offset=0, device="cuda"):
+        import torch
+        from exact_io_aware_48_b200 import _lib
+        self.w = w
+        self.lib = _lib
+        w.seed += seed_offset  # independent problem per rank
+        q, k, v, do = w.tensors()
+        w.seed -= seed_offset
+        self.host = [t.pin_memory() for t in (q, k, v, do)]
+        self.q, self.k, self.v, self.do = [t.to(device) for t in self.host]
+        self.o = torch.empty_like(self.q)
+        self.lse = torch.empty((w.B, w.H, w.N), device=device, dtype=torch.float32)
+        self.dq, self.dk, self.dv = (torch.empty_like(self.q) for _ in range(3))
+        self.ws_bytes = _lib.fa_bwd_workspace_size(w.B, w.H, w.N, w.d, False)
+        self.ws = torch.empty(self.ws_bytes, device=device, dtype=torch.uint8)
+        self.dt = _lib.FA_BF16 if w.dtype == "bf16" else _lib.FA_FP16
+        self.pairs = visible_pairs(w.B, w.H, w.N, w.causal, w.key_lens_array())
+        self.fwd_flops = fwd_flops(w.d, self.pairs)
+        self.kl = None
+        if w.key_lens:
+            self.kl = torch.as_tensor(w.key_lens_array(), dtype=torch.int32, device=device)
+
+    def fwd(self, stream):
+        w, L = self.w, self.lib
+        rc = L.fa_fwd(self.q, self.k, self.v, self.o, self.lse, w.B, w.H, w.N, w.d, w.scale, w.causal, self.kl,
+                      self.dt, stream)
+        if rc:
+            raise RuntimeError(f"fa_fwd: {L.fa_status_string(rc)}")
+
+    def bwd(self, stream):
+        w, L = self.w, self.lib
+        rc = L.fa_bwd(self.q, self.k, self.v, self.o, self.do, self.lse, self.dq, self.dk, self.dv, w.B, w.H, w.N,
+                      w.d, w.scale, w.causal, self.kl, None, self.ws, self.ws_bytes, self.dt, stream)
+        if rc:
+            raise RuntimeError(f"fa_bwd: {L.fa_status_string(rc)}")
+
+    def step(self, stream):
+        self.fwd(stream)
+        self.bwd(stream)
+
+
+def time_loop(fn, steps, stream, flush, kernel_events=None):
+    """Device time (ms) of each call of fn, L2 flushed before each (flush not timed).  kernel_events: optional
+    (kernel_id, lib) whose launches are bracketed by per-step events; returns (step_ms list, kernel_ms list)."""
+    import torch
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)] \
+        if kernel_events else None
+    with torch.cuda.stream(stream):
+        for s in range(steps):
+            flush.zero_()
+            if kev:
+                kernel_events[1].fa_set_kernel_events(kernel_events[0], kev[s][0], kev[s][1])
+            ev[s][0].record(stream)
+            fn(stream)
+            ev[s][1].record(stream)
+    if kev:
+        kernel_events[1].fa_set_kernel_events(kernel_events[0], None, None)
+    stream.synchronize()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    k_ms = [a.elapsed_time(b) for a, b in kev] if kev else None
+    return step_ms, k_ms
+
+
+def measure_targets(stream, flush, peak):
+    """Long-context causal rows (d=128): fwd and bwd TFLOP/s, fraction of the dense BF16 peak."""
+    from exact_io_aware_48_b200 import inputs
+    out = {}
+    for name in ("lc4k", "lc8k", "lc16k"):
+        w = inputs.workloads()[name]
+        p = Problem(w)
+        for _ in range(3):
+            p.step(stream)
+        f_ms, _ = time_loop(p.fwd, 10, stream, flush)
+        b_ms, _ = time_loop(p.bwd, 10, stream, flush)
+        f, b = statistics.median(f_ms), statistics.median(b_ms)
+        ftf = p.fwd_flops / f / 1e9
+        btf = 2.5 * p.fwd_flops / b / 1e9
+        out[name] = {"fwd_ms": round(f, 4), "bwd_ms": round(b, 4), "fwd_tflops": round(ftf, 1),
+                     "bwd_tflops": round(btf, 1), "fwd_frac": round(ftf / peak, 4), "bwd_frac": round(btf / peak, 4),
+                     "fwd_bwd_tflops": round(3.5 * p.fwd_flops / (f + b) / 1e9, 1)}
+        del p
+    return out
+
+
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    from exact_io_aware_48_b200 import _lib, inputs
+    from datetime import timedelta
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local))
+    _lib.load()
+    peak, peak_sus, hbm, peak_src = peaks()
+    stream = torch.cuda.Stream()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+
+    w = inputs.workloads()["gpt2"]
+    p = Problem(w, seed_offset=rank)
+    for _ in range(args.warmup):
+        p.step(stream)
+    stream.synchronize()
+    if _lib.fa_last_device_status(stream.cuda_stream) != 0:
+        raise RuntimeError("device status error during warm-up")
+
+    # ------------------------------------------------------------------ timed region: K steps, device-timed
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        step_ms, kern_ms = time_loop(p.step, args.steps, stream, flush, (_lib.FA_KERNEL_BWD_MAIN, _lib))
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    total_ms = float(sum(step_ms))
+    if world > 1:
+        t = torch.tensor([total_ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    if _lib.fa_last_device_status(stream.cuda_stream) != 0:
+        raise RuntimeError("device status error in timed region")
+
+    step_flops = 3.5 * p.fwd_flops
+    value = world * step_flops * args.steps / (total_ms / 1e3) / 1e12
+    ms_per_step = total_ms / args.steps
+
+    # separate fwd / bwd breakdown (not part of the headline value)
+    f_ms, fk = time_loop(p.fwd, max(10, args.steps // 2), stream, flush)
+    b_ms, _ = time_loop(p.bwd, max(10, args.steps // 2), stream, flush)
+    fwd_tf = p.fwd_flops / statistics.median(f_ms) / 1e9
+    bwd_tf = 2.5 * p.fwd_flops / statistics.median(b_ms) / 1e9
+
+    # roofline of the dominant kernel (bwd main: 2.5x forward FLOPs per launch), timed live by events
+    kmean = float(np.mean(kern_ms))
+    achieved = 2.5 * p.fwd_flops / (kmean / 1e3) / 1e12
+    roofline = {"kernel": "bwd_kernel<64,bf16>", "bound": "tensor", "achieved": round(achieved, 2),
+                "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                "peak_source": f"{peak_src} bf16_tflops (burst)", "kernel_ms": round(kmean, 4),
+                "traffic": None}
+    # ------------------------------------------------------------------ end to end through the C ABI, host buffers
+    e2e = run_e2e(p, stream, args, world)
+
+    targets = measure_targets(stream, flush, peak) if (args.targets and rank == 0) else None
+    cpu = cpu_baseline(p.w) if rank == 0 and world == 1 and args.cpu_baseline else None
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "gpt2-small-shaped causal self-attention fwd+bwd B8 H12 N1024 d64 bf16",
+                       "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": True, "global_batch": w.B * world,
+                       "seq_len": w.N, "parallelism": f"dp{world} (independent heads per rank, no collective)",
+                       "l2": "flushed (256 MiB write, untimed) before every timed step",
+                       "flop_convention": "fwd 4*d*visible pairs; bwd 2.5x; step 3.5x"},
+            "fwd_tflops": round(fwd_tf, 2), "bwd_tflops": round(bwd_tf, 2),
+            "frac_of_peak": {"step": round(value / world / peak, 4), "fwd": round(fwd_tf / peak, 4),
+                             "bwd": round(bwd_tf / peak, 4), "peak_tflops": peak, "peak_source": peak_src},
+            "roofline": roofline,
+            "e2e": e2e,
+            "gpu_launches": 4 * args.steps,
+            "clocks": clk.summary(),
+            "targets": targets,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_e2e(p, stream, args, world):
+    """Same metric through the public C ABI with host buffers: per step, copy q, k, v, dO from pinned host memory,
+    run fa_fwd + fa_bwd, copy O, LSE, dQ, dK, dV back to pinned host memory; device-timed on the stream."""
+    import torch
+    outs = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (p.o, p.lse, p.dq, p.dk, p.dv)]
+    h2d = sum(t.numel() * t.element_size() for t in p.host)
+    d2h = sum(t.numel() * t.element_size() for t in outs)
+
+    def e2e_step(s):
+        for dst, src in zip((p.q, p.k, p.v, p.do), p.host):
+            dst.copy_(src, non_blocking=True)
+        p.step(s)
+        for dst, src in zip(outs, (p.o, p.lse, p.dq, p.dk, p.dv)):
+            dst.copy_(src, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            e2e_step(stream)
+    stream.synchronize()
+    n = max(5, args.steps // 4)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        for _ in range(n):
+            e2e_step(stream)
+        ev1.record(stream)
+    stream.synchronize()
+    ms = ev0.elapsed_time(ev1) / n
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    val = world * 3.5 * p.fwd_flops / (ms / 1e3) / 1e12
+    return {"value": round(val, 3), "unit": "TFLOP/s", "ms_per_step": round(ms, 4), "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h}
+
+
+# ---------------------------------------------------------------------------------------------- CPU oracle
+def oracle_step(w, heads=None):
+    """One fwd+bwd of the fp64 oracle on the workload (optionally the first `heads` flattened heads).
+    Returns (seconds, algorithmic FLOPs of the part computed)."""
+    import oracle
+    from exact_io_aware_48_b200 import inputs
+    q, k, v, do = (inputs.to_f64(t) for t in w.tensors())
+    B, H = w.B, w.H
+    if heads is not None and heads < B * H:
+        sl = lambda x: x.reshape(B * H, w.N, w.d)[:heads].reshape(1, heads, w.N, w.d)
+        q, k, v, do = sl(q), sl(k), sl(v), sl(do)
+        B, H = 1, heads
+    kl = w.key_lens_array()
+    t0 = time.perf_counter()
+    oracle.attn_bwd(q, k, v, do, w.scale, causal=w.causal, key_lens=kl if B == w.B else None)
+    dt = time.perf_counter() - t0
+    return dt, 3.5 * fwd_flops(w.d, visible_pairs(B, H, w.N, w.causal))
+
+
+def cpu_baseline(w):
+    import oracle
+    oracle.build()
+    reps, secs, flops = 0, 0.0, 0.0
+    while secs < 10.0 and reps < 20:  # about 10-30 s of CPU work
+        dt, f = oracle_step(w)
+        secs += dt
+        flops += f
+        reps += 1
+    return {"value": round(flops / secs / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"full workload fwd+bwd (fp64 C oracle, OpenMP over heads) x{reps}, {secs:.1f} s"}
+
+
+def run_reference(args):
+    import oracle
+    from exact_io_aware_48_b200 import inputs
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    oracle.build()
+    w = inputs.workloads()["gpt2"]
+    heads = 24  # each step: a quarter of the workload's heads (bounded sample)
+    for _ in range(args.warmup):
+        oracle_step(w, heads)
+    secs, flops = 0.0, 0.0
+    for _ in range(args.steps):
+        dt, f = oracle_step(w, heads)
+        secs += dt
+        flops += f
+    val = flops / secs / 1e12
+    ms = secs / args.steps * 1e3
+    cores = oracle.num_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": round(val, 6), "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "gpt2-small-shaped causal self-attention fwd+bwd B8 H12 N1024 d64 bf16",
+                       "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": True, "global_batch": w.B,
+                       "seq_len": w.N, "parallelism": "host cores (OpenMP)"},
+            "cpu_baseline": {"value": round(val, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{heads} of {w.B * w.H} heads per step, fwd+bwd, fp64"},
+            "e2e": {"value": round(val, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-targets", dest="targets", action="store_false")
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,103 @@
+"""exact_io_aware_48_b200: exact IO-aware attention (FlashAttention-style tiling) for NVIDIA B200 (sm_100a).
+
+The computation lives in libfa.so (hand-written CUDA kernels behind the C ABI of include/fa.h); this package is
+its thin Python face.  ``_lib`` mirrors the C entry points one to one; the helpers below only allocate outputs
+and workspace with torch (device memory and streams), call the library and turn a non-zero status into an
+exception.  There is no CPU or library fallback: without a CUDA device and a loadable libfa.so every call raises.
+"""
+from __future__ import annotations
+
+import math
+
+from . import _lib
+from ._lib import (FA_BF16, FA_FP16, FA_OK, FA_ERR_CUDA, FA_ERR_INVALID_ARG, FA_ERR_TIMEOUT, FA_ERR_UNSUPPORTED,
+                   FA_ERR_WORKSPACE)
+
+__all__ = ["attention_fwd", "attention_bwd", "blockmask_lists", "FAError", "FA_BF16", "FA_FP16"]
+
+
+class FAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        detail = _lib.fa_last_error_string() if status == FA_ERR_CUDA else ""
+        super().__init__(f"{where}: {_lib.fa_status_string(status)}{(' (' + detail + ')') if detail else ''}")
+        self.status = status
+
+
+def _check(rc: int, where: str):
+    if rc != FA_OK:
+        raise FAError(rc, where)
+
+
+def _dtype_code(t):
+    import torch
+    if t.dtype == torch.bfloat16:
+        return FA_BF16
+    if t.dtype == torch.float16:
+        return FA_FP16
+    raise TypeError(f"q/k/v must be bfloat16 or float16, got {t.dtype}")
+
+
+def _require_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise RuntimeError("exact_io_aware_48_b200 runs on CUDA tensors only (no CPU fallback)")
+
+
+def attention_fwd(q, k, v, causal=False, softmax_scale=None, key_lens=None, block_mask=None, stream=None):
+    """O, LSE = exact attention of [B, H, N, d] CUDA tensors (bf16 or fp16).
+
+    key_lens: optional int32 CUDA tensor [B]; block_mask: optional uint8 CUDA tensor [nT, nT] (128x128 tiles).
+    Returns O (same dtype) and LSE (fp32, natural log) [B, H, N].
+    """
+    import torch
+    _require_cuda(q, k, v, key_lens, block_mask)
+    B, H, N, d = q.shape
+    scale = softmax_scale if softmax_scale is not None else 1.0 / math.sqrt(d)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), device=q.device, dtype=torch.float32)
+    dt = _dtype_code(q)
+    if block_mask is None:
+        _check(_lib.fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, key_lens, dt, stream), "fa_fwd")
+    else:
+        ws_bytes = _lib.fa_blocksparse_workspace_size(N)
+        ws = torch.empty(ws_bytes, device=q.device, dtype=torch.uint8)
+        _check(_lib.fa_fwd_blocksparse(q, k, v, o, lse, B, H, N, d, scale, causal, key_lens, block_mask, ws,
+                                       ws_bytes, dt, stream), "fa_fwd_blocksparse")
+    return o, lse
+
+
+def attention_bwd(q, k, v, o, dout, lse, causal=False, softmax_scale=None, key_lens=None, block_mask=None,
+                  stream=None):
+    """dQ, dK, dV of sum(O * dout) for the attention computed by attention_fwd with the same arguments."""
+    import torch
+    _require_cuda(q, k, v, o, dout, lse, key_lens, block_mask)
+    B, H, N, d = q.shape
+    scale = softmax_scale if softmax_scale is not None else 1.0 / math.sqrt(d)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws_bytes = _lib.fa_bwd_workspace_size(B, H, N, d, block_mask is not None)
+    ws = torch.empty(ws_bytes, device=q.device, dtype=torch.uint8)
+    _check(_lib.fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, causal, key_lens, block_mask, ws,
+                       ws_bytes, _dtype_code(q), stream), "fa_bwd")
+    return dq, dk, dv
+
+
+def blockmask_lists(mask, stream=None):
+    """Device CSR/CSC lists of a [nT, nT] uint8 CUDA mask: (row_ptr, col_idx, col_ptr, row_idx), int32, with
+    col_idx/row_idx cut to the number of kept tiles."""
+    import torch
+    _require_cuda(mask)
+    nT = mask.shape[0]
+    dev = mask.device
+    row_ptr = torch.empty(nT + 1, device=dev, dtype=torch.int32)
+    col_ptr = torch.empty(nT + 1, device=dev, dtype=torch.int32)
+    col_idx = torch.empty(nT * nT, device=dev, dtype=torch.int32)
+    row_idx = torch.empty(nT * nT, device=dev, dtype=torch.int32)
+    _check(_lib.fa_blockmask_lists(mask.contiguous(), nT, row_ptr, col_idx, col_ptr, row_idx, stream),
+           "fa_blockmask_lists")
+    nnz = int(row_ptr[-1].item())
+    return row_ptr, col_idx[:nnz], col_ptr, row_idx[:nnz]
+
+
+def last_device_status(stream=None) -> int:
+    """Synchronise and return (then clear) the device status word: FA_OK or FA_ERR_TIMEOUT."""
+    return _lib.fa_last_device_status(stream)

@@ -1,0 +1,138 @@
+"""ctypes binding of libfa.so: one Python function per C entry point, with the same names and arguments.
+
+Argument marshalling only: pointers may be given as ints or as torch tensors (their data_ptr() is passed), the
+stream as an int handle, a torch.cuda.Stream or None (current torch stream).  Every step of the computation runs
+in the library's CUDA kernels; there is no fallback.  If libfa.so is missing or cannot be loaded, every call
+raises RuntimeError.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfa.so")
+
+FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT, FA_ERR_WORKSPACE = range(6)
+FA_BF16, FA_FP16 = 0, 1
+
+# C signatures, exactly as declared in include/fa.h
+_P, _I, _F, _SZ, _U64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_uint64
+SIGNATURES = {
+    "fa_version": ([], _I),
+    "fa_status_string": ([_I], ctypes.c_char_p),
+    "fa_last_error_string": ([], ctypes.c_char_p),
+    "fa_fwd": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P, _I, _P], _I),
+    "fa_blocksparse_workspace_size": ([_I], _SZ),
+    "fa_fwd_blocksparse": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P, _P, _P, _SZ, _I, _P], _I),
+    "fa_bwd_workspace_size": ([_I, _I, _I, _I, _I], _SZ),
+    "fa_bwd": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P, _P, _P, _SZ, _I, _P], _I),
+    "fa_blockmask_lists": ([_P, _I, _P, _P, _P, _P, _P], _I),
+    "fa_last_device_status": ([_P], _I),
+    "fa_set_wait_budget_ns": ([_U64], _I),
+    "fa_selftest_wait_timeout": ([_U64, _P], _I),
+    "fa_set_kernel_events": ([_I, _P, _P], _I),
+}
+FA_KERNEL_FWD, FA_KERNEL_BWD_MAIN = 0, 1
+
+_lib = None
+
+
+def load(path: str = LIB_PATH):
+    """Load libfa.so once and declare its signatures.  Raises RuntimeError if it cannot be loaded."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise RuntimeError(f"libfa.so not found at {path}: build it with `python -m exact_io_aware_48_b200.build`")
+        try:
+            lib = ctypes.CDLL(path)
+        except OSError as e:  # pragma: no cover - environment dependent
+            raise RuntimeError(f"cannot load libfa.so: {e}") from e
+        for name, (args, res) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = lib
+    return _lib
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(s):
+    if s is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def fa_version() -> int:
+    return load().fa_version()
+
+
+def fa_status_string(status: int) -> str:
+    return load().fa_status_string(status).decode()
+
+
+def fa_last_error_string() -> str:
+    return load().fa_last_error_string().decode()
+
+
+def fa_fwd(q, k, v, o, lse, B, H, N, d, softmax_scale, causal, key_lens, dtype, stream=None) -> int:
+    return load().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, softmax_scale, int(causal),
+                         _ptr(key_lens), dtype, _stream(stream))
+
+
+def fa_blocksparse_workspace_size(N) -> int:
+    return load().fa_blocksparse_workspace_size(N)
+
+
+def fa_fwd_blocksparse(q, k, v, o, lse, B, H, N, d, softmax_scale, causal, key_lens, block_mask, workspace,
+                       workspace_bytes, dtype, stream=None) -> int:
+    return load().fa_fwd_blocksparse(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, softmax_scale,
+                                     int(causal), _ptr(key_lens), _ptr(block_mask), _ptr(workspace),
+                                     workspace_bytes, dtype, _stream(stream))
+
+
+def fa_bwd_workspace_size(B, H, N, d, has_block_mask) -> int:
+    return load().fa_bwd_workspace_size(B, H, N, d, int(bool(has_block_mask)))
+
+
+def fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, softmax_scale, causal, key_lens, block_mask, workspace,
+           workspace_bytes, dtype, stream=None) -> int:
+    return load().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
+                         B, H, N, d, softmax_scale, int(causal), _ptr(key_lens), _ptr(block_mask), _ptr(workspace),
+                         workspace_bytes, dtype, _stream(stream))
+
+
+def fa_blockmask_lists(mask, nT, row_ptr, col_idx, col_ptr, row_idx, stream=None) -> int:
+    return load().fa_blockmask_lists(_ptr(mask), nT, _ptr(row_ptr), _ptr(col_idx), _ptr(col_ptr), _ptr(row_idx),
+                                     _stream(stream))
+
+
+def fa_last_device_status(stream=None) -> int:
+    return load().fa_last_device_status(_stream(stream))
+
+
+def fa_set_wait_budget_ns(budget_ns) -> int:
+    return load().fa_set_wait_budget_ns(int(budget_ns))
+
+
+def fa_selftest_wait_timeout(budget_ns, stream=None) -> int:
+    return load().fa_selftest_wait_timeout(int(budget_ns), _stream(stream))
+
+
+def fa_set_kernel_events(kernel, start_event, stop_event) -> int:
+    """Events are torch.cuda.Event (their cuda_event handle is passed), raw int handles, or None."""
+    def h(e):
+        if e is None:
+            return None
+        return e if isinstance(e, int) else e.cuda_event
+    return load().fa_set_kernel_events(kernel, h(start_event), h(stop_event))

@@ -1,0 +1,574 @@
+// fa_bwd.cuh -- backward kernels: gradients by recomputation from the saved logsumexp (sm_100a).
+//
+// Method (FlashAttention review page, claim C7 / E-recompute: the forward keeps only the softmax normalisation and
+// the backward recomputes attention tiles on chip instead of reading an N x N matrix).  The pages print no backward
+// equations; the reading used is the calculus of softmax attention for the loss sum(O * dO):
+//     P = exp(scale * Q K^T - LSE),  D = rowsum(dO * O),  dV = P^T dO,  dP = dO V^T,  dS = P * (dP - D),
+//     dQ = scale * dS K,  dK = scale * dS^T Q.
+//
+// Three launches:
+//   bwd_pre_kernel   D_r = sum_j dO_rj O_rj (fp32) and LSE in base 2 for every row of a 128-padded row space
+//                    (padded rows and rows with no visible key get +inf, so their recomputed P is exactly 0);
+//                    zeroes the fp32 dQ accumulator.  HBM-bound.
+//   bwd_kernel       one CTA per 128-key tile j of one (b, h); loops over the visible 128-row Q tiles i.
+//                    Five tcgen05 GEMMs per (i, j): S^T = K Q^T and dP^T = V dO^T (recompute), dV += P^T dO (P^T read
+//                    from TMEM), dK += dS^T Q and dQ_i = dS K (dS^T staged in shared memory, used K-major for dK and
+//                    M-major for dQ).  dK, dV accumulate in TMEM for the whole loop; each dQ_i partial is added to
+//                    the fp32 accumulator with vector atomics by a dedicated warpgroup.
+//   bwd_dq_kernel    fp32 dQ accumulator -> 16-bit dQ.  HBM-bound.
+//
+// Roles in bwd_kernel (320 threads): warps 0-3 recompute P^T and dS^T (thread = key row = TMEM lane), warps 4-7
+// drain dQ_i from TMEM into global atomics (thread = query row), warp 8 issues MMAs, warp 9 issues TMA loads.
+// TMEM (512 columns): S^T [0,128) with P^T (16-bit pairs) over its first 64; dP^T [128,256), reused for dQ_i once
+// dP^T has been read; dV [256,256+d); dK [256+d,256+2d).
+#pragma once
+#include "fa_common.cuh"
+
+namespace fa {
+
+template <int D>
+struct BwdCfg {
+  static_assert(D == 64 || D == 128, "head dim");
+  static constexpr int kTileBytes = kTile * D * 2;       // 128 x D 16-bit tile
+  static constexpr int kSlotBytes = kTileBytes + 1024;   // Q or dO tile, plus 128 LSE2 + 128 D floats (Q slots)
+  static constexpr int kSubTiles = D / 64;
+  static constexpr int kNumSlots = D == 128 ? 3 : 6;
+  static constexpr int kDsBytes = kTile * kTile * 2;      // dS^T, 128 keys x 128 queries
+  static constexpr int kSmemBytes = 2 * kTileBytes + kDsBytes + kNumSlots * kSlotBytes + 1024;
+  static constexpr int kThreads = 320;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
+};
+
+// Workspace layout: dq_acc [BH][Npad][D] fp32 | lse2 [BH][Npad] fp32 | Dv [BH][Npad] fp32 (each 256-B aligned)
+inline size_t bwd_workspace_bytes(int BH, int nT, int d) {
+  const size_t npad = (size_t)nT * kTile;
+  auto al = [](size_t x) { return (x + 255) / 256 * 256; };
+  return al((size_t)BH * npad * d * 4) + 2 * al((size_t)BH * npad * 4);
+}
+
+struct BwdArgs {
+  void* dk;
+  void* dv;
+  float* dq_acc;
+  const float* lse2;
+  const float* Dv;
+  const int32_t* key_lens;
+  const int32_t* col_ptr;  // CSC of the block mask (nullptr: dense)
+  const int32_t* row_idx;
+  int H, N, nT, BH;
+  int causal;
+  float scale;       // softmax scale
+  float scale_log2;  // softmax scale * log2(e)
+  uint64_t budget_ns;
+};
+
+// Ascending Q tiles visible to K/V tile j: [i0, nT), or the CSC list of column j cut to i >= i0.
+struct ColTileIter {
+  const int32_t* list;
+  int len, pos, i0, dense_next;
+  bool sparse;
+  __device__ __forceinline__ void init(const int32_t* col_ptr, const int32_t* row_idx, int j, int nT, int first,
+                                       bool visible) {
+    pos = 0;
+    i0 = first;
+    dense_next = first;
+    sparse = col_ptr != nullptr;
+    list = nullptr;
+    len = 0;
+    if (!visible) {
+      sparse = true;  // empty
+      return;
+    }
+    if (sparse) {
+      const int a = col_ptr[j], b = col_ptr[j + 1];
+      list = row_idx + a;
+      len = b - a;
+      while (pos < len && list[pos] < first) ++pos;  // ascending
+    } else {
+      len = nT;
+    }
+  }
+  __device__ __forceinline__ bool next(int& i) {
+    if (sparse) {
+      if (pos >= len) return false;
+      i = list[pos++];
+      return true;
+    }
+    if (dense_next >= len) return false;
+    i = dense_next++;
+    return true;
+  }
+  __device__ __forceinline__ int count() const { return sparse ? len - pos : len - dense_next; }
+};
+
+// ------------------------------------------------------------------------------------------------ preprocess
+template <int D, bool kBF16>
+__global__ void __launch_bounds__(256) bwd_pre_kernel(const void* __restrict__ o, const void* __restrict__ dout,
+                                                      const float* __restrict__ lse, float* __restrict__ dq_acc,
+                                                      float* __restrict__ lse2, float* __restrict__ Dv, int N,
+                                                      int Npad, long long rows) {
+  // one warp per padded row
+  const long long row = (long long)blockIdx.x * 8 + threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  if (row >= rows) return;
+  const long long bh = row / Npad;
+  const int r = (int)(row % Npad);
+  float4* acc = reinterpret_cast<float4*>(dq_acc + row * D);
+  for (int c = lane; c < D / 4; c += 32) acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+  float dsum = 0.f;
+  if (r < N) {
+    const size_t off = ((size_t)bh * N + r) * D;
+    constexpr int kPer = D / 32;  // elements per lane: 2 or 4
+    const uint16_t* po = reinterpret_cast<const uint16_t*>(o) + off + lane * kPer;
+    const uint16_t* pd = reinterpret_cast<const uint16_t*>(dout) + off + lane * kPer;
+    uint32_t vo[kPer / 2], vd[kPer / 2];
+    if constexpr (kPer == 4) {
+      const uint2 a = *reinterpret_cast<const uint2*>(po), b = *reinterpret_cast<const uint2*>(pd);
+      vo[0] = a.x; vo[1] = a.y; vd[0] = b.x; vd[1] = b.y;
+    } else {
+      vo[0] = *reinterpret_cast<const uint32_t*>(po);
+      vd[0] = *reinterpret_cast<const uint32_t*>(pd);
+    }
+#pragma unroll
+    for (int u = 0; u < kPer / 2; ++u) {
+      float o0, o1, d0, d1;
+      if constexpr (kBF16) {
+        o0 = __uint_as_float(vo[u] << 16); o1 = __uint_as_float(vo[u] & 0xffff0000u);
+        d0 = __uint_as_float(vd[u] << 16); d1 = __uint_as_float(vd[u] & 0xffff0000u);
+      } else {
+        o0 = __half2float(__ushort_as_half((unsigned short)(vo[u] & 0xffff)));
+        o1 = __half2float(__ushort_as_half((unsigned short)(vo[u] >> 16)));
+        d0 = __half2float(__ushort_as_half((unsigned short)(vd[u] & 0xffff)));
+        d1 = __half2float(__ushort_as_half((unsigned short)(vd[u] >> 16)));
+      }
+      dsum = fmaf(o0, d0, dsum);
+      dsum = fmaf(o1, d1, dsum);
+    }
+  }
+#pragma unroll
+  for (int m = 16; m > 0; m >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, m);
+  if (lane == 0) {
+    float l2 = INFINITY;  // padded row or no visible key: recomputed P = exp2(x - inf) = 0
+    if (r < N) {
+      const float l = lse[(size_t)bh * N + r];
+      if (l != -INFINITY) l2 = l * 1.4426950408889634f;
+    }
+    lse2[row] = l2;
+    Dv[row] = dsum;
+  }
+}
+
+// ------------------------------------------------------------------------------------------------ dQ convert
+template <int D, bool kBF16>
+__global__ void __launch_bounds__(256) bwd_dq_kernel(const float* __restrict__ dq_acc, void* __restrict__ dq, int N,
+                                                     int Npad, long long total_vec4) {
+  // each thread converts 4 consecutive elements of the N-row (unpadded) output
+  for (long long v = (long long)blockIdx.x * blockDim.x + threadIdx.x; v < total_vec4;
+       v += (long long)gridDim.x * blockDim.x) {
+    const long long e = v * 4;
+    const long long row = e / D;  // bh * N + r
+    const int c = (int)(e % D);
+    const long long bh = row / N;
+    const int r = (int)(row % N);
+    const float4 a = *reinterpret_cast<const float4*>(dq_acc + ((size_t)bh * Npad + r) * D + c);
+    uint2 out;
+    out.x = ptx::pack2<kBF16>(a.x, a.y);
+    out.y = ptx::pack2<kBF16>(a.z, a.w);
+    *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(dq) + e) = out;
+  }
+}
+
+// ------------------------------------------------------------------------------------------------ main kernel
+template <int D, bool kBF16>
+__global__ void __launch_bounds__(320, 1)
+    bwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+               const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_do,
+               const BwdArgs args) {
+  using C = BwdCfg<D>;
+  constexpr int NS = C::kNumSlots;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sK = smem;
+  uint8_t* sV = smem + C::kTileBytes;
+  uint8_t* sDS = smem + 2 * C::kTileBytes;
+  uint8_t* sRing = sDS + C::kDsBytes;
+
+  __shared__ __align__(8) uint64_t bar_kv, bar_full[NS], bar_empty[NS], bar_s, bar_dp, bar_p, bar_ds, bar_dq_full,
+      bar_dq_free, bar_ds_free, bar_done, bar_drain;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_flag;
+  volatile int* abortp = &abort_flag;
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int L = blockIdx.x;
+  const int j = L / args.BH;  // K/V tile; ascending j = longest causal work first
+  const int bh = L % args.BH;
+  const int b = bh / args.H;
+  const bool causal = args.causal != 0;
+  const int kv_lim = key_limit(args.key_lens, b, args.N);
+  const bool visible = j * kTile < kv_lim;  // some key of this tile is visible to someone
+  const int Npad = args.nT * kTile;
+
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(ptx::smem_addr(&bar_kv), 1);
+    for (int s = 0; s < NS; ++s) {
+      ptx::mbar_init(ptx::smem_addr(&bar_full[s]), 1);
+      ptx::mbar_init(ptx::smem_addr(&bar_empty[s]), 1);
+    }
+    ptx::mbar_init(ptx::smem_addr(&bar_s), 1);
+    ptx::mbar_init(ptx::smem_addr(&bar_dp), 1);
+    ptx::mbar_init(ptx::smem_addr(&bar_p), 128);
+    ptx::mbar_init(ptx::smem_addr(&bar_ds), 128);
+    ptx::mbar_init(ptx::smem_addr(&bar_dq_full), 1);
+    ptx::mbar_init(ptx::smem_addr(&bar_dq_free), 128);
+    ptx::mbar_init(ptx::smem_addr(&bar_ds_free), 1);
+    ptx::mbar_init(ptx::smem_addr(&bar_done), 1);
+    ptx::mbar_init(ptx::smem_addr(&bar_drain), 1);
+    abort_flag = 0;
+    ptx::fence_barrier_init();
+  }
+  if (warp == 8) {
+    ptx::tmem_alloc(ptx::smem_addr(&tmem_base_sh), C::kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+
+  ColTileIter it;
+  it.init(args.col_ptr, args.row_idx, j, args.nT, causal ? j : 0, visible);
+  const int n_iters = it.count();
+
+  if (warp == 9) {
+    // ------------------------------------------------------------------------------------------ TMA producer
+    if (lane == 0 && n_iters > 0) {
+      ptx::prefetch_tensormap(&map_q);
+      ptx::prefetch_tensormap(&map_do);
+      const uint32_t bkv = ptx::smem_addr(&bar_kv);
+      ptx::mbar_arrive_expect_tx(bkv, 2 * C::kTileBytes);
+      for (int c = 0; c < C::kSubTiles; ++c) {
+        ptx::tma_load_3d(ptx::smem_addr(sK + c * 16384), &map_k, 64 * c, j * kTile, bh, bkv);
+        ptx::tma_load_3d(ptx::smem_addr(sV + c * 16384), &map_v, 64 * c, j * kTile, bh, bkv);
+      }
+      int n = 0, i;
+      bool ok = true;
+      while (ok && it.next(i)) {
+        for (int u = 0; u < 2; ++u) {  // u = 0: Q_i (+ LSE2, D rows), u = 1: dO_i
+          const int s = n % NS;
+          const uint32_t ph = (n / NS) & 1;
+          if (!wait_or_abort(ptx::smem_addr(&bar_empty[s]), ph ^ 1, args.budget_ns, abortp)) { ok = false; break; }
+          const uint32_t bf = ptx::smem_addr(&bar_full[s]);
+          uint8_t* slot = sRing + s * C::kSlotBytes;
+          ptx::mbar_arrive_expect_tx(bf, C::kTileBytes + (u == 0 ? 1024 : 0));
+          for (int c = 0; c < C::kSubTiles; ++c)
+            ptx::tma_load_3d(ptx::smem_addr(slot + c * 16384), u == 0 ? &map_q : &map_do, 64 * c, i * kTile, bh, bf);
+          if (u == 0) {
+            const size_t row0 = (size_t)bh * Npad + (size_t)i * kTile;
+            ptx::bulk_load(ptx::smem_addr(slot + C::kTileBytes), args.lse2 + row0, 512, bf);
+            ptx::bulk_load(ptx::smem_addr(slot + C::kTileBytes + 512), args.Dv + row0, 512, bf);
+          }
+          ++n;
+        }
+      }
+      ptx::mbar_wait(bkv, 0, args.budget_ns);
+      for (int k = (n > NS ? n - NS : 0); k < n; ++k)
+        ptx::mbar_wait(ptx::smem_addr(&bar_full[k % NS]), (k / NS) & 1, args.budget_ns);
+    }
+  } else if (warp == 8) {
+    // ------------------------------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t id_sq = ptx::idesc_f16(kBF16, false, false, 128, 128);  // S^T, dP^T
+      constexpr uint32_t id_dv = ptx::idesc_f16(kBF16, false, true, 128, D);     // dV (A from TMEM), dK
+      constexpr uint32_t id_dq = ptx::idesc_f16(kBF16, true, true, 128, D);      // dQ
+      const uint32_t k_base = ptx::smem_addr(sK), v_base = ptx::smem_addr(sV), ds_base = ptx::smem_addr(sDS);
+      const uint32_t ring = ptx::smem_addr(sRing);
+      bool ok = true;
+      if (n_iters > 0) {
+        ok = wait_or_abort(ptx::smem_addr(&bar_kv), 0, args.budget_ns, abortp);
+        ptx::tc_fence_after();
+      }
+      int n = 0, iter = 0, i;
+      while (ok && it.next(i)) {
+        const int sq = n % NS;
+        const uint32_t phq = (n / NS) & 1;
+        ++n;
+        const int so = n % NS;
+        const uint32_t pho = (n / NS) & 1;
+        ++n;
+        const uint32_t q_base = ring + sq * C::kSlotBytes, do_base = ring + so * C::kSlotBytes;
+        const uint32_t ph = iter & 1, ph_prev = (iter - 1) & 1;
+        // S^T = K Q_i^T
+        if (!(ok = wait_or_abort(ptx::smem_addr(&bar_full[sq]), phq, args.budget_ns, abortp))) break;
+        ptx::tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * 16384 + (kk % 4) * 32;
+          ptx::mma_ss(tmem + C::kColS, ptx::sw128_desc(k_base + off, 16, 1024),
+                      ptx::sw128_desc(q_base + off, 16, 1024), id_sq, kk > 0 ? 1u : 0u);
+        }
+        ptx::mma_commit(ptx::smem_addr(&bar_s));
+        // dP^T = V dO_i^T (its TMEM columns hold dQ_{i-1} until the dQ warps have drained it)
+        if (!(ok = wait_or_abort(ptx::smem_addr(&bar_full[so]), pho, args.budget_ns, abortp))) break;
+        if (iter > 0 && !(ok = wait_or_abort(ptx::smem_addr(&bar_dq_free), ph_prev, args.budget_ns, abortp))) break;
+        ptx::tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * 16384 + (kk % 4) * 32;
+          ptx::mma_ss(tmem + C::kColDP, ptx::sw128_desc(v_base + off, 16, 1024),
+                      ptx::sw128_desc(do_base + off, 16, 1024), id_sq, kk > 0 ? 1u : 0u);
+        }
+        ptx::mma_commit(ptx::smem_addr(&bar_dp));
+        // dV += P^T dO_i   (P^T from TMEM; dO_i M/N-major)
+        if (!(ok = wait_or_abort(ptx::smem_addr(&bar_p), ph, args.budget_ns, abortp))) break;
+        ptx::tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          ptx::mma_ts(tmem + C::kColDV, tmem + C::kColS + kk * 8, ptx::sw128_desc(do_base + kk * 2048, 16384, 1024),
+                      id_dv, (iter > 0 || kk > 0) ? 1u : 0u);
+        ptx::mma_commit(ptx::smem_addr(&bar_empty[so]));  // dO_i no longer needed
+        // dK += dS^T Q_i and dQ_i = dS K_j  (dS^T in shared memory)
+        if (!(ok = wait_or_abort(ptx::smem_addr(&bar_ds), ph, args.budget_ns, abortp))) break;
+        ptx::tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk) {
+          const uint32_t off = (kk / 4) * 16384 + (kk % 4) * 32;
+          ptx::mma_ss(tmem + C::kColDK, ptx::sw128_desc(ds_base + off, 16, 1024),
+                      ptx::sw128_desc(q_base + kk * 2048, 16384, 1024), id_dv, (iter > 0 || kk > 0) ? 1u : 0u);
+        }
+        ptx::mma_commit(ptx::smem_addr(&bar_empty[sq]));  // Q_i (and its LSE2/D rows) no longer needed
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          ptx::mma_ss(tmem + C::kColDP, ptx::sw128_desc(ds_base + kk * 2048, 16384, 1024),
+                      ptx::sw128_desc(k_base + kk * 2048, 16384, 1024), id_dq, kk > 0 ? 1u : 0u);
+        ptx::mma_commit(ptx::smem_addr(&bar_dq_full));
+        ptx::mma_commit(ptx::smem_addr(&bar_ds_free));
+        ++iter;
+      }
+      if (ok) ptx::mma_commit(ptx::smem_addr(&bar_done));
+      ptx::mma_commit(ptx::smem_addr(&bar_drain));
+      ptx::mbar_wait(ptx::smem_addr(&bar_drain), 0, args.budget_ns);
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------------------------------------------------------ P^T / dS^T warps
+    const int c = warp * 32 + lane;            // key row within the tile == TMEM lane
+    const int gc = j * kTile + c;              // key index in the sequence
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const float sl2 = args.scale_log2, sc = args.scale;
+    int n = 0, iter = 0, i;
+    bool ok = true;
+    while (it.next(i)) {
+      const int sq = n % NS;
+      const uint32_t phq = (n / NS) & 1;
+      n += 2;
+      const float* lse2 = reinterpret_cast<const float*>(sRing + sq * C::kSlotBytes + C::kTileBytes);
+      const float* Drow = lse2 + 128;
+      const uint32_t ph = iter & 1;
+      // the LSE2/D rows came in by bulk copy with Q_i: observe that copy's barrier before reading them (the slot
+      // cannot be refilled before this iteration's dS^T is published, so the phase is stable)
+      ok = __all_sync(0xffffffffu, wait_or_abort(ptx::smem_addr(&bar_full[sq]), phq, args.budget_ns, abortp));
+      if (ok) ok = __all_sync(0xffffffffu, wait_or_abort(ptx::smem_addr(&bar_s), ph, args.budget_ns, abortp));
+      if (!ok) break;
+      ptx::tc_fence_after();
+      const bool masked = (causal && i == j) || (j + 1) * kTile > kv_lim;
+      // visible queries of key gc: r >= gc (causal) and the key itself below the key limit
+      const int rmin = causal ? gc - i * kTile : 0;   // first visible query column within the tile
+      const bool key_ok = gc < kv_lim;
+      uint32_t pk[64];
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t sr[32];
+        ptx::tmem_ld32(tmem + lane_base + C::kColS + ch * 32, sr);
+        ptx::tmem_ld_wait();
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int r0 = ch * 32 + 2 * u;
+          float p0 = ptx::ex2(fmaf(__uint_as_float(sr[2 * u]), sl2, -lse2[r0]));
+          float p1 = ptx::ex2(fmaf(__uint_as_float(sr[2 * u + 1]), sl2, -lse2[r0 + 1]));
+          if (masked) {
+            if (!key_ok || r0 < rmin) p0 = 0.f;
+            if (!key_ok || r0 + 1 < rmin) p1 = 0.f;
+          }
+          pk[ch * 16 + u] = ptx::pack2<kBF16>(p0, p1);
+        }
+      }
+      ptx::tmem_st32(tmem + lane_base + C::kColS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+      ptx::tmem_st32(tmem + lane_base + C::kColS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+      ptx::tmem_st_wait();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(ptx::smem_addr(&bar_p));
+      // dS^T = P^T * (dP^T - D) * scale, written 16-bit into the swizzled dS^T tile
+      ok = __all_sync(0xffffffffu, wait_or_abort(ptx::smem_addr(&bar_dp), ph, args.budget_ns, abortp));
+      if (ok && iter > 0)
+        ok = __all_sync(0xffffffffu, wait_or_abort(ptx::smem_addr(&bar_ds_free), (iter - 1) & 1, args.budget_ns,
+                                                    abortp));
+      if (!ok) break;
+      ptx::tc_fence_after();
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t dr[32];
+        ptx::tmem_ld32(tmem + lane_base + C::kColDP + ch * 32, dr);
+        ptx::tmem_ld_wait();
+        uint32_t o[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int r0 = ch * 32 + 2 * u;
+          float p0, p1;
+          if constexpr (kBF16) {
+            p0 = __uint_as_float(pk[ch * 16 + u] << 16);
+            p1 = __uint_as_float(pk[ch * 16 + u] & 0xffff0000u);
+          } else {
+            p0 = __half2float(__ushort_as_half((unsigned short)(pk[ch * 16 + u] & 0xffff)));
+            p1 = __half2float(__ushort_as_half((unsigned short)(pk[ch * 16 + u] >> 16)));
+          }
+          const float ds0 = p0 * (__uint_as_float(dr[2 * u]) - Drow[r0]) * sc;
+          const float ds1 = p1 * (__uint_as_float(dr[2 * u + 1]) - Drow[r0 + 1]) * sc;
+          o[u] = ptx::pack2<kBF16>(ds0, ds1);
+        }
+        // queries ch*32 .. ch*32+31 live in sub-tile ch/2, 16-byte chunks (ch%2)*4 .. +3 of row c (swizzled)
+        uint8_t* rowp = sDS + (ch / 2) * 16384 + c * 128;
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const int chunk = ((ch % 2) * 4 + v) ^ (c & 7);
+          *reinterpret_cast<uint4*>(rowp + chunk * 16) = make_uint4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+        }
+      }
+      ptx::fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(ptx::smem_addr(&bar_ds));
+      ++iter;
+    }
+    // ------------------------------------------------------------------------------------------ dK, dV epilogue
+    if (ok && n_iters > 0)
+      ok = __all_sync(0xffffffffu, wait_or_abort(ptx::smem_addr(&bar_done), 0, args.budget_ns, abortp));
+    if (ok) {
+      ptx::tc_fence_after();
+      const bool row_ok = gc < args.N;
+      const size_t off = ((size_t)bh * args.N + gc) * D * 2;
+#pragma unroll 1
+      for (int which = 0; which < 2; ++which) {
+        uint8_t* dst_row = reinterpret_cast<uint8_t*>(which == 0 ? args.dv : args.dk) + off;
+        const uint32_t col = which == 0 ? C::kColDV : C::kColDK;
+#pragma unroll 1
+        for (int ch = 0; ch < D / 32; ++ch) {
+          uint32_t r[32];
+          if (n_iters > 0) {
+            ptx::tmem_ld32(tmem + lane_base + col + ch * 32, r);
+            ptx::tmem_ld_wait();
+          } else {
+#pragma unroll
+            for (int u = 0; u < 32; ++u) r[u] = 0u;  // no visible query: zero gradient
+          }
+          uint32_t pkd[16];
+#pragma unroll
+          for (int u = 0; u < 16; ++u) pkd[u] = ptx::pack2<kBF16>(__uint_as_float(r[2 * u]), __uint_as_float(r[2 * u + 1]));
+          if (row_ok) {
+            uint4* dst = reinterpret_cast<uint4*>(dst_row + ch * 64);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pkd[4 * v], pkd[4 * v + 1], pkd[4 * v + 2], pkd[4 * v + 3]);
+          }
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------------------------------ dQ drain warps
+    const int q = (warp - 4) * 32 + lane;  // query row within the tile == TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>((warp - 4) * 32) << 16;
+    int iter = 0, i;
+    while (it.next(i)) {
+      const bool ok = __all_sync(0xffffffffu, wait_or_abort(ptx::smem_addr(&bar_dq_full), iter & 1, args.budget_ns,
+                                                            abortp));
+      if (!ok) break;
+      ptx::tc_fence_after();
+      uint32_t r[D];
+#pragma unroll
+      for (int ch = 0; ch < D / 32; ++ch) ptx::tmem_ld32(tmem + lane_base + C::kColDP + ch * 32,
+                                                         *reinterpret_cast<uint32_t(*)[32]>(&r[ch * 32]));
+      ptx::tmem_ld_wait();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(ptx::smem_addr(&bar_dq_free));  // TMEM columns may now be overwritten
+      float4* dst = reinterpret_cast<float4*>(args.dq_acc + ((size_t)bh * Npad + (size_t)i * kTile + q) * D);
+#pragma unroll
+      for (int v = 0; v < D / 4; ++v)
+        atomicAdd(dst + v, make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                       __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3])));
+      ++iter;
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------------------------------------ host side
+template <int D, bool BF>
+cudaError_t launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
+                       const void* o, const void* dout, const float* lse, void* dq, const BwdArgs& a,
+                       cudaStream_t st, cudaEvent_t ev_start, cudaEvent_t ev_stop) {
+  using C = BwdCfg<D>;
+  const int Npad = a.nT * kTile;
+  const long long rows = (long long)a.BH * Npad;
+  bwd_pre_kernel<D, BF><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(o, dout, lse, a.dq_acc,
+                                                                     const_cast<float*>(a.lse2),
+                                                                     const_cast<float*>(a.Dv), a.N, Npad, rows);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  static std::atomic<uint64_t> smem_set{0};
+  int dev = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if (!(smem_set.load() & (1ull << (dev & 63)))) {
+    e = cudaFuncSetAttribute(bwd_kernel<D, BF>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    smem_set.fetch_or(1ull << (dev & 63));
+  }
+  if (ev_start && (e = cudaEventRecord(ev_start, st)) != cudaSuccess) return e;
+  bwd_kernel<D, BF><<<(unsigned)(a.nT * a.BH), C::kThreads, C::kSmemBytes, st>>>(mq, mk, mv, mdo, a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (ev_stop && (e = cudaEventRecord(ev_stop, st)) != cudaSuccess) return e;
+  const long long total_vec4 = (long long)a.BH * a.N * D / 4;
+  const unsigned blocks = (unsigned)std::min<long long>((total_vec4 + 255) / 256, 148LL * 16);
+  bwd_dq_kernel<D, BF><<<blocks, 256, 0, st>>>(a.dq_acc, dq, a.N, Npad, total_vec4);
+  return cudaGetLastError();
+}
+
+inline cudaError_t run_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                           const CUtensorMap& mdo, const void* o, const void* dout, const float* lse, void* dq,
+                           void* dk, void* dv, int B, int H, int N, int d, float scale, bool causal,
+                           const int32_t* key_lens, const int32_t* col_ptr, const int32_t* row_idx, void* workspace,
+                           bool bf16, uint64_t budget_ns, cudaStream_t st, cudaEvent_t ev_start,
+                           cudaEvent_t ev_stop) {
+  const int nT = (N + kTile - 1) / kTile;
+  const int BH = B * H;
+  const size_t npad = (size_t)nT * kTile;
+  auto al = [](size_t x) { return (x + 255) / 256 * 256; };
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  BwdArgs a;
+  a.dk = dk;
+  a.dv = dv;
+  a.dq_acc = reinterpret_cast<float*>(ws);
+  a.lse2 = reinterpret_cast<const float*>(ws + al((size_t)BH * npad * d * 4));
+  a.Dv = reinterpret_cast<const float*>(ws + al((size_t)BH * npad * d * 4) + al((size_t)BH * npad * 4));
+  a.key_lens = key_lens;
+  a.col_ptr = col_ptr;
+  a.row_idx = row_idx;
+  a.H = H;
+  a.N = N;
+  a.nT = nT;
+  a.BH = BH;
+  a.causal = causal ? 1 : 0;
+  a.scale = scale;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.budget_ns = budget_ns;
+  if (d == 64)
+    return bf16 ? launch_bwd<64, true>(mq, mk, mv, mdo, o, dout, lse, dq, a, st, ev_start, ev_stop)
+                : launch_bwd<64, false>(mq, mk, mv, mdo, o, dout, lse, dq, a, st, ev_start, ev_stop);
+  return bf16 ? launch_bwd<128, true>(mq, mk, mv, mdo, o, dout, lse, dq, a, st, ev_start, ev_stop)
+              : launch_bwd<128, false>(mq, mk, mv, mdo, o, dout, lse, dq, a, st, ev_start, ev_stop);
+}
+
+}  // namespace fa

@@ -1,0 +1,115 @@
+// fa_common.cuh -- pieces shared by the forward and backward kernels: the device status word, tile geometry,
+// and the per-tile visibility rules (causal, key lengths, block-mask lists) applied at tile granularity.
+#pragma once
+#include <algorithm>
+#include <atomic>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include "ptx.cuh"
+
+namespace fa {
+
+constexpr int kTile = 128;  // rows of a Q tile and keys of a K/V tile
+
+enum DeviceError : int { kDevOk = 0, kDevTimeout = 4 };
+
+// One status word per device; the first error wins.  Read and cleared by fa_last_device_status().
+__device__ int g_device_status = 0;
+
+__device__ __forceinline__ void record_error(int code) { atomicCAS(&g_device_status, 0, code); }
+
+// Bounded wait used by every pipeline role.  Gives up when the CTA's abort flag is raised by another role, or
+// after `budget_ns` (then it records FA_ERR_TIMEOUT in the status word and raises the abort flag itself).
+__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, uint64_t budget_ns,
+                                              volatile int* abort_flag) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 16; ++i)
+      if (ptx::mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (ptx::globaltimer_ns() - t0 > budget_ns) {
+      record_error(kDevTimeout);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+
+// Number of keys visible to sequence b at all (key length clamped to N).
+__device__ __forceinline__ int key_limit(const int32_t* key_lens, int b, int N) {
+  if (key_lens == nullptr) return N;
+  int l = key_lens[b];
+  return l < 0 ? 0 : (l > N ? N : l);
+}
+
+// Exclusive end of the K/V tiles query tile i may see: tiles at or beyond it are fully hidden by the key
+// limit or (causal) lie entirely above the diagonal.
+__device__ __forceinline__ int kv_tile_end(int i, int kv_lim, bool causal) {
+  int end = (kv_lim + kTile - 1) / kTile;
+  if (causal && end > i + 1) end = i + 1;
+  return end;
+}
+
+// Iterates, in ascending order, the K/V tiles visible to either of the two Q tiles a forward CTA owns.  Every
+// role (loader, MMA issuer, softmax warps) walks the same sequence, so their pipelines stay in step.
+//   dense : tile t sees [0, end_t)
+//   sparse: tile t sees the ascending CSR list of its row, cut at end_t
+struct PairTileIter {
+  const int32_t* list[2];
+  int len[2];   // dense: end_t; sparse: entries in list (already cut to < end_t)
+  int pos[2];
+  bool sparse;
+  int next_dense;
+
+  __device__ __forceinline__ void init_dense(int end0, int end1) {
+    sparse = false;
+    len[0] = end0; len[1] = end1;
+    pos[0] = pos[1] = 0;
+    next_dense = 0;
+    list[0] = list[1] = nullptr;
+  }
+
+  __device__ __forceinline__ void init_sparse(const int32_t* row_ptr, const int32_t* col_idx, int row0, int nT,
+                                              int end0, int end1) {
+    sparse = true;
+    next_dense = 0;
+    for (int t = 0; t < 2; ++t) {
+      const int r = row0 + t;
+      pos[t] = 0;
+      if (r >= nT) { list[t] = col_idx; len[t] = 0; continue; }
+      const int a = row_ptr[r], b = row_ptr[r + 1];
+      list[t] = col_idx + a;
+      const int end = t == 0 ? end0 : end1;
+      int n = 0;
+      while (n < b - a && list[t][n] < end) ++n;  // lists are ascending
+      len[t] = n;
+    }
+  }
+
+  // Next visible tile j and a 2-bit mask of the Q tiles that see it.  Returns false when both are exhausted.
+  __device__ __forceinline__ bool next(int& j, int& flags) {
+    if (!sparse) {
+      const int end = len[0] > len[1] ? len[0] : len[1];
+      if (next_dense >= end) return false;
+      j = next_dense++;
+      flags = (j < len[0] ? 1 : 0) | (j < len[1] ? 2 : 0);
+      return true;
+    }
+    const int a = pos[0] < len[0] ? list[0][pos[0]] : 0x7fffffff;
+    const int b = pos[1] < len[1] ? list[1][pos[1]] : 0x7fffffff;
+    if (a == 0x7fffffff && b == 0x7fffffff) return false;
+    j = a < b ? a : b;
+    flags = (a == j ? 1 : 0) | (b == j ? 2 : 0);
+    if (a == j) ++pos[0];
+    if (b == j) ++pos[1];
+    return true;
+  }
+
+  __device__ __forceinline__ int count(int t) const { return len[t]; }
+};
+
+}  // namespace fa

@@ -1,0 +1,353 @@
+// fa_fwd.cuh -- forward kernel: exact attention tile by tile with online softmax on sm_100a.
+//
+// Method (FlashAttention review page, "Method"; explainer page, "online softmax"; slide deck "Executable shape"):
+// Q, K, V are cut into 128-row tiles; K/V tiles stream through shared memory past resident Q tiles; per row the
+// running max m and denominator l are kept on chip and earlier partial outputs are rescaled when m grows; only O
+// and the per-row logsumexp reach HBM.  The slide deck's loop runs K/V outer and Q inner with the state
+// round-tripped per Q block; here the Q tiles stay resident (Q outer) so the state never leaves the chip -- the
+// result is the same (online softmax is order independent in exact arithmetic).
+//
+// B200 mapping (one CTA = two 128-row Q tiles of one (b, h), 320 threads, one CTA per SM):
+//   warp 9      TMA producer: Q tiles once, then K_j, V_j into a ring of shared-memory slots (mbarrier full/empty)
+//   warp 8      MMA issuer (one thread): S_t = Q_t K_j^T into TMEM (fp32), O_t += P_t V_j with P_t read from TMEM
+//   warps 0-3   softmax for Q tile 0, warps 4-7 for Q tile 1: each thread owns one query row (the TMEM 32x32b
+//               access pattern hands a thread a whole row), so row max and row sum need no shuffles.
+// TMEM (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,256+d), O_1 [256+d,256+2d); P_t (16-bit pairs)
+// overwrites the first 64 columns of S_t after they have been read into registers.
+// The two Q tiles ping-pong: while the softmax warps of one tile work, the tensor core runs the other tile's
+// P V and next Q K^T.  Rescaling of O is lazy: a row's reference max only moves when the tile max exceeds it by
+// more than 8 (log2 units), so O is read-modified-written in TMEM rarely; O / l stays exact in real arithmetic
+// because acc and l always share the same reference max.
+#pragma once
+#include "fa_common.cuh"
+
+namespace fa {
+
+template <int D>
+struct FwdCfg {
+  static_assert(D == 64 || D == 128, "head dim");
+  static constexpr int kSlotBytes = kTile * D * 2;  // one 128 x D tile of 16-bit values
+  static constexpr int kSubTiles = D / 64;           // 128-byte-wide column blocks (one TMA box each)
+  static constexpr int kNumSlots = D == 128 ? 4 : 8;
+  static constexpr int kQBytes = 2 * kSlotBytes;
+  static constexpr int kSmemBytes = kQBytes + kNumSlots * kSlotBytes + 1024;
+  static constexpr int kThreads = 320;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kColO = 256;  // O_t at kColO + t * D
+};
+
+struct FwdArgs {
+  void* o;
+  float* lse;
+  const int32_t* key_lens;
+  const int32_t* row_ptr;  // CSR of the block mask (nullptr: dense)
+  const int32_t* col_idx;
+  int H, N, nT, npairs, BH;
+  int causal;
+  float scale_log2;  // softmax_scale * log2(e)
+  uint64_t budget_ns;
+};
+
+template <int D, bool kBF16>
+__global__ void __launch_bounds__(320, 1)
+    fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+               const __grid_constant__ CUtensorMap map_v, const FwdArgs args) {
+  using C = FwdCfg<D>;
+  constexpr int NS = C::kNumSlots;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sKV = smem + C::kQBytes;
+
+  __shared__ __align__(8) uint64_t bar_q, bar_full[NS], bar_empty[NS], bar_s[2], bar_p[2], bar_o[2], bar_drain;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_flag;
+  volatile int* abortp = &abort_flag;
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int L = blockIdx.x;
+  const int pair = args.npairs - 1 - L / args.BH;  // longest (latest) Q tiles first: causal load balance
+  const int bh = L % args.BH;
+  const int b = bh / args.H;
+  const int qt0 = 2 * pair;
+  const bool has1 = qt0 + 1 < args.nT;
+  const bool causal = args.causal != 0;
+  const int kv_lim = key_limit(args.key_lens, b, args.N);
+  const int end0 = kv_tile_end(qt0, kv_lim, causal);
+  const int end1 = has1 ? kv_tile_end(qt0 + 1, kv_lim, causal) : 0;
+
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(ptx::smem_addr(&bar_q), 1);
+    for (int s = 0; s < NS; ++s) {
+      ptx::mbar_init(ptx::smem_addr(&bar_full[s]), 1);
+      ptx::mbar_init(ptx::smem_addr(&bar_empty[s]), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      ptx::mbar_init(ptx::smem_addr(&bar_s[t]), 1);
+      ptx::mbar_init(ptx::smem_addr(&bar_p[t]), 128);
+      ptx::mbar_init(ptx::smem_addr(&bar_o[t]), 1);
+    }
+    ptx::mbar_init(ptx::smem_addr(&bar_drain), 1);
+    abort_flag = 0;
+    ptx::fence_barrier_init();
+  }
+  if (warp == 8) {
+    ptx::tmem_alloc(ptx::smem_addr(&tmem_base_sh), C::kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+
+  PairTileIter it;
+  if (args.row_ptr != nullptr)
+    it.init_sparse(args.row_ptr, args.col_idx, qt0, args.nT, end0, end1);
+  else
+    it.init_dense(end0, end1);
+
+  if (warp == 9) {
+    // ------------------------------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      ptx::prefetch_tensormap(&map_q);
+      ptx::prefetch_tensormap(&map_k);
+      ptx::prefetch_tensormap(&map_v);
+      const uint32_t bq = ptx::smem_addr(&bar_q);
+      ptx::mbar_arrive_expect_tx(bq, (has1 ? 2 : 1) * C::kSlotBytes);
+      for (int t = 0; t < (has1 ? 2 : 1); ++t)
+        for (int c = 0; c < C::kSubTiles; ++c)
+          ptx::tma_load_3d(ptx::smem_addr(sQ + t * C::kSlotBytes + c * 16384), &map_q, 64 * c, (qt0 + t) * kTile,
+                           bh, bq);
+      int n = 0, j, fl;
+      bool ok = true;
+      while (ok && it.next(j, fl)) {
+        for (int kv = 0; kv < 2; ++kv) {
+          const int s = n % NS;
+          const uint32_t ph = (n / NS) & 1;
+          if (!wait_or_abort(ptx::smem_addr(&bar_empty[s]), ph ^ 1, args.budget_ns, abortp)) { ok = false; break; }
+          const uint32_t bf = ptx::smem_addr(&bar_full[s]);
+          ptx::mbar_arrive_expect_tx(bf, C::kSlotBytes);
+          const CUtensorMap* map = kv == 0 ? &map_k : &map_v;
+          for (int c = 0; c < C::kSubTiles; ++c)
+            ptx::tma_load_3d(ptx::smem_addr(sKV + s * C::kSlotBytes + c * 16384), map, 64 * c, j * kTile, bh, bf);
+          ++n;
+        }
+      }
+      // Let every copy this thread issued land before the CTA can exit (immediate in the normal path).
+      ptx::mbar_wait(bq, 0, args.budget_ns);
+      for (int k = (n > NS ? n - NS : 0); k < n; ++k)
+        ptx::mbar_wait(ptx::smem_addr(&bar_full[k % NS]), (k / NS) & 1, args.budget_ns);
+    }
+  } else if (warp == 8) {
+    // ------------------------------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = ptx::idesc_f16(kBF16, false, false, 128, 128);
+      constexpr uint32_t idesc_o = ptx::idesc_f16(kBF16, false, true, 128, D);
+      const uint32_t q_base = ptx::smem_addr(sQ), kv_base = ptx::smem_addr(sKV);
+      bool ok = wait_or_abort(ptx::smem_addr(&bar_q), 0, args.budget_ns, abortp);
+      ptx::tc_fence_after();
+      int n = 0, j, fl;
+      int pend_slot = 0, pend_flags = 0;
+      uint32_t pend_phase = 0;
+      uint32_t p_phase[2] = {0, 0};
+      int pv_count[2] = {0, 0};
+
+      // O_t += P_t V  (A = P_t from TMEM, B = V tile, M/N-major, 128-byte swizzle)
+      auto issue_pv = [&](int t, int slot) {
+        const uint32_t v_base = kv_base + slot * C::kSlotBytes;
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk) {
+          const uint64_t bdesc = ptx::sw128_desc(v_base + kk * 2048, 16384, 1024);
+          ptx::mma_ts(tmem + C::kColO + t * D, tmem + t * 128 + kk * 8, bdesc, idesc_o,
+                      (pv_count[t] > 0 || kk > 0) ? 1u : 0u);
+        }
+        ++pv_count[t];
+      };
+      // S_t = Q_t K^T  (both K-major, 128-byte swizzle, K = D in steps of 16)
+      auto issue_s = [&](int t, int slot) {
+        const uint32_t qa = q_base + t * C::kSlotBytes, kb = kv_base + slot * C::kSlotBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * 16384 + (kk % 4) * 32;
+          ptx::mma_ss(tmem + t * 128, ptx::sw128_desc(qa + off, 16, 1024), ptx::sw128_desc(kb + off, 16, 1024),
+                      idesc_s, kk > 0 ? 1u : 0u);
+        }
+      };
+      // Issue the pending P V of the previous visible tile for tile t (waits for its P).
+      bool v_ready = false;
+      auto flush_pv = [&](int t) -> bool {
+        if (!(pend_flags & (1 << t))) return true;
+        if (!wait_or_abort(ptx::smem_addr(&bar_p[t]), p_phase[t], args.budget_ns, abortp)) return false;
+        p_phase[t] ^= 1;
+        if (!v_ready) {
+          if (!wait_or_abort(ptx::smem_addr(&bar_full[pend_slot]), pend_phase, args.budget_ns, abortp)) return false;
+          v_ready = true;
+        }
+        ptx::tc_fence_after();
+        issue_pv(t, pend_slot);
+        return true;
+      };
+
+      while (ok && it.next(j, fl)) {
+        const int sK = n % NS;
+        const uint32_t phK = (n / NS) & 1;
+        ++n;
+        const int sV = n % NS;
+        const uint32_t phV = (n / NS) & 1;
+        ++n;
+        bool k_ready = false;
+        for (int t = 0; t < 2 && ok; ++t) {
+          ok = flush_pv(t);
+          if (ok && (fl & (1 << t))) {
+            if (!k_ready) {
+              ok = wait_or_abort(ptx::smem_addr(&bar_full[sK]), phK, args.budget_ns, abortp);
+              ptx::tc_fence_after();
+              k_ready = true;
+            }
+            if (ok) {
+              issue_s(t, sK);
+              ptx::mma_commit(ptx::smem_addr(&bar_s[t]));
+            }
+          }
+        }
+        if (!ok) break;
+        if (pend_flags) ptx::mma_commit(ptx::smem_addr(&bar_empty[pend_slot]));  // previous V consumed
+        ptx::mma_commit(ptx::smem_addr(&bar_empty[sK]));                          // this K consumed
+        pend_slot = sV;
+        pend_phase = phV;
+        pend_flags = fl;
+        v_ready = false;
+      }
+      if (ok) {
+        for (int t = 0; t < 2 && ok; ++t) ok = flush_pv(t);
+        if (ok && pend_flags) ptx::mma_commit(ptx::smem_addr(&bar_empty[pend_slot]));
+        if (ok) {
+          ptx::mma_commit(ptx::smem_addr(&bar_o[0]));
+          ptx::mma_commit(ptx::smem_addr(&bar_o[1]));
+        }
+      }
+      // No MMA may still be running when the tensor memory is released.
+      ptx::mma_commit(ptx::smem_addr(&bar_drain));
+      ptx::mbar_wait(ptx::smem_addr(&bar_drain), 0, args.budget_ns);
+    }
+  } else {
+    // ------------------------------------------------------------------------------------------ softmax warps
+    const int t = warp / 4;
+    const int quarter = warp % 4;
+    const int qt = qt0 + t;
+    const int row = quarter * 32 + lane;  // row within the Q tile == TMEM lane
+    const int grow = qt * kTile + row;    // row within the sequence
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_base + t * 128;
+    const uint32_t tO = tmem + lane_base + C::kColO + t * D;
+    const float scale_log2 = args.scale_log2;
+    float m_ref = -INFINITY, l_sum = 0.f;
+    uint32_t s_phase = 0;
+    int kidx = 0;
+    bool ok = true;
+    int j, fl;
+    while (it.next(j, fl)) {
+      if (!(fl & (1 << t))) continue;
+      // every lane waits; the verdict is made warp-uniform before any warp-collective TMEM access
+      ok = __all_sync(0xffffffffu, wait_or_abort(ptx::smem_addr(&bar_s[t]), s_phase, args.budget_ns, abortp));
+      if (!ok) break;
+      s_phase ^= 1;
+      ptx::tc_fence_after();
+      uint32_t sr[128];
+      ptx::tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      ptx::tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      ptx::tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+      ptx::tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+      ptx::tmem_ld_wait();
+      float* s = reinterpret_cast<float*>(sr);
+      // element masks only on tiles that straddle the diagonal or the key limit
+      if ((causal && j >= qt) || (j + 1) * kTile > kv_lim) {
+        const int c0 = j * kTile;
+        const int lim = causal ? min(kv_lim, grow + 1) : kv_lim;  // keys c < lim are visible
+#pragma unroll
+        for (int i = 0; i < 128; ++i)
+          if (c0 + i >= lim) s[i] = -INFINITY;
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int i = 1; i < 128; ++i) mx = fmaxf(mx, s[i]);
+      const float m_tile = mx * scale_log2;
+      const bool need = m_tile > m_ref + 8.0f;
+      float alpha = 1.0f;
+      if (need) {
+        alpha = ptx::ex2(m_ref - m_tile);  // 0 when nothing was visible before
+        m_ref = m_tile;
+      }
+      const float m_use = (m_ref == -INFINITY) ? 0.0f : m_ref;
+      float sum = 0.f;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float p0 = ptx::ex2(fmaf(s[h * 64 + 2 * i], scale_log2, -m_use));
+          const float p1 = ptx::ex2(fmaf(s[h * 64 + 2 * i + 1], scale_log2, -m_use));
+          pk[i] = ptx::pack2<kBF16>(p0, p1);
+          sum += ptx::unpack2_sum<kBF16>(pk[i]);  // l sums the rounded P that P V uses: O stays a convex mix
+        }
+        ptx::tmem_st32(tS + h * 32, pk);
+      }
+      // rescale the running output (only if some row of this warp moved its reference max)
+      if (kidx > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t orr[32];
+          ptx::tmem_ld32(tO + c * 32, orr);
+          ptx::tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) orr[i] = __float_as_uint(__uint_as_float(orr[i]) * alpha);
+          ptx::tmem_st32(tO + c * 32, orr);
+        }
+      }
+      ptx::tmem_st_wait();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(ptx::smem_addr(&bar_p[t]));
+      l_sum = l_sum * alpha + sum;
+      ++kidx;
+    }
+    // ------------------------------------------------------------------------------------------ epilogue
+    if (ok) ok = __all_sync(0xffffffffu, wait_or_abort(ptx::smem_addr(&bar_o[t]), 0, args.budget_ns, abortp));
+    if (ok) {
+      ptx::tc_fence_after();
+      const bool row_ok = grow < args.N && (t == 0 || has1);
+      const bool nonempty = l_sum > 0.f;
+      const float inv = nonempty ? 1.0f / l_sum : 0.0f;
+      uint8_t* orow = reinterpret_cast<uint8_t*>(args.o) + ((size_t)bh * args.N + grow) * D * 2;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t orr[32];
+        ptx::tmem_ld32(tO + c * 32, orr);
+        ptx::tmem_ld_wait();
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float a = nonempty ? __uint_as_float(orr[2 * i]) * inv : 0.0f;
+          const float bb = nonempty ? __uint_as_float(orr[2 * i + 1]) * inv : 0.0f;
+          pk[i] = ptx::pack2<kBF16>(a, bb);
+        }
+        if (row_ok) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 64);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        }
+      }
+      if (row_ok)
+        args.lse[(size_t)bh * args.N + grow] = nonempty ? (m_ref + __log2f(l_sum)) * 0.69314718055994530942f
+                                                        : -INFINITY;
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+}  // namespace fa

@@ -1,0 +1,311 @@
+// fa_lib.cu -- the C ABI declared in include/fa.h: argument checks, TMA tensor maps, kernel launches, status.
+// All kernels live in this one translation unit so they share the per-device status word.
+#include <atomic>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "fa.h"
+#include "fa_common.cuh"
+#include "fa_fwd.cuh"
+#include "fa_bwd.cuh"
+#include "fa_mask.cuh"
+
+namespace {
+
+constexpr int kVersion = 10000;  // 1.0.0
+constexpr int kMaxN = 1 << 20;
+constexpr long long kMaxElems = 1LL << 34;
+
+thread_local std::string t_last_error;
+thread_local cudaEvent_t t_events[2][2] = {{nullptr, nullptr}, {nullptr, nullptr}};  // [kernel][start, stop]
+
+// Records the caller's event (if any) for `kernel` on stream `st`.
+cudaError_t mark(int kernel, int which, cudaStream_t st) {
+  cudaEvent_t e = t_events[kernel][which];
+  return e ? cudaEventRecord(e, st) : cudaSuccess;
+}
+std::atomic<uint64_t> g_budget_ns{2000000000ull};
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+int cuda_fail(cudaError_t e) {
+  t_last_error = cudaGetErrorString(e);
+  return FA_ERR_CUDA;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// Shape/pointer checks shared by every attention entry point.
+int check_common(const void* q, const void* k, const void* v, int B, int H, int N, int d, float scale, int dtype) {
+  if (!q || !k || !v) return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16)) return FA_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || N < 1 || N > kMaxN) return FA_ERR_INVALID_ARG;
+  if (dtype != FA_BF16 && dtype != FA_FP16) return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.0f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if ((long long)B * H * N * d > kMaxElems) return FA_ERR_INVALID_ARG;
+  return FA_OK;
+}
+
+// [B*H, N, d] view of a [B, H, N, d] tensor: rows past N of a head are out of bounds (zero-filled by TMA),
+// so a ragged last tile never reads the next head.  Box: 128 rows x 64 columns (128 bytes), 128-byte swizzle.
+int make_map(CUtensorMap* m, const void* ptr, int BH, int N, int d, int dtype) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) {
+    t_last_error = "cuTensorMapEncodeTiled unavailable";
+    return FA_ERR_CUDA;
+  }
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)N * d * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = enc(m, dtype == FA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+                   const_cast<void*>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    t_last_error = "cuTensorMapEncodeTiled failed with CUresult " + std::to_string((int)r);
+    return FA_ERR_CUDA;
+  }
+  return FA_OK;
+}
+
+// cudaFuncSetAttribute for the dynamic shared memory size, once per (kernel, device).  `done_mask` must be a
+// distinct object per kernel (kernels of identical signature would otherwise share one cache).
+template <typename Kernel>
+cudaError_t ensure_smem(Kernel kernel, int bytes, std::atomic<uint64_t>& done_mask) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = 1ull << (dev & 63);
+  if (done_mask.load() & bit) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done_mask.fetch_or(bit);
+  return e;
+}
+
+template <int D, bool BF>
+cudaError_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const fa::FwdArgs& a,
+                       cudaStream_t st) {
+  using C = fa::FwdCfg<D>;
+  static std::atomic<uint64_t> smem_set{0};
+  cudaError_t e = ensure_smem(fa::fwd_kernel<D, BF>, C::kSmemBytes, smem_set);
+  if (e != cudaSuccess) return e;
+  const unsigned grid = (unsigned)a.BH * (unsigned)a.npairs;
+  if ((e = mark(FA_KERNEL_FWD, 0, st)) != cudaSuccess) return e;
+  fa::fwd_kernel<D, BF><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mk, mv, a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  return mark(FA_KERNEL_FWD, 1, st);
+}
+
+int run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+            float scale, int causal, const int32_t* key_lens, const int32_t* row_ptr, const int32_t* col_idx,
+            int dtype, cudaStream_t st) {
+  CUtensorMap mq, mk, mv;
+  int rc;
+  if ((rc = make_map(&mq, q, B * H, N, d, dtype)) != FA_OK) return rc;
+  if ((rc = make_map(&mk, k, B * H, N, d, dtype)) != FA_OK) return rc;
+  if ((rc = make_map(&mv, v, B * H, N, d, dtype)) != FA_OK) return rc;
+  fa::FwdArgs a;
+  a.o = o;
+  a.lse = lse;
+  a.key_lens = key_lens;
+  a.row_ptr = row_ptr;
+  a.col_idx = col_idx;
+  a.H = H;
+  a.N = N;
+  a.nT = (N + fa::kTile - 1) / fa::kTile;
+  a.npairs = (a.nT + 1) / 2;
+  a.BH = B * H;
+  a.causal = causal ? 1 : 0;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.budget_ns = g_budget_ns.load();
+  cudaError_t e;
+  const bool bf = dtype == FA_BF16;
+  if (d == 64)
+    e = bf ? launch_fwd<64, true>(mq, mk, mv, a, st) : launch_fwd<64, false>(mq, mk, mv, a, st);
+  else
+    e = bf ? launch_fwd<128, true>(mq, mk, mv, a, st) : launch_fwd<128, false>(mq, mk, mv, a, st);
+  return e == cudaSuccess ? FA_OK : cuda_fail(e);
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+size_t lists_bytes(int nT) {
+  // row_ptr, col_ptr [nT+1] and col_idx, row_idx [nT*nT], each 256-byte aligned
+  return 2 * align_up((size_t)(nT + 1) * 4, 256) + 2 * align_up((size_t)nT * nT * 4, 256);
+}
+
+struct Lists {
+  int32_t *row_ptr, *col_idx, *col_ptr, *row_idx;
+};
+
+Lists carve_lists(void* ws, int nT) {
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  Lists l;
+  l.row_ptr = reinterpret_cast<int32_t*>(p);
+  p += align_up((size_t)(nT + 1) * 4, 256);
+  l.col_ptr = reinterpret_cast<int32_t*>(p);
+  p += align_up((size_t)(nT + 1) * 4, 256);
+  l.col_idx = reinterpret_cast<int32_t*>(p);
+  p += align_up((size_t)nT * nT * 4, 256);
+  l.row_idx = reinterpret_cast<int32_t*>(p);
+  return l;
+}
+
+int launch_lists(const uint8_t* mask, int nT, const Lists& l, cudaStream_t st) {
+  fa::blockmask_lists_kernel<<<1, fa::kMaskThreads, 0, st>>>(mask, nT, l.row_ptr, l.col_idx, l.col_ptr, l.row_idx);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? FA_OK : cuda_fail(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_version(void) { return kVersion; }
+
+const char* fa_status_string(int s) {
+  switch (s) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA";
+    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
+    case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE";
+    default: return "FA_UNKNOWN_STATUS";
+  }
+}
+
+const char* fa_last_error_string(void) { return t_last_error.c_str(); }
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+           float softmax_scale, int causal, const int32_t* key_lens, int dtype, void* stream) {
+  int rc = check_common(q, k, v, B, H, N, d, softmax_scale, dtype);
+  if (rc != FA_OK) return rc;
+  if (!o || !lse || !aligned(o, 16) || !aligned(lse, 4) || (key_lens && !aligned(key_lens, 4)))
+    return FA_ERR_INVALID_ARG;
+  return run_fwd(q, k, v, o, lse, B, H, N, d, softmax_scale, causal, key_lens, nullptr, nullptr, dtype,
+                 static_cast<cudaStream_t>(stream));
+}
+
+size_t fa_blocksparse_workspace_size(int N) {
+  if (N < 1 || N > kMaxN) return 0;
+  return lists_bytes((N + fa::kTile - 1) / fa::kTile);
+}
+
+int fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                       float softmax_scale, int causal, const int32_t* key_lens, const uint8_t* block_mask,
+                       void* workspace, size_t workspace_bytes, int dtype, void* stream) {
+  int rc = check_common(q, k, v, B, H, N, d, softmax_scale, dtype);
+  if (rc != FA_OK) return rc;
+  if (!o || !lse || !block_mask || !aligned(o, 16) || !aligned(lse, 4) || (key_lens && !aligned(key_lens, 4)))
+    return FA_ERR_INVALID_ARG;
+  const int nT = (N + fa::kTile - 1) / fa::kTile;
+  if (nT > fa::kMaxMaskTiles) return FA_ERR_INVALID_ARG;
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < lists_bytes(nT)) return FA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Lists l = carve_lists(workspace, nT);
+  if ((rc = launch_lists(block_mask, nT, l, st)) != FA_OK) return rc;
+  return run_fwd(q, k, v, o, lse, B, H, N, d, softmax_scale, causal, key_lens, l.row_ptr, l.col_idx, dtype, st);
+}
+
+int fa_blockmask_lists(const uint8_t* mask, int nT, int32_t* row_ptr, int32_t* col_idx, int32_t* col_ptr,
+                       int32_t* row_idx, void* stream) {
+  if (!mask || !row_ptr || !col_idx || !col_ptr || !row_idx || nT < 1 || nT > fa::kMaxMaskTiles)
+    return FA_ERR_INVALID_ARG;
+  Lists l{row_ptr, col_idx, col_ptr, row_idx};
+  return launch_lists(mask, nT, l, static_cast<cudaStream_t>(stream));
+}
+
+size_t fa_bwd_workspace_size(int B, int H, int N, int d, int has_block_mask) {
+  if (B < 1 || H < 1 || N < 1 || N > kMaxN || (d != 64 && d != 128)) return 0;
+  const int nT = (N + fa::kTile - 1) / fa::kTile;
+  return fa::bwd_workspace_bytes(B * H, nT, d) + (has_block_mask ? lists_bytes(nT) : 0);
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse, void* dq,
+           void* dk, void* dv, int B, int H, int N, int d, float softmax_scale, int causal, const int32_t* key_lens,
+           const uint8_t* block_mask, void* workspace, size_t workspace_bytes, int dtype, void* stream) {
+  int rc = check_common(q, k, v, B, H, N, d, softmax_scale, dtype);
+  if (rc != FA_OK) return rc;
+  if (!o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  if (!aligned(o, 16) || !aligned(dout, 16) || !aligned(lse, 4) || !aligned(dq, 16) || !aligned(dk, 16) ||
+      !aligned(dv, 16) || (key_lens && !aligned(key_lens, 4)))
+    return FA_ERR_INVALID_ARG;
+  const int nT = (N + fa::kTile - 1) / fa::kTile;
+  if (block_mask && nT > fa::kMaxMaskTiles) return FA_ERR_INVALID_ARG;
+  const size_t need = fa_bwd_workspace_size(B, H, N, d, block_mask != nullptr);
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < need) return FA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int32_t *col_ptr = nullptr, *row_idx = nullptr;
+  if (block_mask) {
+    const Lists l = carve_lists(static_cast<uint8_t*>(workspace) + fa::bwd_workspace_bytes(B * H, nT, d), nT);
+    if ((rc = launch_lists(block_mask, nT, l, st)) != FA_OK) return rc;
+    col_ptr = l.col_ptr;
+    row_idx = l.row_idx;
+  }
+  CUtensorMap mq, mk, mv, mdo;
+  if ((rc = make_map(&mq, q, B * H, N, d, dtype)) != FA_OK) return rc;
+  if ((rc = make_map(&mk, k, B * H, N, d, dtype)) != FA_OK) return rc;
+  if ((rc = make_map(&mv, v, B * H, N, d, dtype)) != FA_OK) return rc;
+  if ((rc = make_map(&mdo, dout, B * H, N, d, dtype)) != FA_OK) return rc;
+  cudaError_t e = fa::run_bwd(mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, B, H, N, d, softmax_scale, causal != 0,
+                              key_lens, col_ptr, row_idx, workspace, dtype == FA_BF16, g_budget_ns.load(), st,
+                              t_events[FA_KERNEL_BWD_MAIN][0], t_events[FA_KERNEL_BWD_MAIN][1]);
+  return e == cudaSuccess ? FA_OK : cuda_fail(e);
+}
+
+int fa_last_device_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  int v = 0;
+  e = cudaMemcpyFromSymbol(&v, fa::g_device_status, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (v != 0) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(fa::g_device_status, &zero, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  return v == 0 ? FA_OK : v;
+}
+
+int fa_set_wait_budget_ns(uint64_t budget_ns) {
+  if (budget_ns < 1000) return FA_ERR_INVALID_ARG;
+  g_budget_ns.store(budget_ns);
+  return FA_OK;
+}
+
+int fa_set_kernel_events(int kernel, void* start_event, void* stop_event) {
+  if (kernel != FA_KERNEL_FWD && kernel != FA_KERNEL_BWD_MAIN) return FA_ERR_INVALID_ARG;
+  if ((start_event == nullptr) != (stop_event == nullptr)) return FA_ERR_INVALID_ARG;
+  t_events[kernel][0] = static_cast<cudaEvent_t>(start_event);
+  t_events[kernel][1] = static_cast<cudaEvent_t>(stop_event);
+  return FA_OK;
+}
+
+int fa_selftest_wait_timeout(uint64_t budget_ns, void* stream) {
+  if (budget_ns < 1000 || budget_ns > 1000000000ull) return FA_ERR_INVALID_ARG;
+  fa::selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(budget_ns);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? FA_OK : cuda_fail(e);
+}
+
+}  // extern "C"

@@ -1,0 +1,147 @@
+/*
+ * fa.h -- C ABI of libfa.so: exact IO-aware attention (tiled forward with online softmax, backward by
+ * recomputation, optional 128x128 block-sparse tile mask) for NVIDIA B200 (sm_100a).
+ *
+ * What the library computes (FlashAttention review page, "Method" and claim C2: exact attention, only the output
+ * and a small normalisation state written to HBM; claim C7: backward recomputes tiles from the saved state;
+ * explainer page, "standard attention", "online softmax" and block-sparse sections):
+ *     S = softmax_scale * Q K^T with masked entries at -inf,  P = softmax(S) per row,  O = P V,
+ *     LSE_r = log sum_c exp(S_rc)   (natural log; -inf for a row with no visible key, whose O row is 0),
+ *     and for the loss sum(O * dO):  D = rowsum(dO * O),  dV = P^T dO,  dS = P * (dO V^T - D),
+ *     dQ = softmax_scale * dS K,  dK = softmax_scale * dS^T Q.
+ * Key c is visible from query row r of sequence b iff (causal == 0 || c <= r) && (key_lens == NULL ||
+ * c < key_lens[b]) && (block_mask == NULL || block_mask[(r/128)*nT + c/128] != 0).
+ *
+ * Conventions shared by every call
+ *   Layout      q, k, v, o, dO, dq, dk, dv: [B, H, N, d] contiguous, d innermost, 16-bit (dtype below).
+ *               lse: [B, H, N] fp32.  key_lens: [B] int32 with 0 <= key_lens[b] <= N.
+ *               block_mask: [nT, nT] uint8 (0 = skip tile), nT = ceil(N/128), shared by all b and h.
+ *   Pointers    Device pointers, 16-byte aligned, caller-owned; the library never allocates, frees or keeps them.
+ *               Scratch that a call needs is passed in as `workspace` (device memory, 256-byte aligned) of at
+ *               least the size returned by the matching *_workspace_size query.
+ *   Shapes      B >= 1, H >= 1, 1 <= N <= 1048576 (2^20), d in {64, 128}, B*H*N*d <= 2^34, softmax_scale finite
+ *               and > 0.
+ *   Execution   Asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).  Inputs must stay valid
+ *               until the stream reaches the work.
+ *   Errors      Argument errors are detected on the host before anything is launched and returned as an
+ *               fa_status; launch failures return FA_ERR_CUDA.  Errors found by the kernels while running (a
+ *               pipeline wait that exceeded its time budget) are recorded in a per-device status word and
+ *               returned by fa_last_device_status().  Non-finite inputs are not checked; they propagate.
+ *   Threads     Calls may come from several host threads; each call only reads library state that is set once.
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad shape, scale <= 0, bad dtype */
+  FA_ERR_UNSUPPORTED = 2, /* head dimension other than 64 or 128 */
+  FA_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed (message: fa_last_error_string) */
+  FA_ERR_TIMEOUT = 4,     /* a kernel wait ran out of its time budget (device-detected) */
+  FA_ERR_WORKSPACE = 5    /* workspace missing, misaligned or smaller than the query says */
+} fa_status;
+
+typedef enum { FA_BF16 = 0, FA_FP16 = 1 } fa_dtype;
+
+/* Library version as major*10000 + minor*100 + patch. */
+int fa_version(void);
+
+/* Human-readable name of an fa_status value (static string). */
+const char* fa_status_string(int status);
+
+/* Text of the last CUDA error seen by a call on this host thread ("" if none). */
+const char* fa_last_error_string(void);
+
+/*
+ * Forward (review page "Method"; slide deck "Executable shape"): each CTA owns two 128-row Q tiles, streams the
+ * visible 128-key K/V tiles through shared memory, keeps the running max and denominator per row on chip and
+ * writes only O and LSE.  Tiles that the causal mask or the key lengths hide entirely are never loaded.
+ *   q, k, v   in   [B,H,N,d]     o   out [B,H,N,d]     lse  out [B,H,N] fp32 (natural log)
+ *   causal    nonzero: key c visible from row r only if c <= r
+ *   key_lens  optional [B] int32 device array (NULL: every key visible)
+ *   dtype     fa_dtype of q, k, v and o
+ */
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+           float softmax_scale, int causal, const int32_t* key_lens, int dtype, void* stream);
+
+/* Bytes of workspace fa_fwd_blocksparse needs for sequence length N (the tile lists). */
+size_t fa_blocksparse_workspace_size(int N);
+
+/*
+ * Block-sparse forward (explainer page, block-sparse section: masking whole tiles means never loading them).
+ * Same arguments as fa_fwd plus a device block_mask [nT*nT] uint8.  The call first converts the mask into
+ * per-row lists of kept tiles in `workspace` (device kernel), then runs the forward over those lists only;
+ * causal and key_lens still apply inside kept tiles.  The result is exact attention under the combined mask.
+ */
+int fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
+                       int d, float softmax_scale, int causal, const int32_t* key_lens, const uint8_t* block_mask,
+                       void* workspace, size_t workspace_bytes, int dtype, void* stream);
+
+/* Bytes of workspace fa_bwd needs (fp32 dQ accumulator, per-row LSE/D in base 2, tile lists if masked). */
+size_t fa_bwd_workspace_size(int B, int H, int N, int d, int has_block_mask);
+
+/*
+ * Backward (review page claim C7: P is recomputed tile by tile from the saved LSE; the N x N matrix never exists
+ * in HBM).  Inputs q, k, v, o, dO [B,H,N,d] and lse [B,H,N] from fa_fwd with the same mask arguments; outputs
+ * dq, dk, dv [B,H,N,d] (fully overwritten).  block_mask may be NULL.  Runs a preprocessing kernel (D = rowsum(dO*O),
+ * zeroed dQ accumulator), the main kernel (one CTA per 128-key tile, looping over the visible Q tiles; dK, dV
+ * accumulate on chip, dQ by fp32 atomics into the workspace) and a conversion kernel for dQ.
+ */
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+           void* dq, void* dk, void* dv, int B, int H, int N, int d, float softmax_scale, int causal,
+           const int32_t* key_lens, const uint8_t* block_mask, void* workspace, size_t workspace_bytes, int dtype,
+           void* stream);
+
+/*
+ * Block-mask index lists on the device (explainer page, block-sparse section), exposed for exact checks:
+ * from mask [nT*nT] uint8 builds CSR row_ptr [nT+1] / col_idx [nT*nT] (kept tiles per row, ascending) and CSC
+ * col_ptr [nT+1] / row_idx [nT*nT] (kept tiles per column, ascending).  All pointers are device pointers;
+ * 1 <= nT <= 8192.
+ */
+int fa_blockmask_lists(const uint8_t* mask, int nT, int32_t* row_ptr, int32_t* col_idx, int32_t* col_ptr,
+                       int32_t* row_idx, void* stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the current device's status word: FA_OK, or FA_ERR_TIMEOUT if a
+ * kernel abandoned a wait since the last query (its outputs are then unspecified).  FA_ERR_CUDA if the
+ * synchronisation itself failed.
+ */
+int fa_last_device_status(void* stream);
+
+/*
+ * Time budget of every pipeline wait inside the kernels, in nanoseconds (default 2e9).  A wait that exceeds it
+ * records FA_ERR_TIMEOUT and the kernel unwinds (drains its own copies, frees its tensor memory, returns).
+ * Values below 1000 are rejected with FA_ERR_INVALID_ARG.  Process-wide; affects launches made after the call.
+ */
+int fa_set_wait_budget_ns(uint64_t budget_ns);
+
+/*
+ * Self-test of the timeout path: launches one CTA that waits on an mbarrier nobody arrives on, with the given
+ * budget (1000 ns .. 1e9 ns).  The wait gives up, records FA_ERR_TIMEOUT in the status word and the kernel returns
+ * normally; read the result with fa_last_device_status().
+ */
+int fa_selftest_wait_timeout(uint64_t budget_ns, void* stream);
+
+/* Kernels that fa_set_kernel_events can bracket. */
+typedef enum { FA_KERNEL_FWD = 0, FA_KERNEL_BWD_MAIN = 1 } fa_kernel_id;
+
+/*
+ * Measurement hook (no counterpart on the pages): on this host thread, make the next calls record `start_event`
+ * immediately before and `stop_event` immediately after the launch of the given kernel (fa_fwd's kernel, or the
+ * main kernel of fa_bwd), on the call's stream.  Events are cudaEvent_t handles owned by the caller; NULL for both
+ * turns the hook off.  Returns FA_ERR_INVALID_ARG for an unknown kernel id or a half-set pair.
+ */
+int fa_set_kernel_events(int kernel, void* start_event, void* stop_event);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */

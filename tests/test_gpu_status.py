@@ -1,0 +1,27 @@
+"""Device-side failure detection without a GPU fault: a kernel waits on an mbarrier that nothing arrives on, its
+bounded wait gives up, records FA_ERR_TIMEOUT in the status word and returns; the host reads and clears it."""
+import pytest
+import torch
+
+import exact_io_aware_48_b200 as fa
+from exact_io_aware_48_b200 import _lib
+
+pytestmark = pytest.mark.gpu
+
+
+def test_wait_timeout_is_reported_and_cleared():
+    assert fa.last_device_status() == _lib.FA_OK
+    assert _lib.fa_selftest_wait_timeout(1_000_000) == _lib.FA_OK  # 1 ms budget
+    assert fa.last_device_status() == _lib.FA_ERR_TIMEOUT
+    assert fa.last_device_status() == _lib.FA_OK  # cleared by the read
+    # the context is still usable afterwards
+    q = torch.randn(1, 1, 128, 64, device="cuda", dtype=torch.bfloat16)
+    o, lse = fa.attention_fwd(q, q, q)
+    assert fa.last_device_status() == _lib.FA_OK
+    assert torch.isfinite(o.float()).all()
+
+
+def test_cpu_tensors_are_rejected():
+    q = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16)
+    with pytest.raises(RuntimeError):
+        fa.attention_fwd(q, q, q)
