@@ -28,6 +28,14 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "attention fwd / fwd+bwd TFLOP/s on 1 B200 and % of dense BF16 tensor peak"
+WORKLOAD_NAMES = {
+    "gpt2": "gpt2-small-shaped causal self-attention fwd+bwd B8 H12 N1024 d64 bf16",
+    "tiny": "tiny exact attention fwd+bwd B1 H2 N256 d64 bf16",
+    "bert": "bert-large-shaped attention with key lengths fwd+bwd B16 H16 N512 d64 bf16",
+    "lc4k": "long-context causal fwd+bwd B1 H16 N4096 d128 bf16",
+    "lc8k": "long-context causal fwd+bwd B1 H16 N8192 d128 bf16",
+    "lc16k": "long-context causal fwd+bwd B1 H16 N16384 d128 bf16",
+}
 L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
 
 
@@ -179,6 +187,11 @@ def time_loop(fn, steps, stream, flush, kernel_events=None):
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)] \
         if kernel_events else None
+    if kev:  # torch creates the CUDA event lazily on first record: create them before handing them to the library
+        for a, b in kev:
+            a.record(stream)
+            b.record(stream)
+        stream.synchronize()
     with torch.cuda.stream(stream):
         for s in range(steps):
             flush.zero_()
@@ -236,7 +249,7 @@ def run_ours(args):
     stream = torch.cuda.Stream()
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
 
-    w = inputs.workloads()["gpt2"]
+    w = inputs.workloads()[args.workload]
     p = Problem(w, seed_offset=rank)
     for _ in range(args.warmup):
         p.step(stream)
@@ -274,12 +287,12 @@ def run_ours(args):
     # roofline of the dominant kernel (bwd main: 2.5x forward FLOPs per launch), timed live by events
     kmean = float(np.mean(kern_ms))
     achieved = 2.5 * p.fwd_flops / (kmean / 1e3) / 1e12
-    roofline = {"kernel": "bwd_kernel<64,bf16>", "bound": "tensor", "achieved": round(achieved, 2),
+    roofline = {"kernel": f"bwd_kernel<{w.d},{w.dtype}>", "bound": "tensor", "achieved": round(achieved, 2),
                 "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                 "peak_source": f"{peak_src} bf16_tflops (burst)", "kernel_ms": round(kmean, 4),
                 "traffic": None}
     # ------------------------------------------------------------------ end to end through the C ABI, host buffers
-    e2e = run_e2e(p, stream, args, world)
+    e2e = run_e2e(p, stream, args, world) if args.e2e else None
 
     targets = measure_targets(stream, flush, peak) if (args.targets and rank == 0) else None
     cpu = cpu_baseline(p.w) if rank == 0 and world == 1 and args.cpu_baseline else None
@@ -288,9 +301,9 @@ def run_ours(args):
         line = {
             "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": "gpt2-small-shaped causal self-attention fwd+bwd B8 H12 N1024 d64 bf16",
-                       "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": True, "global_batch": w.B * world,
+            "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": WORKLOAD_NAMES.get(w.name, w.name),
+                       "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal, "global_batch": w.B * world,
                        "seq_len": w.N, "parallelism": f"dp{world} (independent heads per rank, no collective)",
                        "l2": "flushed (256 MiB write, untimed) before every timed step",
                        "flop_convention": "fwd 4*d*visible pairs; bwd 2.5x; step 3.5x"},
@@ -420,6 +433,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-targets", dest="targets", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--no-e2e", dest="e2e", action="store_false")
+    ap.add_argument("--workload", default="gpt2", choices=sorted(WORKLOAD_NAMES),
+                    help="timed workload (default: the GPT-2-small shape; others are for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

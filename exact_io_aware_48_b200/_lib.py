@@ -134,5 +134,8 @@ def fa_set_kernel_events(kernel, start_event, stop_event) -> int:
     def h(e):
         if e is None:
             return None
-        return e if isinstance(e, int) else e.cuda_event
+        handle = e if isinstance(e, int) else e.cuda_event
+        if not handle:
+            raise ValueError("CUDA event not created yet (torch creates events on their first record())")
+        return handle
     return load().fa_set_kernel_events(kernel, h(start_event), h(stop_event))
