@@ -180,6 +180,19 @@ class Problem:
         self.bwd(stream)
 
 
+def aggregate(local_ms, step_flops, steps, world, device):
+    """Whole-job throughput: every rank ran `steps` steps of `step_flops` each; the job time is the max of the
+    ranks' device times (one all-reduce MAX when world > 1).  Returns (TFLOP/s, max ms)."""
+    total_ms = float(local_ms)
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        t = torch.tensor([total_ms], device=device, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    return world * step_flops * steps / (total_ms / 1e3) / 1e12, total_ms
+
+
 def time_loop(fn, steps, stream, flush, kernel_events=None):
     """Device time (ms) of each call of fn, L2 flushed before each (flush not timed).  kernel_events: optional
     (kernel_id, lib) whose launches are bracketed by per-step events; returns (step_ms list, kernel_ms list)."""
@@ -266,16 +279,10 @@ def run_ours(args):
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    total_ms = float(sum(step_ms))
-    if world > 1:
-        t = torch.tensor([total_ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
     if _lib.fa_last_device_status(stream.cuda_stream) != 0:
         raise RuntimeError("device status error in timed region")
-
     step_flops = 3.5 * p.fwd_flops
-    value = world * step_flops * args.steps / (total_ms / 1e3) / 1e12
+    value, total_ms = aggregate(float(sum(step_ms)), step_flops, args.steps, world, "cuda")
     ms_per_step = total_ms / args.steps
 
     # separate fwd / bwd breakdown (not part of the headline value)
