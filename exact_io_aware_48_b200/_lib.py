@@ -32,7 +32,9 @@ SIGNATURES = {
     "fa_set_wait_budget_ns": ([_U64], _I),
     "fa_selftest_wait_timeout": ([_U64, _P], _I),
     "fa_set_kernel_events": ([_I, _P, _P], _I),
+    "fa_bwd_noalloc": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P, _P, _I, _P], _I),
 }
+FA_NOALLOC_SCRATCH_BYTES = 32 << 20
 FA_KERNEL_FWD, FA_KERNEL_BWD_MAIN = 0, 1
 
 _lib = None
@@ -139,3 +141,11 @@ def fa_set_kernel_events(kernel, start_event, stop_event) -> int:
             raise ValueError("CUDA event not created yet (torch creates events on their first record())")
         return handle
     return load().fa_set_kernel_events(kernel, h(start_event), h(stop_event))
+
+
+def fa_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, softmax_scale, causal, key_lens, block_mask,
+                   dtype, stream=None) -> int:
+    """fa_bwd with the library's fixed device scratch instead of a caller workspace (allocates nothing)."""
+    return load().fa_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
+                                 _ptr(dv), B, H, N, d, softmax_scale, int(causal), _ptr(key_lens), _ptr(block_mask),
+                                 dtype, _stream(stream))

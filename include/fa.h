@@ -129,6 +129,29 @@ int fa_set_wait_budget_ns(uint64_t budget_ns);
  */
 int fa_selftest_wait_timeout(uint64_t budget_ns, void* stream);
 
+/* Size of the fixed device scratch array behind fa_bwd_noalloc: 32 MiB, held by every GPU that loads the library
+ * until the process exits. */
+#define FA_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/*
+ * fa_bwd without a workspace argument, for callers that cannot allocate device memory when they run the backward
+ * (for example code inside a framework or plugin host that owns all device memory and forbids allocation during
+ * execution, or a latency-sensitive loop that cannot pay for cudaMalloc's implicit synchronisation).  No
+ * counterpart in the paper: it is a packaging of the same computation.  The scratch fa_bwd needs comes from a
+ * file-scope device array of FA_NOALLOC_SCRATCH_BYTES inside the library; this call allocates nothing and calls no
+ * allocating routine.  Arguments, layouts and results are exactly those of fa_bwd.
+ *   Size limit  problems whose fa_bwd_workspace_size() exceeds FA_NOALLOC_SCRATCH_BYTES are rejected with
+ *               FA_ERR_WORKSPACE before anything is launched (e.g. B*H = 96, N = 1024, d = 64 needs 24.75 MiB: fits).
+ *   Set-up      the first call on a device looks up the array's device address (cudaGetSymbolAddress) with that
+ *               device current; make that first call before any stream capture.
+ *   Sharing     every call on a device uses the same array and it keeps the last call's contents (each call
+ *               rewrites what it reads, including zeroing its dQ accumulator).  Calls that overlap on the GPU (on
+ *               different streams, or from different host threads without ordering) race on the array.
+ */
+int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                   void* dq, void* dk, void* dv, int B, int H, int N, int d, float softmax_scale, int causal,
+                   const int32_t* key_lens, const uint8_t* block_mask, int dtype, void* stream);
+
 /* Kernels that fa_set_kernel_events can bracket. */
 typedef enum { FA_KERNEL_FWD = 0, FA_KERNEL_BWD_MAIN = 1 } fa_kernel_id;
 
