@@ -13,14 +13,17 @@
 //   bwd_kernel       one CTA per 128-key tile j of one (b, h); loops over the visible 128-row Q tiles i.
 //                    Five tcgen05 GEMMs per (i, j): S^T = K Q^T and dP^T = V dO^T (recompute), dV += P^T dO (P^T read
 //                    from TMEM), dK += dS^T Q and dQ_i = dS K (dS^T staged in shared memory, used K-major for dK and
-//                    M-major for dQ).  dK, dV accumulate in TMEM for the whole loop; each dQ_i partial is added to
-//                    the fp32 accumulator with vector atomics by a dedicated warpgroup.
+//                    M-major for dQ).  dK, dV accumulate in TMEM for the whole loop.  Each dQ_i partial leaves
+//                    through a 128-byte-swizzled shared-memory staging box and TMA bulk tensor reductions (add) into
+//                    the fp32 accumulator: whole-line reductions in L2, no per-thread atomics.
 //   bwd_dq_kernel    fp32 dQ accumulator -> 16-bit dQ.  HBM-bound.
 //
 // Roles in bwd_kernel (320 threads): warps 0-3 recompute P^T and dS^T (thread = key row = TMEM lane), warps 4-7
-// drain dQ_i from TMEM into global atomics (thread = query row), warp 8 issues MMAs, warp 9 issues TMA loads.
-// TMEM (512 columns): S^T [0,128) with P^T (16-bit pairs) over its first 64; dP^T [128,256), reused for dQ_i once
-// dP^T has been read; dV [256,256+d); dK [256+d,256+2d).
+// drain dQ_i (thread = query row), warp 8 issues MMAs, warp 9 issues TMA loads.
+// MMA order per Q tile i: dP^T_i, dV_i, S^T_{i+1}, dK_i, dQ_i -- the next tile's scores are computed before this
+// tile's dK/dQ so the P^T warps recompute P_{i+1} while the tensor core finishes tile i.
+// TMEM (512 columns): S^T [0,128) with P^T (16-bit pairs) over its first 64; dP^T [128,256); dV [256,256+d);
+// dK [256+d,256+2d); dQ_i [384,448) for d = 64, and for d = 128 (no room left) the dP^T columns once read.
 #pragma once
 #include "fa_common.cuh"
 
@@ -34,10 +37,13 @@ struct BwdCfg {
   static constexpr int kSubTiles = D / 64;
   static constexpr int kNumSlots = D == 128 ? 3 : 6;
   static constexpr int kDsBytes = kTile * kTile * 2;      // dS^T, 128 keys x 128 queries
-  static constexpr int kSmemBytes = 2 * kTileBytes + kDsBytes + kNumSlots * kSlotBytes + 1024;
+  static constexpr int kStageBytes = 4 * 4096;             // dQ staging: one 32 x 32 fp32 box per drain warp
+  static constexpr int kSmemBytes = 2 * kTileBytes + kDsBytes + kNumSlots * kSlotBytes + kStageBytes + 1024;
   static constexpr int kThreads = 320;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
+  static constexpr bool kDqOwnCols = (D == 64);            // d = 64: dQ has its own columns
+  static constexpr uint32_t kColDQ = kDqOwnCols ? 384 : kColDP;
 };
 
 // Workspace layout: dq_acc [BH][Npad][D] fp32 | lse2 [BH][Npad] fp32 | Dv [BH][Npad] fp32 (each 256-B aligned)
@@ -184,7 +190,7 @@ template <int D, bool kBF16>
 __global__ void __launch_bounds__(320, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_do,
-               const BwdArgs args) {
+               const __grid_constant__ CUtensorMap map_dq, const BwdArgs args) {
   using C = BwdCfg<D>;
   constexpr int NS = C::kNumSlots;
   extern __shared__ uint8_t smem_raw[];
@@ -193,6 +199,7 @@ __global__ void __launch_bounds__(320, 1)
   uint8_t* sV = smem + C::kTileBytes;
   uint8_t* sDS = smem + 2 * C::kTileBytes;
   uint8_t* sRing = sDS + C::kDsBytes;
+  uint8_t* sStage = sRing + NS * C::kSlotBytes;  // 1024-aligned: slot bytes are multiples of 1024
 
   __shared__ __align__(8) uint64_t bar_kv, bar_full[NS], bar_empty[NS], bar_s, bar_dp, bar_p, bar_ds, bar_dq_full,
       bar_dq_free, bar_ds_free, bar_done, bar_drain;
@@ -284,24 +291,15 @@ __global__ void __launch_bounds__(320, 1)
       constexpr uint32_t id_dq = ptx::idesc_f16(kBF16, true, true, 128, D);      // dQ
       const uint32_t k_base = ptx::smem_addr(sK), v_base = ptx::smem_addr(sV), ds_base = ptx::smem_addr(sDS);
       const uint32_t ring = ptx::smem_addr(sRing);
-      bool ok = true;
-      if (n_iters > 0) {
-        ok = wait_or_abort(ptx::smem_addr(&bar_kv), 0, args.budget_ns, abortp);
+      auto slot_base = [&](int k) { return ring + (k % NS) * C::kSlotBytes; };
+      auto slot_full = [&](int k) { return ptx::smem_addr(&bar_full[k % NS]); };
+      auto slot_empty = [&](int k) { return ptx::smem_addr(&bar_empty[k % NS]); };
+      auto slot_phase = [&](int k) { return (uint32_t)((k / NS) & 1); };
+      // S^T = K Q^T for the Q tile in ring position kq
+      auto issue_s = [&](int kq) -> bool {
+        if (!wait_or_abort(slot_full(kq), slot_phase(kq), args.budget_ns, abortp)) return false;
         ptx::tc_fence_after();
-      }
-      int n = 0, iter = 0, i;
-      while (ok && it.next(i)) {
-        const int sq = n % NS;
-        const uint32_t phq = (n / NS) & 1;
-        ++n;
-        const int so = n % NS;
-        const uint32_t pho = (n / NS) & 1;
-        ++n;
-        const uint32_t q_base = ring + sq * C::kSlotBytes, do_base = ring + so * C::kSlotBytes;
-        const uint32_t ph = iter & 1, ph_prev = (iter - 1) & 1;
-        // S^T = K Q_i^T
-        if (!(ok = wait_or_abort(ptx::smem_addr(&bar_full[sq]), phq, args.budget_ns, abortp))) break;
-        ptx::tc_fence_after();
+        const uint32_t q_base = slot_base(kq);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * 16384 + (kk % 4) * 32;
@@ -309,9 +307,26 @@ __global__ void __launch_bounds__(320, 1)
                       ptx::sw128_desc(q_base + off, 16, 1024), id_sq, kk > 0 ? 1u : 0u);
         }
         ptx::mma_commit(ptx::smem_addr(&bar_s));
-        // dP^T = V dO_i^T (its TMEM columns hold dQ_{i-1} until the dQ warps have drained it)
-        if (!(ok = wait_or_abort(ptx::smem_addr(&bar_full[so]), pho, args.budget_ns, abortp))) break;
-        if (iter > 0 && !(ok = wait_or_abort(ptx::smem_addr(&bar_dq_free), ph_prev, args.budget_ns, abortp))) break;
+        return true;
+      };
+      bool ok = true;
+      int i;
+      bool have = it.next(i);
+      if (have) {
+        ok = wait_or_abort(ptx::smem_addr(&bar_kv), 0, args.budget_ns, abortp);
+        ptx::tc_fence_after();
+        if (ok) ok = issue_s(0);
+      }
+      int iter = 0;
+      while (ok && have) {
+        const int kq = 2 * iter, ko = 2 * iter + 1;
+        const uint32_t q_base = slot_base(kq), do_base = slot_base(ko);
+        const uint32_t ph = iter & 1, ph_prev = (iter - 1) & 1;
+        // dP^T = V dO_i^T (for d = 128 its columns hold dQ_{i-1} until the drain warps have read it)
+        if (!(ok = wait_or_abort(slot_full(ko), slot_phase(ko), args.budget_ns, abortp))) break;
+        if (!C::kDqOwnCols && iter > 0 &&
+            !(ok = wait_or_abort(ptx::smem_addr(&bar_dq_free), ph_prev, args.budget_ns, abortp)))
+          break;
         ptx::tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -327,7 +342,11 @@ __global__ void __launch_bounds__(320, 1)
         for (int kk = 0; kk < kTile / 16; ++kk)
           ptx::mma_ts(tmem + C::kColDV, tmem + C::kColS + kk * 8, ptx::sw128_desc(do_base + kk * 2048, 16384, 1024),
                       id_dv, (iter > 0 || kk > 0) ? 1u : 0u);
-        ptx::mma_commit(ptx::smem_addr(&bar_empty[so]));  // dO_i no longer needed
+        ptx::mma_commit(slot_empty(ko));  // dO_i no longer needed
+        // next tile's scores (P^T_i has been consumed by dV_i, which precedes it in the MMA pipe)
+        int inext;
+        const bool have_next = it.next(inext);
+        if (have_next && !(ok = issue_s(kq + 2))) break;
         // dK += dS^T Q_i and dQ_i = dS K_j  (dS^T in shared memory)
         if (!(ok = wait_or_abort(ptx::smem_addr(&bar_ds), ph, args.budget_ns, abortp))) break;
         ptx::tc_fence_after();
@@ -337,14 +356,20 @@ __global__ void __launch_bounds__(320, 1)
           ptx::mma_ss(tmem + C::kColDK, ptx::sw128_desc(ds_base + off, 16, 1024),
                       ptx::sw128_desc(q_base + kk * 2048, 16384, 1024), id_dv, (iter > 0 || kk > 0) ? 1u : 0u);
         }
-        ptx::mma_commit(ptx::smem_addr(&bar_empty[sq]));  // Q_i (and its LSE2/D rows) no longer needed
+        ptx::mma_commit(slot_empty(kq));  // Q_i (and its LSE2/D rows) no longer needed
+        if (C::kDqOwnCols && iter > 0 &&
+            !(ok = wait_or_abort(ptx::smem_addr(&bar_dq_free), ph_prev, args.budget_ns, abortp)))
+          break;
+        ptx::tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)
-          ptx::mma_ss(tmem + C::kColDP, ptx::sw128_desc(ds_base + kk * 2048, 16384, 1024),
+          ptx::mma_ss(tmem + C::kColDQ, ptx::sw128_desc(ds_base + kk * 2048, 16384, 1024),
                       ptx::sw128_desc(k_base + kk * 2048, 16384, 1024), id_dq, kk > 0 ? 1u : 0u);
         ptx::mma_commit(ptx::smem_addr(&bar_dq_full));
         ptx::mma_commit(ptx::smem_addr(&bar_ds_free));
         ++iter;
+        have = have_next;
+        i = inext;
       }
       if (ok) ptx::mma_commit(ptx::smem_addr(&bar_done));
       ptx::mma_commit(ptx::smem_addr(&bar_drain));
@@ -473,8 +498,14 @@ __global__ void __launch_bounds__(320, 1)
     }
   } else {
     // ------------------------------------------------------------------------------------------ dQ drain warps
-    const int q = (warp - 4) * 32 + lane;  // query row within the tile == TMEM lane
-    const uint32_t lane_base = static_cast<uint32_t>((warp - 4) * 32) << 16;
+    // Each warp owns 32 query rows (its TMEM lanes).  Per 32-column chunk it writes a 32 x 32 fp32 box into its
+    // staging buffer in the 128-byte-swizzled layout of the dq_acc tensor map (16-byte chunk k of row r lands at
+    // k ^ (r % 8): conflict-free), then one lane issues a TMA reduce-add of that box into dq_acc.
+    const int wq = warp - 4;
+    const int q = wq * 32 + lane;  // query row within the tile == TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
+    uint8_t* stage = sStage + wq * 4096;
+    const uint32_t stage_addr = ptx::smem_addr(stage);
     int iter = 0, i;
     while (it.next(i)) {
       const bool ok = __all_sync(0xffffffffu, wait_or_abort(ptx::smem_addr(&bar_dq_full), iter & 1, args.budget_ns,
@@ -483,18 +514,31 @@ __global__ void __launch_bounds__(320, 1)
       ptx::tc_fence_after();
       uint32_t r[D];
 #pragma unroll
-      for (int ch = 0; ch < D / 32; ++ch) ptx::tmem_ld32(tmem + lane_base + C::kColDP + ch * 32,
+      for (int ch = 0; ch < D / 32; ++ch) ptx::tmem_ld32(tmem + lane_base + C::kColDQ + ch * 32,
                                                          *reinterpret_cast<uint32_t(*)[32]>(&r[ch * 32]));
       ptx::tmem_ld_wait();
       ptx::tc_fence_before();
       ptx::mbar_arrive(ptx::smem_addr(&bar_dq_free));  // TMEM columns may now be overwritten
-      float4* dst = reinterpret_cast<float4*>(args.dq_acc + ((size_t)bh * Npad + (size_t)i * kTile + q) * D);
+      const int row0 = (int)((size_t)bh * Npad + (size_t)i * kTile) + wq * 32;
 #pragma unroll
-      for (int v = 0; v < D / 4; ++v)
-        atomicAdd(dst + v, make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
-                                       __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3])));
+      for (int ch = 0; ch < D / 32; ++ch) {
+        if (lane == 0) ptx::bulk_wait_group_read<0>();  // previous box has been read out of the staging buffer
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          *reinterpret_cast<uint4*>(stage + lane * 128 + ((k ^ (lane & 7)) * 16)) =
+              make_uint4(r[ch * 32 + 4 * k], r[ch * 32 + 4 * k + 1], r[ch * 32 + 4 * k + 2], r[ch * 32 + 4 * k + 3]);
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          ptx::tma_reduce_add_2d(&map_dq, ch * 32, row0, stage_addr);
+          ptx::bulk_commit_group();
+        }
+      }
       ++iter;
     }
+    if (lane == 0) ptx::bulk_wait_group<0>();  // all reductions performed before the CTA retires
+    __syncwarp();
   }
 
   ptx::tc_fence_before();
@@ -508,6 +552,7 @@ __global__ void __launch_bounds__(320, 1)
 // ------------------------------------------------------------------------------------------------ host side
 template <int D, bool BF>
 cudaError_t launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
+                       const CUtensorMap& mdq,
                        const void* o, const void* dout, const float* lse, void* dq, const BwdArgs& a,
                        cudaStream_t st, cudaEvent_t ev_start, cudaEvent_t ev_stop) {
   using C = BwdCfg<D>;
@@ -527,7 +572,7 @@ cudaError_t launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
     smem_set.fetch_or(1ull << (dev & 63));
   }
   if (ev_start && (e = cudaEventRecord(ev_start, st)) != cudaSuccess) return e;
-  bwd_kernel<D, BF><<<(unsigned)(a.nT * a.BH), C::kThreads, C::kSmemBytes, st>>>(mq, mk, mv, mdo, a);
+  bwd_kernel<D, BF><<<(unsigned)(a.nT * a.BH), C::kThreads, C::kSmemBytes, st>>>(mq, mk, mv, mdo, mdq, a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (ev_stop && (e = cudaEventRecord(ev_stop, st)) != cudaSuccess) return e;
   const long long total_vec4 = (long long)a.BH * a.N * D / 4;
@@ -537,7 +582,7 @@ cudaError_t launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
 }
 
 inline cudaError_t run_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                           const CUtensorMap& mdo, const void* o, const void* dout, const float* lse, void* dq,
+                           const CUtensorMap& mdo, const CUtensorMap& mdq, const void* o, const void* dout, const float* lse, void* dq,
                            void* dk, void* dv, int B, int H, int N, int d, float scale, bool causal,
                            const int32_t* key_lens, const int32_t* col_ptr, const int32_t* row_idx, void* workspace,
                            bool bf16, uint64_t budget_ns, cudaStream_t st, cudaEvent_t ev_start,
@@ -565,10 +610,10 @@ inline cudaError_t run_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const C
   a.scale_log2 = scale * 1.4426950408889634f;
   a.budget_ns = budget_ns;
   if (d == 64)
-    return bf16 ? launch_bwd<64, true>(mq, mk, mv, mdo, o, dout, lse, dq, a, st, ev_start, ev_stop)
-                : launch_bwd<64, false>(mq, mk, mv, mdo, o, dout, lse, dq, a, st, ev_start, ev_stop);
-  return bf16 ? launch_bwd<128, true>(mq, mk, mv, mdo, o, dout, lse, dq, a, st, ev_start, ev_stop)
-              : launch_bwd<128, false>(mq, mk, mv, mdo, o, dout, lse, dq, a, st, ev_start, ev_stop);
+    return bf16 ? launch_bwd<64, true>(mq, mk, mv, mdo, mdq, o, dout, lse, dq, a, st, ev_start, ev_stop)
+                : launch_bwd<64, false>(mq, mk, mv, mdo, mdq, o, dout, lse, dq, a, st, ev_start, ev_stop);
+  return bf16 ? launch_bwd<128, true>(mq, mk, mv, mdo, mdq, o, dout, lse, dq, a, st, ev_start, ev_stop)
+              : launch_bwd<128, false>(mq, mk, mv, mdo, mdq, o, dout, lse, dq, a, st, ev_start, ev_stop);
 }
 
 }  // namespace fa

@@ -87,6 +87,27 @@ int make_map(CUtensorMap* m, const void* ptr, int BH, int N, int d, int dtype) {
   return FA_OK;
 }
 
+// 2-D fp32 view {cols, rows} of the dQ accumulator for TMA reduce-add: box 32 columns (128 bytes) x 32 rows,
+// 128-byte swizzle (matches the drain warps' staging layout).
+int make_map_f32(CUtensorMap* m, void* ptr, long long rows, int cols) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) {
+    t_last_error = "cuTensorMapEncodeTiled unavailable";
+    return FA_ERR_CUDA;
+  }
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * 4};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, ptr, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    t_last_error = "cuTensorMapEncodeTiled (fp32) failed with CUresult " + std::to_string((int)r);
+    return FA_ERR_CUDA;
+  }
+  return FA_OK;
+}
+
 // cudaFuncSetAttribute for the dynamic shared memory size, once per (kernel, device).  `done_mask` must be a
 // distinct object per kernel (kernels of identical signature would otherwise share one cache).
 template <typename Kernel>
@@ -267,7 +288,9 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
   if ((rc = make_map(&mk, k, B * H, N, d, dtype)) != FA_OK) return rc;
   if ((rc = make_map(&mv, v, B * H, N, d, dtype)) != FA_OK) return rc;
   if ((rc = make_map(&mdo, dout, B * H, N, d, dtype)) != FA_OK) return rc;
-  cudaError_t e = fa::run_bwd(mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, B, H, N, d, softmax_scale, causal != 0,
+  CUtensorMap mdq;  // the fp32 dQ accumulator sits at the start of the workspace: [B*H*Npad, d]
+  if ((rc = make_map_f32(&mdq, workspace, (long long)B * H * nT * fa::kTile, d)) != FA_OK) return rc;
+  cudaError_t e = fa::run_bwd(mq, mk, mv, mdo, mdq, o, dout, lse, dq, dk, dv, B, H, N, d, softmax_scale, causal != 0,
                               key_lens, col_ptr, row_idx, workspace, dtype == FA_BF16, g_budget_ns.load(), st,
                               t_events[FA_KERNEL_BWD_MAIN][0], t_events[FA_KERNEL_BWD_MAIN][1]);
   return e == cudaSuccess ? FA_OK : cuda_fail(e);
