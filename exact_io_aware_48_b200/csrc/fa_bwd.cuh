@@ -18,8 +18,9 @@
 //                    the fp32 accumulator: whole-line reductions in L2, no per-thread atomics.
 //   bwd_dq_kernel    fp32 dQ accumulator -> 16-bit dQ.  HBM-bound.
 //
-// Roles in bwd_kernel (320 threads): warps 0-3 recompute P^T and dS^T (thread = key row = TMEM lane), warps 4-7
-// drain dQ_i (thread = query row), warp 8 issues MMAs, warp 9 issues TMA loads.
+// Roles in bwd_kernel (512 threads): warps 0-7 recompute P^T and dS^T (thread = key row = TMEM lane; warpgroup g
+// takes queries [64g, 64g+64), so every SM sub-partition interleaves two such warps), warps 8-11 drain dQ_i
+// (thread = query row), warp 12 issues MMAs, warp 13 issues TMA loads, warps 14-15 only pad the fourth warpgroup.
 // MMA order per Q tile i: dP^T_i, dV_i, S^T_{i+1}, dK_i, dQ_i -- the next tile's scores are computed before this
 // tile's dK/dQ so the P^T warps recompute P_{i+1} while the tensor core finishes tile i.
 // TMEM (512 columns): S^T [0,128) with P^T (16-bit pairs) over its first 64; dP^T [128,256); dV [256,256+d);
@@ -39,7 +40,7 @@ struct BwdCfg {
   static constexpr int kDsBytes = kTile * kTile * 2;      // dS^T, 128 keys x 128 queries
   static constexpr int kStageBytes = 4 * 4096;             // dQ staging: one 32 x 32 fp32 box per drain warp
   static constexpr int kSmemBytes = 2 * kTileBytes + kDsBytes + kNumSlots * kSlotBytes + kStageBytes + 1024;
-  static constexpr int kThreads = 320;
+  static constexpr int kThreads = 512;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
   static constexpr bool kDqOwnCols = (D == 64);            // d = 64: dQ has its own columns
@@ -187,7 +188,7 @@ __global__ void __launch_bounds__(256) bwd_dq_kernel(const float* __restrict__ d
 
 // ------------------------------------------------------------------------------------------------ main kernel
 template <int D, bool kBF16>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(512, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_do,
                const __grid_constant__ CUtensorMap map_dq, const BwdArgs args) {
@@ -208,6 +209,8 @@ __global__ void __launch_bounds__(320, 1)
   volatile int* abortp = &abort_flag;
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  // warps 0-7: P^T/dS^T (two warpgroups, one per 64-query half), 8-11: dQ drain, 12: MMA, 13: TMA, 14-15: idle
+  constexpr int kWarpDrain = 8, kWarpMma = 12, kWarpLoad = 13;
   const int L = blockIdx.x;
   const int j = L / args.BH;  // K/V tile; ascending j = longest causal work first
   const int bh = L % args.BH;
@@ -225,8 +228,8 @@ __global__ void __launch_bounds__(320, 1)
     }
     ptx::mbar_init(ptx::smem_addr(&bar_s), 1);
     ptx::mbar_init(ptx::smem_addr(&bar_dp), 1);
-    ptx::mbar_init(ptx::smem_addr(&bar_p), 128);
-    ptx::mbar_init(ptx::smem_addr(&bar_ds), 128);
+    ptx::mbar_init(ptx::smem_addr(&bar_p), 256);
+    ptx::mbar_init(ptx::smem_addr(&bar_ds), 256);
     ptx::mbar_init(ptx::smem_addr(&bar_dq_full), 1);
     ptx::mbar_init(ptx::smem_addr(&bar_dq_free), 128);
     ptx::mbar_init(ptx::smem_addr(&bar_ds_free), 1);
@@ -235,7 +238,7 @@ __global__ void __launch_bounds__(320, 1)
     abort_flag = 0;
     ptx::fence_barrier_init();
   }
-  if (warp == 8) {
+  if (warp == kWarpMma) {
     ptx::tmem_alloc(ptx::smem_addr(&tmem_base_sh), C::kTmemCols);
     ptx::tmem_relinquish();
   }
@@ -248,7 +251,7 @@ __global__ void __launch_bounds__(320, 1)
   it.init(args.col_ptr, args.row_idx, j, args.nT, causal ? j : 0, visible);
   const int n_iters = it.count();
 
-  if (warp == 9) {
+  if (warp == kWarpLoad) {
     // ------------------------------------------------------------------------------------------ TMA producer
     if (lane == 0 && n_iters > 0) {
       ptx::prefetch_tensormap(&map_q);
@@ -283,7 +286,7 @@ __global__ void __launch_bounds__(320, 1)
       for (int k = (n > NS ? n - NS : 0); k < n; ++k)
         ptx::mbar_wait(ptx::smem_addr(&bar_full[k % NS]), (k / NS) & 1, args.budget_ns);
     }
-  } else if (warp == 8) {
+  } else if (warp == kWarpMma) {
     // ------------------------------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t id_sq = ptx::idesc_f16(kBF16, false, false, 128, 128);  // S^T, dP^T
@@ -375,11 +378,13 @@ __global__ void __launch_bounds__(320, 1)
       ptx::mma_commit(ptx::smem_addr(&bar_drain));
       ptx::mbar_wait(ptx::smem_addr(&bar_drain), 0, args.budget_ns);
     }
-  } else if (warp < 4) {
+  } else if (warp < kWarpDrain) {
     // ------------------------------------------------------------------------------------------ P^T / dS^T warps
-    const int c = warp * 32 + lane;            // key row within the tile == TMEM lane
+    // Warpgroup g handles queries [64g, 64g+64) of every key row; the 4 warps of a group cover the 128 key rows.
+    const int g = warp / 4, quarter = warp % 4;
+    const int c = quarter * 32 + lane;         // key row within the tile == TMEM lane
     const int gc = j * kTile + c;              // key index in the sequence
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const float sl2 = args.scale_log2, sc = args.scale;
     int n = 0, iter = 0, i;
     bool ok = true;
@@ -387,7 +392,7 @@ __global__ void __launch_bounds__(320, 1)
       const int sq = n % NS;
       const uint32_t phq = (n / NS) & 1;
       n += 2;
-      const float* lse2 = reinterpret_cast<const float*>(sRing + sq * C::kSlotBytes + C::kTileBytes);
+      const float* lse2 = reinterpret_cast<const float*>(sRing + sq * C::kSlotBytes + C::kTileBytes) + 64 * g;
       const float* Drow = lse2 + 128;
       const uint32_t ph = iter & 1;
       // the LSE2/D rows came in by bulk copy with Q_i: observe that copy's barrier before reading them (the slot
@@ -398,64 +403,65 @@ __global__ void __launch_bounds__(320, 1)
       ptx::tc_fence_after();
       const bool masked = (causal && i == j) || (j + 1) * kTile > kv_lim;
       // visible queries of key gc: r >= gc (causal) and the key itself below the key limit
-      const int rmin = causal ? gc - i * kTile : 0;   // first visible query column within the tile
+      const int rmin = causal ? gc - i * kTile - 64 * g : 0;  // first visible query column within this half
       const bool key_ok = gc < kv_lim;
-      uint32_t pk[64];
+      uint32_t pk[32];  // P^T of this half, 16-bit pairs
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
+      for (int h = 0; h < 2; ++h) {
         uint32_t sr[32];
-        ptx::tmem_ld32(tmem + lane_base + C::kColS + ch * 32, sr);
+        ptx::tmem_ld32(tmem + lane_base + C::kColS + 64 * g + 32 * h, sr);
         ptx::tmem_ld_wait();
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
-          const int r0 = ch * 32 + 2 * u;
-          float p0 = ptx::ex2(fmaf(__uint_as_float(sr[2 * u]), sl2, -lse2[r0]));
-          float p1 = ptx::ex2(fmaf(__uint_as_float(sr[2 * u + 1]), sl2, -lse2[r0 + 1]));
+          const int r0 = 32 * h + 2 * u;
+          const float2 l2 = *reinterpret_cast<const float2*>(lse2 + r0);
+          float p0 = ptx::ex2(fmaf(__uint_as_float(sr[2 * u]), sl2, -l2.x));
+          float p1 = ptx::ex2(fmaf(__uint_as_float(sr[2 * u + 1]), sl2, -l2.y));
           if (masked) {
             if (!key_ok || r0 < rmin) p0 = 0.f;
             if (!key_ok || r0 + 1 < rmin) p1 = 0.f;
           }
-          pk[ch * 16 + u] = ptx::pack2<kBF16>(p0, p1);
+          pk[16 * h + u] = ptx::pack2<kBF16>(p0, p1);
         }
       }
-      ptx::tmem_st32(tmem + lane_base + C::kColS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-      ptx::tmem_st32(tmem + lane_base + C::kColS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+      ptx::tmem_st32(tmem + lane_base + C::kColS + 32 * g, pk);  // P^T columns: 2 queries per 32-bit column
       ptx::tmem_st_wait();
       ptx::tc_fence_before();
       ptx::mbar_arrive(ptx::smem_addr(&bar_p));
-      // dS^T = P^T * (dP^T - D) * scale, written 16-bit into the swizzled dS^T tile
+      // dS^T = P^T * (dP^T - D) * scale, written 16-bit into sub-tile g of the swizzled dS^T tile
       ok = __all_sync(0xffffffffu, wait_or_abort(ptx::smem_addr(&bar_dp), ph, args.budget_ns, abortp));
       if (ok && iter > 0)
         ok = __all_sync(0xffffffffu, wait_or_abort(ptx::smem_addr(&bar_ds_free), (iter - 1) & 1, args.budget_ns,
                                                     abortp));
       if (!ok) break;
       ptx::tc_fence_after();
+      uint8_t* rowp = sDS + g * 16384 + c * 128;
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
+      for (int h = 0; h < 2; ++h) {
         uint32_t dr[32];
-        ptx::tmem_ld32(tmem + lane_base + C::kColDP + ch * 32, dr);
+        ptx::tmem_ld32(tmem + lane_base + C::kColDP + 64 * g + 32 * h, dr);
         ptx::tmem_ld_wait();
         uint32_t o[16];
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
-          const int r0 = ch * 32 + 2 * u;
+          const int r0 = 32 * h + 2 * u;
+          const float2 dd = *reinterpret_cast<const float2*>(Drow + r0);
           float p0, p1;
           if constexpr (kBF16) {
-            p0 = __uint_as_float(pk[ch * 16 + u] << 16);
-            p1 = __uint_as_float(pk[ch * 16 + u] & 0xffff0000u);
+            p0 = __uint_as_float(pk[16 * h + u] << 16);
+            p1 = __uint_as_float(pk[16 * h + u] & 0xffff0000u);
           } else {
-            p0 = __half2float(__ushort_as_half((unsigned short)(pk[ch * 16 + u] & 0xffff)));
-            p1 = __half2float(__ushort_as_half((unsigned short)(pk[ch * 16 + u] >> 16)));
+            p0 = __half2float(__ushort_as_half((unsigned short)(pk[16 * h + u] & 0xffff)));
+            p1 = __half2float(__ushort_as_half((unsigned short)(pk[16 * h + u] >> 16)));
           }
-          const float ds0 = p0 * (__uint_as_float(dr[2 * u]) - Drow[r0]) * sc;
-          const float ds1 = p1 * (__uint_as_float(dr[2 * u + 1]) - Drow[r0 + 1]) * sc;
+          const float ds0 = p0 * (__uint_as_float(dr[2 * u]) - dd.x) * sc;
+          const float ds1 = p1 * (__uint_as_float(dr[2 * u + 1]) - dd.y) * sc;
           o[u] = ptx::pack2<kBF16>(ds0, ds1);
         }
-        // queries ch*32 .. ch*32+31 live in sub-tile ch/2, 16-byte chunks (ch%2)*4 .. +3 of row c (swizzled)
-        uint8_t* rowp = sDS + (ch / 2) * 16384 + c * 128;
+        // queries 32h .. 32h+31 of this half: 16-byte chunks 4h .. 4h+3 of row c (128-byte swizzle)
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
-          const int chunk = ((ch % 2) * 4 + v) ^ (c & 7);
+          const int chunk = (4 * h + v) ^ (c & 7);
           *reinterpret_cast<uint4*>(rowp + chunk * 16) = make_uint4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
         }
       }
@@ -465,44 +471,41 @@ __global__ void __launch_bounds__(320, 1)
       ++iter;
     }
     // ------------------------------------------------------------------------------------------ dK, dV epilogue
+    // warpgroup 0 writes dV, warpgroup 1 writes dK (dK already carries the softmax scale through dS)
     if (ok && n_iters > 0)
       ok = __all_sync(0xffffffffu, wait_or_abort(ptx::smem_addr(&bar_done), 0, args.budget_ns, abortp));
     if (ok) {
       ptx::tc_fence_after();
       const bool row_ok = gc < args.N;
-      const size_t off = ((size_t)bh * args.N + gc) * D * 2;
+      uint8_t* dst_row = reinterpret_cast<uint8_t*>(g == 0 ? args.dv : args.dk) + ((size_t)bh * args.N + gc) * D * 2;
+      const uint32_t col = g == 0 ? C::kColDV : C::kColDK;
 #pragma unroll 1
-      for (int which = 0; which < 2; ++which) {
-        uint8_t* dst_row = reinterpret_cast<uint8_t*>(which == 0 ? args.dv : args.dk) + off;
-        const uint32_t col = which == 0 ? C::kColDV : C::kColDK;
-#pragma unroll 1
-        for (int ch = 0; ch < D / 32; ++ch) {
-          uint32_t r[32];
-          if (n_iters > 0) {
-            ptx::tmem_ld32(tmem + lane_base + col + ch * 32, r);
-            ptx::tmem_ld_wait();
-          } else {
+      for (int ch = 0; ch < D / 32; ++ch) {
+        uint32_t r[32];
+        if (n_iters > 0) {
+          ptx::tmem_ld32(tmem + lane_base + col + ch * 32, r);
+          ptx::tmem_ld_wait();
+        } else {
 #pragma unroll
-            for (int u = 0; u < 32; ++u) r[u] = 0u;  // no visible query: zero gradient
-          }
-          uint32_t pkd[16];
+          for (int u = 0; u < 32; ++u) r[u] = 0u;  // no visible query: zero gradient
+        }
+        uint32_t pkd[16];
 #pragma unroll
-          for (int u = 0; u < 16; ++u) pkd[u] = ptx::pack2<kBF16>(__uint_as_float(r[2 * u]), __uint_as_float(r[2 * u + 1]));
-          if (row_ok) {
-            uint4* dst = reinterpret_cast<uint4*>(dst_row + ch * 64);
+        for (int u = 0; u < 16; ++u) pkd[u] = ptx::pack2<kBF16>(__uint_as_float(r[2 * u]), __uint_as_float(r[2 * u + 1]));
+        if (row_ok) {
+          uint4* dst = reinterpret_cast<uint4*>(dst_row + ch * 64);
 #pragma unroll
-            for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pkd[4 * v], pkd[4 * v + 1], pkd[4 * v + 2], pkd[4 * v + 3]);
-          }
+          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pkd[4 * v], pkd[4 * v + 1], pkd[4 * v + 2], pkd[4 * v + 3]);
         }
       }
     }
-  } else {
+  } else if (warp < kWarpMma) {
     // ------------------------------------------------------------------------------------------ dQ drain warps
     // Each warp owns 32 query rows (its TMEM lanes).  Per 32-column chunk it writes a 32 x 32 fp32 box into its
     // staging buffer in the 128-byte-swizzled layout of the dq_acc tensor map (16-byte chunk k of row r lands at
-    // k ^ (r % 8): conflict-free), then one lane issues a TMA reduce-add of that box into dq_acc.
-    const int wq = warp - 4;
-    const int q = wq * 32 + lane;  // query row within the tile == TMEM lane
+    // k ^ (r % 8): conflict-free), then one lane issues a TMA reduce-add of that box into dq_acc.  Columns are read
+    // out of TMEM 64 at a time; the TMEM region is released as soon as the last columns are in registers.
+    const int wq = warp - kWarpDrain;
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
     uint8_t* stage = sStage + wq * 4096;
     const uint32_t stage_addr = ptx::smem_addr(stage);
@@ -512,27 +515,31 @@ __global__ void __launch_bounds__(320, 1)
                                                             abortp));
       if (!ok) break;
       ptx::tc_fence_after();
-      uint32_t r[D];
-#pragma unroll
-      for (int ch = 0; ch < D / 32; ++ch) ptx::tmem_ld32(tmem + lane_base + C::kColDQ + ch * 32,
-                                                         *reinterpret_cast<uint32_t(*)[32]>(&r[ch * 32]));
-      ptx::tmem_ld_wait();
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(ptx::smem_addr(&bar_dq_free));  // TMEM columns may now be overwritten
       const int row0 = (int)((size_t)bh * Npad + (size_t)i * kTile) + wq * 32;
 #pragma unroll
-      for (int ch = 0; ch < D / 32; ++ch) {
-        if (lane == 0) ptx::bulk_wait_group_read<0>();  // previous box has been read out of the staging buffer
-        __syncwarp();
+      for (int half = 0; half < D / 64; ++half) {
+        uint32_t r[2][32];
+        ptx::tmem_ld32(tmem + lane_base + C::kColDQ + 64 * half, r[0]);
+        ptx::tmem_ld32(tmem + lane_base + C::kColDQ + 64 * half + 32, r[1]);
+        ptx::tmem_ld_wait();
+        if (half == D / 64 - 1) {
+          ptx::tc_fence_before();
+          ptx::mbar_arrive(ptx::smem_addr(&bar_dq_free));  // TMEM columns may now be overwritten
+        }
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-          *reinterpret_cast<uint4*>(stage + lane * 128 + ((k ^ (lane & 7)) * 16)) =
-              make_uint4(r[ch * 32 + 4 * k], r[ch * 32 + 4 * k + 1], r[ch * 32 + 4 * k + 2], r[ch * 32 + 4 * k + 3]);
-        ptx::fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          ptx::tma_reduce_add_2d(&map_dq, ch * 32, row0, stage_addr);
-          ptx::bulk_commit_group();
+        for (int cc = 0; cc < 2; ++cc) {
+          if (lane == 0) ptx::bulk_wait_group_read<0>();  // previous box has been read out of the staging buffer
+          __syncwarp();
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            *reinterpret_cast<uint4*>(stage + lane * 128 + ((k ^ (lane & 7)) * 16)) =
+                make_uint4(r[cc][4 * k], r[cc][4 * k + 1], r[cc][4 * k + 2], r[cc][4 * k + 3]);
+          ptx::fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            ptx::tma_reduce_add_2d(&map_dq, 64 * half + 32 * cc, row0, stage_addr);
+            ptx::bulk_commit_group();
+          }
         }
       }
       ++iter;
@@ -543,7 +550,7 @@ __global__ void __launch_bounds__(320, 1)
 
   ptx::tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == kWarpMma) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, C::kTmemCols);
   }
