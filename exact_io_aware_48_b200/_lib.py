@@ -32,6 +32,7 @@ SIGNATURES = {
     "fa_set_wait_budget_ns": ([_U64], _I),
     "fa_selftest_wait_timeout": ([_U64, _P], _I),
     "fa_set_kernel_events": ([_I, _P, _P], _I),
+    "fa_selftest_exp2": ([_P, _P, _P, _I, _P], _I),
     "fa_bwd_noalloc": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P, _P, _I, _P], _I),
 }
 FA_NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -149,3 +150,7 @@ def fa_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, softmax_scale,
     return load().fa_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
                                  _ptr(dv), B, H, N, d, softmax_scale, int(causal), _ptr(key_lens), _ptr(block_mask),
                                  dtype, _stream(stream))
+
+
+def fa_selftest_exp2(x, out_fma, out_mufu, n, stream=None) -> int:
+    return load().fa_selftest_exp2(_ptr(x), _ptr(out_fma), _ptr(out_mufu), n, _stream(stream))

@@ -23,7 +23,7 @@
 // (thread = query row), warp 12 issues MMAs, warp 13 issues TMA loads, warps 14-15 only pad the fourth warpgroup.
 // MMA order per Q tile i: dP^T_i, dV_i, S^T_{i+1}, dK_i, dQ_i -- the next tile's scores are computed before this
 // tile's dK/dQ so the P^T warps recompute P_{i+1} while the tensor core finishes tile i.
-// TMEM (512 columns): S^T [0,128) with P^T (16-bit pairs) over its first 64; dP^T [128,256); dV [256,256+d);
+// TMEM (512 columns): S^T [0,128) with P^T (16-bit pairs) over [0,32) and [64,96); dP^T [128,256); dV [256,256+d);
 // dK [256+d,256+2d); dQ_i [384,448) for d = 64, and for d = 128 (no room left) the dP^T columns once read.
 #pragma once
 #include "fa_common.cuh"
@@ -342,9 +342,9 @@ __global__ void __launch_bounds__(512, 1)
         if (!(ok = wait_or_abort(ptx::smem_addr(&bar_p), ph, args.budget_ns, abortp))) break;
         ptx::tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk)
-          ptx::mma_ts(tmem + C::kColDV, tmem + C::kColS + kk * 8, ptx::sw128_desc(do_base + kk * 2048, 16384, 1024),
-                      id_dv, (iter > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < kTile / 16; ++kk)  // queries 16kk..16kk+15: P^T half kk/4 at column 64*(kk/4)
+          ptx::mma_ts(tmem + C::kColDV, tmem + C::kColS + (kk / 4) * 64 + (kk % 4) * 8,
+                      ptx::sw128_desc(do_base + kk * 2048, 16384, 1024), id_dv, (iter > 0 || kk > 0) ? 1u : 0u);
         ptx::mma_commit(slot_empty(ko));  // dO_i no longer needed
         // next tile's scores (P^T_i has been consumed by dV_i, which precedes it in the MMA pipe)
         int inext;
@@ -424,7 +424,9 @@ __global__ void __launch_bounds__(512, 1)
           pk[16 * h + u] = ptx::pack2<kBF16>(p0, p1);
         }
       }
-      ptx::tmem_st32(tmem + lane_base + C::kColS + 32 * g, pk);  // P^T columns: 2 queries per 32-bit column
+      // P^T of this half (2 queries per 32-bit column) goes to columns [64g, 64g+32): inside the S^T columns this
+      // warpgroup has just read, never over columns the other warpgroup may still be reading
+      ptx::tmem_st32(tmem + lane_base + C::kColS + 64 * g, pk);
       ptx::tmem_st_wait();
       ptx::tc_fence_before();
       ptx::mbar_arrive(ptx::smem_addr(&bar_p));

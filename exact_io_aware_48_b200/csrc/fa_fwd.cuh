@@ -36,6 +36,11 @@ struct FwdCfg {
   static constexpr uint32_t kColO = 256;  // O_t at kColO + t * D
 };
 
+// Every kExpFmaEvery-th pair of probabilities is exponentiated on the FMA pipe (see ptx::exp2_fma); 0 = never.
+// Measured on B200: sending 1 pair in 4 to the FMA pipe lowered long-context forward throughput by 6-7% (the
+// softmax warps are issue/latency bound, not MUFU bound), so it is off.
+constexpr int kExpFmaEvery = 0;
+
 struct FwdArgs {
   void* o;
   float* lse;
@@ -196,8 +201,9 @@ __global__ void __launch_bounds__(320, 1)
         const uint32_t phV = (n / NS) & 1;
         ++n;
         bool k_ready = false;
-        for (int t = 0; t < 2 && ok; ++t) {
-          ok = flush_pv(t);
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          if (ok) ok = flush_pv(t);
           if (ok && (fl & (1 << t))) {
             if (!k_ready) {
               ok = wait_or_abort(ptx::smem_addr(&bar_full[sK]), phK, args.budget_ns, abortp);
@@ -219,7 +225,9 @@ __global__ void __launch_bounds__(320, 1)
         v_ready = false;
       }
       if (ok) {
-        for (int t = 0; t < 2 && ok; ++t) ok = flush_pv(t);
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+          if (ok) ok = flush_pv(t);
         if (ok && pend_flags) ptx::mma_commit(ptx::smem_addr(&bar_empty[pend_slot]));
         if (ok) {
           ptx::mma_commit(ptx::smem_addr(&bar_o[0]));
@@ -268,9 +276,16 @@ __global__ void __launch_bounds__(320, 1)
         for (int i = 0; i < 128; ++i)
           if (c0 + i >= lim) s[i] = -INFINITY;
       }
-      float mx = s[0];
+      // row max: 8 independent partial maxima, then a tree (a single serial chain would cost ~127 max latencies)
+      float pm[8];
 #pragma unroll
-      for (int i = 1; i < 128; ++i) mx = fmaxf(mx, s[i]);
+      for (int a = 0; a < 8; ++a) pm[a] = fmaxf(s[a], s[a + 8]);
+#pragma unroll
+      for (int i = 16; i < 128; i += 8)
+#pragma unroll
+        for (int a = 0; a < 8; ++a) pm[a] = fmaxf(pm[a], s[i + a]);
+      const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                             fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
       const float m_tile = mx * scale_log2;
       const bool need = m_tile > m_ref + 8.0f;
       float alpha = 1.0f;
@@ -279,19 +294,24 @@ __global__ void __launch_bounds__(320, 1)
         m_ref = m_tile;
       }
       const float m_use = (m_ref == -INFINITY) ? 0.0f : m_ref;
-      float sum = 0.f;
+      float ps[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial sums
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t pk[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const float p0 = ptx::ex2(fmaf(s[h * 64 + 2 * i], scale_log2, -m_use));
-          const float p1 = ptx::ex2(fmaf(s[h * 64 + 2 * i + 1], scale_log2, -m_use));
+          // one pair in kExpFmaEvery goes through the FMA-pipe exp2 so the MUFU pipe is not the only exp unit
+          const float x0 = fmaf(s[h * 64 + 2 * i], scale_log2, -m_use);
+          const float x1 = fmaf(s[h * 64 + 2 * i + 1], scale_log2, -m_use);
+          const bool emu = kExpFmaEvery > 0 && (i % (kExpFmaEvery > 0 ? kExpFmaEvery : 1)) == kExpFmaEvery - 1;
+          const float p0 = emu ? ptx::exp2_fma(x0) : ptx::ex2(x0);
+          const float p1 = emu ? ptx::exp2_fma(x1) : ptx::ex2(x1);
           pk[i] = ptx::pack2<kBF16>(p0, p1);
-          sum += ptx::unpack2_sum<kBF16>(pk[i]);  // l sums the rounded P that P V uses: O stays a convex mix
+          ps[i & 3] += ptx::unpack2_sum<kBF16>(pk[i]);  // l sums the rounded P that P V uses: O stays a convex mix
         }
         ptx::tmem_st32(tS + h * 32, pk);
       }
+      const float sum = (ps[0] + ps[1]) + (ps[2] + ps[3]);
       // rescale the running output (only if some row of this warp moved its reference max)
       if (kidx > 0 && __any_sync(0xffffffffu, need)) {
 #pragma unroll 1

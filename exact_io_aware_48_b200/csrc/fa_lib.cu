@@ -324,6 +324,14 @@ int fa_set_kernel_events(int kernel, void* start_event, void* stop_event) {
   return FA_OK;
 }
 
+int fa_selftest_exp2(const float* x, float* out_fma, float* out_mufu, int n, void* stream) {
+  if (!x || !out_fma || !out_mufu || n < 1) return FA_ERR_INVALID_ARG;
+  const int blocks = (n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024;
+  fa::selftest_exp2_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, out_fma, out_mufu, n);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? FA_OK : cuda_fail(e);
+}
+
 int fa_selftest_wait_timeout(uint64_t budget_ns, void* stream) {
   if (budget_ns < 1000 || budget_ns > 1000000000ull) return FA_ERR_INVALID_ARG;
   fa::selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(budget_ns);

@@ -75,4 +75,13 @@ __global__ void selftest_wait_kernel(uint64_t budget_ns) {
   wait_or_abort(ptx::smem_addr(&bar), 0, budget_ns, &abort_flag);
 }
 
+// Evaluates the FMA-pipe exp2 (ptx::exp2_fma) and the hardware ex2.approx on the same inputs, for accuracy tests.
+__global__ void selftest_exp2_kernel(const float* __restrict__ x, float* __restrict__ out_fma,
+                                     float* __restrict__ out_mufu, int n) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    out_fma[i] = ptx::exp2_fma(x[i]);
+    out_mufu[i] = ptx::ex2(x[i]);
+  }
+}
+
 }  // namespace fa

@@ -129,6 +129,13 @@ int fa_set_wait_budget_ns(uint64_t budget_ns);
  */
 int fa_selftest_wait_timeout(uint64_t budget_ns, void* stream);
 
+/*
+ * Self-test of the forward's FMA-pipe exponential (no counterpart in the paper): for n device floats x, writes the
+ * library's range-reduced polynomial 2^x to out_fma and the hardware ex2.approx result to out_mufu (device
+ * pointers, caller-owned).  Used by the tests to bound the polynomial's relative error.
+ */
+int fa_selftest_exp2(const float* x, float* out_fma, float* out_mufu, int n, void* stream);
+
 /* Size of the fixed device scratch array behind fa_bwd_noalloc: 32 MiB, held by every GPU that loads the library
  * until the process exits. */
 #define FA_NOALLOC_SCRATCH_BYTES (32u << 20)
