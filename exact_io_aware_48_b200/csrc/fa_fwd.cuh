@@ -249,7 +249,8 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t tS = tmem + lane_base + t * 128;
     const uint32_t tO = tmem + lane_base + C::kColO + t * D;
     const float scale_log2 = args.scale_log2;
-    float m_ref = -INFINITY, l_sum = 0.f;
+    float m_ref = -INFINITY;
+    ptx::f32x2 lacc[2] = {{0.f, 0.f}, {0.f, 0.f}};  // running denominator l, as four partial sums
     uint32_t s_phase = 0;
     int kidx = 0;
     bool ok = true;
@@ -276,16 +277,15 @@ __global__ void __launch_bounds__(320, 1)
         for (int i = 0; i < 128; ++i)
           if (c0 + i >= lim) s[i] = -INFINITY;
       }
-      // row max: 8 independent partial maxima, then a tree (a single serial chain would cost ~127 max latencies)
+      // row max: 8 independent partial maxima with 3-input max (two new elements per instruction), then a tree
       float pm[8];
 #pragma unroll
       for (int a = 0; a < 8; ++a) pm[a] = fmaxf(s[a], s[a + 8]);
 #pragma unroll
-      for (int i = 16; i < 128; i += 8)
+      for (int i = 16; i < 128; i += 16)
 #pragma unroll
-        for (int a = 0; a < 8; ++a) pm[a] = fmaxf(pm[a], s[i + a]);
-      const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
-                             fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+        for (int a = 0; a < 8; ++a) pm[a] = ptx::max3(pm[a], s[i + a], s[i + 8 + a]);
+      const float mx = ptx::max3(ptx::max3(pm[0], pm[1], pm[2]), ptx::max3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
       const float m_tile = mx * scale_log2;
       const bool need = m_tile > m_ref + 8.0f;
       float alpha = 1.0f;
@@ -294,24 +294,26 @@ __global__ void __launch_bounds__(320, 1)
         m_ref = m_tile;
       }
       const float m_use = (m_ref == -INFINITY) ? 0.0f : m_ref;
-      float ps[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial sums
+      if (need) {  // the running partial sums follow the reference max
+        lacc[0].x *= alpha; lacc[0].y *= alpha; lacc[1].x *= alpha; lacc[1].y *= alpha;
+      }
+      const ptx::f32x2 sc2{scale_log2, scale_log2}, nm2{-m_use, -m_use};
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t pk[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
+          const ptx::f32x2 x = ptx::fma2({s[h * 64 + 2 * i], s[h * 64 + 2 * i + 1]}, sc2, nm2);
           // one pair in kExpFmaEvery goes through the FMA-pipe exp2 so the MUFU pipe is not the only exp unit
-          const float x0 = fmaf(s[h * 64 + 2 * i], scale_log2, -m_use);
-          const float x1 = fmaf(s[h * 64 + 2 * i + 1], scale_log2, -m_use);
           const bool emu = kExpFmaEvery > 0 && (i % (kExpFmaEvery > 0 ? kExpFmaEvery : 1)) == kExpFmaEvery - 1;
-          const float p0 = emu ? ptx::exp2_fma(x0) : ptx::ex2(x0);
-          const float p1 = emu ? ptx::exp2_fma(x1) : ptx::ex2(x1);
+          const float p0 = emu ? ptx::exp2_fma(x.x) : ptx::ex2(x.x);
+          const float p1 = emu ? ptx::exp2_fma(x.y) : ptx::ex2(x.y);
           pk[i] = ptx::pack2<kBF16>(p0, p1);
-          ps[i & 3] += ptx::unpack2_sum<kBF16>(pk[i]);  // l sums the rounded P that P V uses: O stays a convex mix
+          // l sums the rounded P that P V multiplies, so O stays a convex mix of V rows
+          lacc[i & 1] = ptx::add2(lacc[i & 1], ptx::unpack2<kBF16>(pk[i]));
         }
         ptx::tmem_st32(tS + h * 32, pk);
       }
-      const float sum = (ps[0] + ps[1]) + (ps[2] + ps[3]);
       // rescale the running output (only if some row of this warp moved its reference max)
       if (kidx > 0 && __any_sync(0xffffffffu, need)) {
 #pragma unroll 1
@@ -327,7 +329,6 @@ __global__ void __launch_bounds__(320, 1)
       ptx::tmem_st_wait();
       ptx::tc_fence_before();
       ptx::mbar_arrive(ptx::smem_addr(&bar_p[t]));
-      l_sum = l_sum * alpha + sum;
       ++kidx;
     }
     // ------------------------------------------------------------------------------------------ epilogue
@@ -335,6 +336,7 @@ __global__ void __launch_bounds__(320, 1)
     if (ok) {
       ptx::tc_fence_after();
       const bool row_ok = grow < args.N && (t == 0 || has1);
+      const float l_sum = (lacc[0].x + lacc[0].y) + (lacc[1].x + lacc[1].y);
       const bool nonempty = l_sum > 0.f;
       const float inv = nonempty ? 1.0f / l_sum : 0.0f;
       uint8_t* orow = reinterpret_cast<uint8_t*>(args.o) + ((size_t)bh * args.N + grow) * D * 2;
