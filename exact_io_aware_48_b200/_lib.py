@@ -33,6 +33,7 @@ SIGNATURES = {
     "fa_selftest_wait_timeout": ([_U64, _P], _I),
     "fa_set_kernel_events": ([_I, _P, _P], _I),
     "fa_selftest_exp2": ([_P, _P, _P, _I, _P], _I),
+    "fa_set_fwd_tiles_per_cta": ([_I], _I),
     "fa_bwd_noalloc": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P, _P, _I, _P], _I),
 }
 FA_NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -154,3 +155,7 @@ def fa_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, softmax_scale,
 
 def fa_selftest_exp2(x, out_fma, out_mufu, n, stream=None) -> int:
     return load().fa_selftest_exp2(_ptr(x), _ptr(out_fma), _ptr(out_mufu), n, _stream(stream))
+
+
+def fa_set_fwd_tiles_per_cta(tiles) -> int:
+    return load().fa_set_fwd_tiles_per_cta(int(tiles))

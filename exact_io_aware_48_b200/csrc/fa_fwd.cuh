@@ -23,17 +23,22 @@
 
 namespace fa {
 
-template <int D>
+// kTiles = Q tiles per CTA.  2: one CTA per SM (320 threads, 512 TMEM columns), the two tiles ping-pong on the
+// tensor core.  1: two CTAs per SM (192 threads, 256 TMEM columns, <= half the shared memory each), the two CTAs'
+// chains interleave on the tensor core and the hardware schedules 128-row units (finer load balance).
+template <int D, int kTiles = 2>
 struct FwdCfg {
   static_assert(D == 64 || D == 128, "head dim");
+  static_assert(kTiles == 1 || kTiles == 2, "Q tiles per CTA");
   static constexpr int kSlotBytes = kTile * D * 2;  // one 128 x D tile of 16-bit values
   static constexpr int kSubTiles = D / 64;           // 128-byte-wide column blocks (one TMA box each)
-  static constexpr int kNumSlots = D == 128 ? 4 : 8;
-  static constexpr int kQBytes = 2 * kSlotBytes;
+  static constexpr int kNumSlots = kTiles == 2 ? (D == 128 ? 4 : 8) : (D == 128 ? 2 : 4);
+  static constexpr int kQBytes = kTiles * kSlotBytes;
   static constexpr int kSmemBytes = kQBytes + kNumSlots * kSlotBytes + 1024;
-  static constexpr int kThreads = 320;
-  static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kColO = 256;  // O_t at kColO + t * D
+  static constexpr int kWarpMma = 4 * kTiles, kWarpLoad = 4 * kTiles + 1;
+  static constexpr int kThreads = 32 * (4 * kTiles + 2);
+  static constexpr uint32_t kTmemCols = kTiles == 2 ? 512 : 256;
+  static constexpr uint32_t kColO = 128 * kTiles;  // O_t at kColO + t * D
 };
 
 // Every kExpFmaEvery-th pair of probabilities is exponentiated on the FMA pipe (see ptx::exp2_fma); 0 = never.
@@ -53,11 +58,11 @@ struct FwdArgs {
   uint64_t budget_ns;
 };
 
-template <int D, bool kBF16>
-__global__ void __launch_bounds__(320, 1)
+template <int D, bool kBF16, int kTiles>
+__global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
     fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                const __grid_constant__ CUtensorMap map_v, const FwdArgs args) {
-  using C = FwdCfg<D>;
+  using C = FwdCfg<D, kTiles>;
   constexpr int NS = C::kNumSlots;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -74,8 +79,8 @@ __global__ void __launch_bounds__(320, 1)
   const int pair = args.npairs - 1 - L / args.BH;  // longest (latest) Q tiles first: causal load balance
   const int bh = L % args.BH;
   const int b = bh / args.H;
-  const int qt0 = 2 * pair;
-  const bool has1 = qt0 + 1 < args.nT;
+  const int qt0 = kTiles * pair;
+  const bool has1 = kTiles == 2 && qt0 + 1 < args.nT;
   const bool causal = args.causal != 0;
   const int kv_lim = key_limit(args.key_lens, b, args.N);
   const int end0 = kv_tile_end(qt0, kv_lim, causal);
@@ -96,7 +101,7 @@ __global__ void __launch_bounds__(320, 1)
     abort_flag = 0;
     ptx::fence_barrier_init();
   }
-  if (warp == 8) {
+  if (warp == C::kWarpMma) {
     ptx::tmem_alloc(ptx::smem_addr(&tmem_base_sh), C::kTmemCols);
     ptx::tmem_relinquish();
   }
@@ -111,7 +116,7 @@ __global__ void __launch_bounds__(320, 1)
   else
     it.init_dense(end0, end1);
 
-  if (warp == 9) {
+  if (warp == C::kWarpLoad) {
     // ------------------------------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       ptx::prefetch_tensormap(&map_q);
@@ -143,7 +148,7 @@ __global__ void __launch_bounds__(320, 1)
       for (int k = (n > NS ? n - NS : 0); k < n; ++k)
         ptx::mbar_wait(ptx::smem_addr(&bar_full[k % NS]), (k / NS) & 1, args.budget_ns);
     }
-  } else if (warp == 8) {
+  } else if (warp == C::kWarpMma) {
     // ------------------------------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_s = ptx::idesc_f16(kBF16, false, false, 128, 128);
@@ -366,7 +371,7 @@ __global__ void __launch_bounds__(320, 1)
 
   ptx::tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == C::kWarpMma) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, C::kTmemCols);
   }

@@ -28,6 +28,7 @@ cudaError_t mark(int kernel, int which, cudaStream_t st) {
   return e ? cudaEventRecord(e, st) : cudaSuccess;
 }
 std::atomic<uint64_t> g_budget_ns{2000000000ull};
+std::atomic<int> g_fwd_tiles{0};  // Q tiles per forward CTA: 0 = choose per call, 1 or 2 = forced
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -122,18 +123,28 @@ cudaError_t ensure_smem(Kernel kernel, int bytes, std::atomic<uint64_t>& done_ma
   return e;
 }
 
-template <int D, bool BF>
-cudaError_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const fa::FwdArgs& a,
+template <int D, bool BF, int T>
+cudaError_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, fa::FwdArgs a,
                        cudaStream_t st) {
-  using C = fa::FwdCfg<D>;
+  using C = fa::FwdCfg<D, T>;
   static std::atomic<uint64_t> smem_set{0};
-  cudaError_t e = ensure_smem(fa::fwd_kernel<D, BF>, C::kSmemBytes, smem_set);
+  cudaError_t e = ensure_smem(fa::fwd_kernel<D, BF, T>, C::kSmemBytes, smem_set);
   if (e != cudaSuccess) return e;
+  a.npairs = (a.nT + T - 1) / T;  // work units (groups of T Q tiles) per (b, h)
   const unsigned grid = (unsigned)a.BH * (unsigned)a.npairs;
   if ((e = mark(FA_KERNEL_FWD, 0, st)) != cudaSuccess) return e;
-  fa::fwd_kernel<D, BF><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mk, mv, a);
+  fa::fwd_kernel<D, BF, T><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mk, mv, a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   return mark(FA_KERNEL_FWD, 1, st);
+}
+
+// Q tiles per forward CTA for this call (see FwdCfg).  Measured on B200 (bf16, causal): d = 64 prefers one-tile
+// CTAs (GPT-2 shape 273 vs 242 TFLOP/s, BERT shape 203 vs 188), d = 128 two-tile CTAs (N = 4096/8192/16384:
+// 763/973/1094 vs 671/930/1034).
+int fwd_tiles_for(int d) {
+  const int forced = g_fwd_tiles.load();
+  if (forced == 1 || forced == 2) return forced;
+  return d == 64 ? 1 : 2;
 }
 
 int run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
@@ -160,10 +171,17 @@ int run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, in
   a.budget_ns = g_budget_ns.load();
   cudaError_t e;
   const bool bf = dtype == FA_BF16;
-  if (d == 64)
-    e = bf ? launch_fwd<64, true>(mq, mk, mv, a, st) : launch_fwd<64, false>(mq, mk, mv, a, st);
-  else
-    e = bf ? launch_fwd<128, true>(mq, mk, mv, a, st) : launch_fwd<128, false>(mq, mk, mv, a, st);
+  if (fwd_tiles_for(d) == 2) {
+    if (d == 64)
+      e = bf ? launch_fwd<64, true, 2>(mq, mk, mv, a, st) : launch_fwd<64, false, 2>(mq, mk, mv, a, st);
+    else
+      e = bf ? launch_fwd<128, true, 2>(mq, mk, mv, a, st) : launch_fwd<128, false, 2>(mq, mk, mv, a, st);
+  } else {
+    if (d == 64)
+      e = bf ? launch_fwd<64, true, 1>(mq, mk, mv, a, st) : launch_fwd<64, false, 1>(mq, mk, mv, a, st);
+    else
+      e = bf ? launch_fwd<128, true, 1>(mq, mk, mv, a, st) : launch_fwd<128, false, 1>(mq, mk, mv, a, st);
+  }
   return e == cudaSuccess ? FA_OK : cuda_fail(e);
 }
 
@@ -321,6 +339,12 @@ int fa_set_kernel_events(int kernel, void* start_event, void* stop_event) {
   if ((start_event == nullptr) != (stop_event == nullptr)) return FA_ERR_INVALID_ARG;
   t_events[kernel][0] = static_cast<cudaEvent_t>(start_event);
   t_events[kernel][1] = static_cast<cudaEvent_t>(stop_event);
+  return FA_OK;
+}
+
+int fa_set_fwd_tiles_per_cta(int tiles) {
+  if (tiles < 0 || tiles > 2) return FA_ERR_INVALID_ARG;
+  g_fwd_tiles.store(tiles);
   return FA_OK;
 }
 

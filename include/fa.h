@@ -130,6 +130,13 @@ int fa_set_wait_budget_ns(uint64_t budget_ns);
 int fa_selftest_wait_timeout(uint64_t budget_ns, void* stream);
 
 /*
+ * Tuning override (no counterpart in the paper): number of 128-row Q tiles one forward CTA owns.  2 = one CTA per
+ * SM whose two tiles alternate on the tensor core; 1 = two one-tile CTAs per SM (finer scheduling); 0 (default) =
+ * chosen per call.  Results are identical up to rounding order.  Process-wide; FA_ERR_INVALID_ARG outside 0..2.
+ */
+int fa_set_fwd_tiles_per_cta(int tiles);
+
+/*
  * Self-test of the forward's FMA-pipe exponential (no counterpart in the paper): for n device floats x, writes the
  * library's range-reduced polynomial 2^x to out_fma and the hardware ex2.approx result to out_mufu (device
  * pointers, caller-owned).  Used by the tests to bound the polynomial's relative error.

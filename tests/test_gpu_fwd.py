@@ -89,3 +89,37 @@ def test_fwd_long_context_sampled_rows(name):
     log_errors(f"fwd_{name}_sampled", o=eo, lse=el)
     # properties that hold at any size: finite everywhere, LSE >= the diagonal score (causal), O rows bounded by V
     assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
+
+
+@pytest.fixture
+def one_tile_ctas():
+    from exact_io_aware_48_b200 import _lib
+    assert _lib.fa_set_fwd_tiles_per_cta(1) == 0
+    yield
+    assert _lib.fa_set_fwd_tiles_per_cta(0) == 0
+
+
+@pytest.mark.parametrize("B,H,N,d,dtype,causal,kl", [SMALL[i] for i in (1, 3, 5, 7, 9, 10, 11)])
+def test_fwd_one_tile_ctas(one_tile_ctas, B, H, N, d, dtype, causal, kl):
+    # the variant with one Q tile per CTA (two CTAs per SM) computes the same attention
+    q, k, v = make(B, H, N, d, dtype, N + d)
+    scale = 1.0 / np.sqrt(d)
+    o, lse = gpu_fwd(q, k, v, causal, scale, key_lens=kl)
+    o_ref, lse_ref = oracle.attn_fwd(f64(q), f64(k), f64(v), scale, causal=causal,
+                                     key_lens=None if kl is None else np.array(kl, np.int32))
+    eo = assert_o_close(o.double().numpy(), o_ref)
+    el = assert_lse_close(lse.numpy(), lse_ref)
+    log_errors(f"fwd_1tile B{B} H{H} N{N} d{d} {dtype} causal={causal} kl={kl}", o=eo, lse=el)
+
+
+def test_fwd_one_tile_ctas_blocksparse(one_tile_ctas):
+    B, H, N, d = 1, 2, 896, 128
+    q, k, v = make(B, H, N, d, "bf16", 77)
+    nT = 7
+    mask = (np.random.default_rng(5).random((nT, nT)) < 0.5).astype(np.uint8)
+    mask[np.arange(nT), np.arange(nT)] = 1
+    scale = 1.0 / np.sqrt(d)
+    o, lse = gpu_fwd(q, k, v, True, scale, block_mask=mask)
+    o_ref, lse_ref = oracle.attn_fwd(f64(q), f64(k), f64(v), scale, causal=True, block_mask=mask, tile=128)
+    assert_o_close(o.double().numpy(), o_ref)
+    assert_lse_close(lse.numpy(), lse_ref)
