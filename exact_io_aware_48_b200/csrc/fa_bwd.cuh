@@ -110,79 +110,77 @@ struct ColTileIter {
 };
 
 // ------------------------------------------------------------------------------------------------ preprocess
+// Row r of a head needs D/8 lanes (16-byte loads of 8 16-bit values), so a warp covers 32*8/D rows per pass; the
+// lanes of a row reduce with xor-shuffles inside their group.  Every padded row's dQ accumulator is zeroed with
+// 16-byte stores.  Grid-stride over all padded rows of all heads.
 template <int D, bool kBF16>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const void* __restrict__ o, const void* __restrict__ dout,
                                                       const float* __restrict__ lse, float* __restrict__ dq_acc,
                                                       float* __restrict__ lse2, float* __restrict__ Dv, int N,
                                                       int Npad, long long rows) {
-  // one warp per padded row
-  const long long row = (long long)blockIdx.x * 8 + threadIdx.x / 32;
+  constexpr int kLanesPerRow = D / 8;          // 8 or 16
+  constexpr int kRowsPerWarp = 32 / kLanesPerRow;  // 4 or 2
   const int lane = threadIdx.x % 32;
-  if (row >= rows) return;
-  const long long bh = row / Npad;
-  const int r = (int)(row % Npad);
-  float4* acc = reinterpret_cast<float4*>(dq_acc + row * D);
-  for (int c = lane; c < D / 4; c += 32) acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-  float dsum = 0.f;
-  if (r < N) {
-    const size_t off = ((size_t)bh * N + r) * D;
-    constexpr int kPer = D / 32;  // elements per lane: 2 or 4
-    const uint16_t* po = reinterpret_cast<const uint16_t*>(o) + off + lane * kPer;
-    const uint16_t* pd = reinterpret_cast<const uint16_t*>(dout) + off + lane * kPer;
-    uint32_t vo[kPer / 2], vd[kPer / 2];
-    if constexpr (kPer == 4) {
-      const uint2 a = *reinterpret_cast<const uint2*>(po), b = *reinterpret_cast<const uint2*>(pd);
-      vo[0] = a.x; vo[1] = a.y; vd[0] = b.x; vd[1] = b.y;
-    } else {
-      vo[0] = *reinterpret_cast<const uint32_t*>(po);
-      vd[0] = *reinterpret_cast<const uint32_t*>(pd);
-    }
+  const int sub = lane / kLanesPerRow, l = lane % kLanesPerRow;
+  const long long warp_global = ((long long)blockIdx.x * blockDim.x + threadIdx.x) / 32;
+  const long long nwarps = ((long long)gridDim.x * blockDim.x) / 32;
+  for (long long row0 = warp_global * kRowsPerWarp; row0 < rows; row0 += nwarps * kRowsPerWarp) {
+    const long long row = row0 + sub;
+    const bool in = row < rows;
+    const long long bh = in ? row / Npad : 0;
+    const int r = in ? (int)(row % Npad) : 0;
+    float dsum = 0.f;
+    if (in && r < N) {
+      const size_t off = ((size_t)bh * N + r) * D + (size_t)l * 8;
+      const uint4 a = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(o) + off);
+      const uint4 c = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(dout) + off);
+      const uint32_t va[4] = {a.x, a.y, a.z, a.w}, vc[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
-    for (int u = 0; u < kPer / 2; ++u) {
-      float o0, o1, d0, d1;
-      if constexpr (kBF16) {
-        o0 = __uint_as_float(vo[u] << 16); o1 = __uint_as_float(vo[u] & 0xffff0000u);
-        d0 = __uint_as_float(vd[u] << 16); d1 = __uint_as_float(vd[u] & 0xffff0000u);
-      } else {
-        o0 = __half2float(__ushort_as_half((unsigned short)(vo[u] & 0xffff)));
-        o1 = __half2float(__ushort_as_half((unsigned short)(vo[u] >> 16)));
-        d0 = __half2float(__ushort_as_half((unsigned short)(vd[u] & 0xffff)));
-        d1 = __half2float(__ushort_as_half((unsigned short)(vd[u] >> 16)));
+      for (int u = 0; u < 4; ++u) {
+        const ptx::f32x2 x = ptx::unpack2<kBF16>(va[u]), y = ptx::unpack2<kBF16>(vc[u]);
+        dsum = fmaf(x.x, y.x, dsum);
+        dsum = fmaf(x.y, y.y, dsum);
       }
-      dsum = fmaf(o0, d0, dsum);
-      dsum = fmaf(o1, d1, dsum);
     }
-  }
 #pragma unroll
-  for (int m = 16; m > 0; m >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, m);
-  if (lane == 0) {
-    float l2 = INFINITY;  // padded row or no visible key: recomputed P = exp2(x - inf) = 0
-    if (r < N) {
-      const float l = lse[(size_t)bh * N + r];
-      if (l != -INFINITY) l2 = l * 1.4426950408889634f;
+    for (int m = kLanesPerRow / 2; m > 0; m >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, m);
+    if (in) {
+      float4* acc = reinterpret_cast<float4*>(dq_acc + row * D);
+      acc[2 * l] = make_float4(0.f, 0.f, 0.f, 0.f);
+      acc[2 * l + 1] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (l == 0) {
+        float l2 = INFINITY;  // padded row or no visible key: recomputed P = exp2(x - inf) = 0
+        if (r < N) {
+          const float lv = lse[(size_t)bh * N + r];
+          if (lv != -INFINITY) l2 = lv * 1.4426950408889634f;
+        }
+        lse2[row] = l2;
+        Dv[row] = dsum;
+      }
     }
-    lse2[row] = l2;
-    Dv[row] = dsum;
   }
 }
 
 // ------------------------------------------------------------------------------------------------ dQ convert
+// Each thread converts 8 consecutive elements (two 16-byte loads, one 16-byte store) of the N-row output.
 template <int D, bool kBF16>
 __global__ void __launch_bounds__(256) bwd_dq_kernel(const float* __restrict__ dq_acc, void* __restrict__ dq, int N,
-                                                     int Npad, long long total_vec4) {
-  // each thread converts 4 consecutive elements of the N-row (unpadded) output
-  for (long long v = (long long)blockIdx.x * blockDim.x + threadIdx.x; v < total_vec4;
+                                                     int Npad, long long total_vec8) {
+  for (long long v = (long long)blockIdx.x * blockDim.x + threadIdx.x; v < total_vec8;
        v += (long long)gridDim.x * blockDim.x) {
-    const long long e = v * 4;
+    const long long e = v * 8;
     const long long row = e / D;  // bh * N + r
     const int c = (int)(e % D);
     const long long bh = row / N;
     const int r = (int)(row % N);
-    const float4 a = *reinterpret_cast<const float4*>(dq_acc + ((size_t)bh * Npad + r) * D + c);
-    uint2 out;
+    const float4* src = reinterpret_cast<const float4*>(dq_acc + ((size_t)bh * Npad + r) * D + c);
+    const float4 a = src[0], b = src[1];
+    uint4 out;
     out.x = ptx::pack2<kBF16>(a.x, a.y);
     out.y = ptx::pack2<kBF16>(a.z, a.w);
-    *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(dq) + e) = out;
+    out.z = ptx::pack2<kBF16>(b.x, b.y);
+    out.w = ptx::pack2<kBF16>(b.z, b.w);
+    *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(dq) + e) = out;
   }
 }
 
@@ -567,9 +565,10 @@ cudaError_t launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   using C = BwdCfg<D>;
   const int Npad = a.nT * kTile;
   const long long rows = (long long)a.BH * Npad;
-  bwd_pre_kernel<D, BF><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(o, dout, lse, a.dq_acc,
-                                                                     const_cast<float*>(a.lse2),
-                                                                     const_cast<float*>(a.Dv), a.N, Npad, rows);
+  const long long pre_warps = (rows + (256 / D) - 1) / (256 / D);  // rows per warp pass: 4 (d=64) or 2 (d=128)
+  const unsigned pre_blocks = (unsigned)std::min<long long>((pre_warps + 7) / 8, 148LL * 16);
+  bwd_pre_kernel<D, BF><<<pre_blocks, 256, 0, st>>>(o, dout, lse, a.dq_acc, const_cast<float*>(a.lse2),
+                                                     const_cast<float*>(a.Dv), a.N, Npad, rows);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   static std::atomic<uint64_t> smem_set{0};
@@ -584,9 +583,9 @@ cudaError_t launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   bwd_kernel<D, BF><<<(unsigned)(a.nT * a.BH), C::kThreads, C::kSmemBytes, st>>>(mq, mk, mv, mdo, mdq, a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (ev_stop && (e = cudaEventRecord(ev_stop, st)) != cudaSuccess) return e;
-  const long long total_vec4 = (long long)a.BH * a.N * D / 4;
-  const unsigned blocks = (unsigned)std::min<long long>((total_vec4 + 255) / 256, 148LL * 16);
-  bwd_dq_kernel<D, BF><<<blocks, 256, 0, st>>>(a.dq_acc, dq, a.N, Npad, total_vec4);
+  const long long total_vec8 = (long long)a.BH * a.N * D / 8;
+  const unsigned blocks = (unsigned)std::min<long long>((total_vec8 + 255) / 256, 148LL * 16);
+  bwd_dq_kernel<D, BF><<<blocks, 256, 0, st>>>(a.dq_acc, dq, a.N, Npad, total_vec8);
   return cudaGetLastError();
 }
 
