@@ -66,8 +66,44 @@ def visible_pairs(B, H, N, causal, key_lens=None, block_mask=None, tile=128):
     return total * H
 
 
+def kernel_src_hash():
+    """sha256 (first 16 hex digits) over the kernel sources and the C header, file name + contents, sorted."""
+    import glob
+    import hashlib
+    files = sorted(glob.glob(os.path.join(ROOT, "exact_io_aware_48_b200", "csrc", "*.cu"))
+                   + glob.glob(os.path.join(ROOT, "exact_io_aware_48_b200", "csrc", "*.cuh")))
+    files.append(os.path.join(ROOT, "include", "fa.h"))
+    h = hashlib.sha256()
+    for f in files:
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload, kernel):
+    """Per-launch DRAM bytes of `kernel` from the committed ncu record, or None if absent or if the kernel sources
+    changed since the counters were taken."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "kernel_traffic.json")) as f:
+            rec = json.load(f)
+        if rec.get("src_hash") != kernel_src_hash():
+            return None
+        e = rec[workload][kernel]
+        return int(e["read"]) + int(e["write"])
+    except Exception:
+        return None
+
+
 def fwd_flops(d, pairs):
     return 4.0 * d * pairs
+
+
+def algorithmic_bwd_bytes(w):
+    """Minimum DRAM bytes of one bwd_kernel launch: Q, K, V, dO read, dK, dV written (16-bit), LSE2 and D rows
+    (fp32) read.  The fp32 dQ partial sums are reduced in L2 and counted separately."""
+    e = 2
+    return 6 * w.B * w.H * w.N * w.d * e + 2 * 4 * w.B * w.H * w.nT * 128
 
 
 def peaks():
@@ -294,10 +330,12 @@ def run_ours(args):
     # roofline of the dominant kernel (bwd main: 2.5x forward FLOPs per launch), timed live by events
     kmean = float(np.mean(kern_ms))
     achieved = 2.5 * p.fwd_flops / (kmean / 1e3) / 1e12
-    roofline = {"kernel": f"bwd_kernel<{w.d},{w.dtype}>", "bound": "tensor", "achieved": round(achieved, 2),
+    kname = f"bwd_kernel<{w.d},{w.dtype}>"
+    roofline = {"kernel": kname, "bound": "tensor", "achieved": round(achieved, 2),
                 "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                 "peak_source": f"{peak_src} bf16_tflops (burst)", "kernel_ms": round(kmean, 4),
-                "traffic": None}
+                "traffic": recorded_traffic(w.name, kname), "traffic_unit": "bytes per launch (ncu DRAM read+write)",
+                "algorithmic_bytes": algorithmic_bwd_bytes(w)}
     # ------------------------------------------------------------------ end to end through the C ABI, host buffers
     e2e = run_e2e(p, stream, args, world) if args.e2e else None
 
@@ -432,12 +470,66 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_standard(args):
+    """The slide deck's suggested experiment ("Run it": a toy that materialises the attention matrix against the
+    tiled streaming version): eager PyTorch standard attention -- S = scale*QK^T written to HBM, masked, softmax, P V,
+    backward through autograd (P and dS also materialised) -- timed next to fa_fwd/fa_bwd on the same workload.
+    Prints one JSON line.  Measurement only: nothing here is on the library's path."""
+    import torch
+    from exact_io_aware_48_b200 import _lib, inputs
+    torch.cuda.set_device(0)
+    stream = torch.cuda.Stream()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    w = inputs.workloads()[args.workload]
+    p = Problem(w)
+    q = p.q.detach().clone().requires_grad_(True)
+    k = p.k.detach().clone().requires_grad_(True)
+    v = p.v.detach().clone().requires_grad_(True)
+    mask = torch.ones(w.N, w.N, device="cuda", dtype=torch.bool).tril() if w.causal else None
+
+    def std_fwd(_s=None):
+        s = torch.matmul(q, k.transpose(-1, -2)) * w.scale
+        if mask is not None:
+            s = s.masked_fill(~mask, float("-inf"))
+        return torch.matmul(torch.softmax(s.float(), dim=-1).to(q.dtype), v)
+
+    def std_step(_s=None):
+        o = std_fwd()
+        o.backward(p.do)
+        q.grad = k.grad = v.grad = None
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            std_step()
+            p.step(stream)
+    stream.synchronize()
+    n = max(5, args.steps // 2)
+    res = {}
+    for name, fn in (("standard_fwd", lambda s: std_fwd()), ("standard_fwd_bwd", std_step),
+                     ("tiled_fwd", p.fwd), ("tiled_fwd_bwd", p.step)):
+        with torch.cuda.stream(stream):
+            ms, _ = time_loop(fn, n, stream, flush)
+        res[name] = statistics.median(ms)
+    o_std = std_fwd().detach()
+    p.fwd(stream)
+    stream.synchronize()
+    err = float((o_std.float() - p.o.float()).abs().max())
+    line = {"mode": "standard-attention baseline", "workload": WORKLOAD_NAMES.get(w.name, w.name),
+            "ms": {k2: round(v2, 4) for k2, v2 in res.items()},
+            "speedup_fwd": round(res["standard_fwd"] / res["tiled_fwd"], 2),
+            "speedup_fwd_bwd": round(res["standard_fwd_bwd"] / res["tiled_fwd_bwd"], 2),
+            "max_abs_diff_O": err, "steps": n, "l2": "flushed before every timed call"}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--standard", action="store_true",
+                    help="time eager standard (materialising) attention next to the tiled kernels and exit")
     ap.add_argument("--no-targets", dest="targets", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
@@ -446,7 +538,9 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
-    if args.impl == "reference":
+    if args.standard:
+        run_standard(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)
