@@ -21,10 +21,12 @@
 // Roles in bwd_kernel (512 threads): warps 0-7 recompute P^T and dS^T (thread = key row = TMEM lane; warpgroup g
 // takes queries [64g, 64g+64), so every SM sub-partition interleaves two such warps), warps 8-11 drain dQ_i
 // (thread = query row), warp 12 issues MMAs, warp 13 issues TMA loads, warps 14-15 only pad the fourth warpgroup.
-// MMA order per Q tile i: dP^T_i, dV_i, S^T_{i+1}, dK_i, dQ_i -- the next tile's scores are computed before this
-// tile's dK/dQ so the P^T warps recompute P_{i+1} while the tensor core finishes tile i.
-// TMEM (512 columns): S^T [0,128) with P^T (16-bit pairs) over [0,32) and [64,96); dP^T [128,256); dV [256,256+d);
-// dK [256+d,256+2d); dQ_i [384,448) for d = 64, and for d = 128 (no room left) the dP^T columns once read.
+// MMA order per Q tile i, so that the P^T warps recompute P_{i+1} while the tensor core finishes tile i:
+//   d = 64:  [P^T_i] S^T_{i+1}, dV_i  [dS^T_i] dP^T_{i+1}, dK_i, dQ_i
+//   d = 128: dP^T_i [P^T_i] dV_i, S^T_{i+1} [dS^T_i] dQ_i, dK_i      ([X] = wait until X is published)
+// TMEM (512 columns): S^T [0,128); dP^T [128,256); dV [256,256+d); dK [256+d,256+2d).  d = 64: dQ_i [384,448) and
+// P^T (16-bit pairs) [448,512).  d = 128 (no room left): P^T over S^T columns [0,32) and [64,96), dQ_i in the
+// dP^T columns once read.
 #pragma once
 #include "fa_common.cuh"
 
@@ -45,6 +47,10 @@ struct BwdCfg {
   static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
   static constexpr bool kDqOwnCols = (D == 64);            // d = 64: dQ has its own columns
   static constexpr uint32_t kColDQ = kDqOwnCols ? 384 : kColDP;
+  // P^T (16-bit pairs, 64 columns): its own columns [448, 512) for d = 64, so the next S^T may overwrite the S^T
+  // columns as soon as they are read; for d = 128 inside the S^T columns ([0,32) and [64,96)).
+  static constexpr uint32_t kColPT = kDqOwnCols ? 448 : kColS;
+  static constexpr uint32_t kPtHalf = kDqOwnCols ? 32 : 64;  // column distance between the two query halves
 };
 
 // Workspace layout: dq_acc [BH][Npad][D] fp32 | lse2 [BH][Npad] fp32 | Dv [BH][Npad] fp32 (each 256-B aligned)
@@ -201,7 +207,7 @@ __global__ void __launch_bounds__(512, 1)
   uint8_t* sStage = sRing + NS * C::kSlotBytes;  // 1024-aligned: slot bytes are multiples of 1024
 
   __shared__ __align__(8) uint64_t bar_kv, bar_full[NS], bar_empty[NS], bar_s, bar_dp, bar_p, bar_ds, bar_dq_full,
-      bar_dq_free, bar_ds_free, bar_done, bar_drain;
+      bar_dq_free, bar_ds_free, bar_pt_free, bar_done, bar_drain;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
   volatile int* abortp = &abort_flag;
@@ -231,6 +237,7 @@ __global__ void __launch_bounds__(512, 1)
     ptx::mbar_init(ptx::smem_addr(&bar_dq_full), 1);
     ptx::mbar_init(ptx::smem_addr(&bar_dq_free), 128);
     ptx::mbar_init(ptx::smem_addr(&bar_ds_free), 1);
+    ptx::mbar_init(ptx::smem_addr(&bar_pt_free), 1);
     ptx::mbar_init(ptx::smem_addr(&bar_done), 1);
     ptx::mbar_init(ptx::smem_addr(&bar_drain), 1);
     abort_flag = 0;
@@ -290,25 +297,69 @@ __global__ void __launch_bounds__(512, 1)
       constexpr uint32_t id_sq = ptx::idesc_f16(kBF16, false, false, 128, 128);  // S^T, dP^T
       constexpr uint32_t id_dv = ptx::idesc_f16(kBF16, false, true, 128, D);     // dV (A from TMEM), dK
       constexpr uint32_t id_dq = ptx::idesc_f16(kBF16, true, true, 128, D);      // dQ
-      const uint32_t k_base = ptx::smem_addr(sK), v_base = ptx::smem_addr(sV), ds_base = ptx::smem_addr(sDS);
-      const uint32_t ring = ptx::smem_addr(sRing);
-      auto slot_base = [&](int k) { return ring + (k % NS) * C::kSlotBytes; };
+      // Operand descriptors are built once; each MMA advances one by a constant (K-major: +32 B per 16-element K
+      // step inside a 64-element sub-tile, +16 KB per sub-tile; M/N-major: +2 KB per 16-row K step).
+      const uint64_t dk_k = ptx::sw128_desc(ptx::smem_addr(sK), 16, 1024);      // K_j, K-major (S^T)
+      const uint64_t dk_mn = ptx::sw128_desc(ptx::smem_addr(sK), 16384, 1024);  // K_j, M/N-major (dQ)
+      const uint64_t dv_k = ptx::sw128_desc(ptx::smem_addr(sV), 16, 1024);      // V_j, K-major (dP^T)
+      const uint64_t dds_k = ptx::sw128_desc(ptx::smem_addr(sDS), 16, 1024);    // dS^T, K-major (dK)
+      const uint64_t dds_mn = ptx::sw128_desc(ptx::smem_addr(sDS), 16384, 1024);  // dS, M-major (dQ)
+      const uint64_t dring_k = ptx::sw128_desc(ptx::smem_addr(sRing), 16, 1024);
+      const uint64_t dring_mn = ptx::sw128_desc(ptx::smem_addr(sRing), 16384, 1024);
+      auto slot_off = [&](int k) { return (uint32_t)((k % NS) * C::kSlotBytes); };
       auto slot_full = [&](int k) { return ptx::smem_addr(&bar_full[k % NS]); };
       auto slot_empty = [&](int k) { return ptx::smem_addr(&bar_empty[k % NS]); };
       auto slot_phase = [&](int k) { return (uint32_t)((k / NS) & 1); };
+      constexpr auto kstep = [](int kk) { return (uint32_t)((kk / 4) * 16384 + (kk % 4) * 32); };
       // S^T = K Q^T for the Q tile in ring position kq
       auto issue_s = [&](int kq) -> bool {
         if (!wait_or_abort(slot_full(kq), slot_phase(kq), args.budget_ns, abortp)) return false;
         ptx::tc_fence_after();
-        const uint32_t q_base = slot_base(kq);
+        const uint64_t dq = ptx::desc_advance(dring_k, slot_off(kq));
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk / 4) * 16384 + (kk % 4) * 32;
-          ptx::mma_ss(tmem + C::kColS, ptx::sw128_desc(k_base + off, 16, 1024),
-                      ptx::sw128_desc(q_base + off, 16, 1024), id_sq, kk > 0 ? 1u : 0u);
-        }
+        for (int kk = 0; kk < D / 16; ++kk)
+          ptx::mma_ss(tmem + C::kColS, ptx::desc_advance(dk_k, kstep(kk)), ptx::desc_advance(dq, kstep(kk)), id_sq,
+                      kk > 0 ? 1u : 0u);
         ptx::mma_commit(ptx::smem_addr(&bar_s));
         return true;
+      };
+      // dP^T = V dO_i^T for the dO tile in ring position ko
+      auto issue_dp = [&](int ko) -> bool {
+        if (!wait_or_abort(slot_full(ko), slot_phase(ko), args.budget_ns, abortp)) return false;
+        ptx::tc_fence_after();
+        const uint64_t ddo = ptx::desc_advance(dring_k, slot_off(ko));
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          ptx::mma_ss(tmem + C::kColDP, ptx::desc_advance(dv_k, kstep(kk)), ptx::desc_advance(ddo, kstep(kk)), id_sq,
+                      kk > 0 ? 1u : 0u);
+        ptx::mma_commit(ptx::smem_addr(&bar_dp));
+        return true;
+      };
+      // dV += P^T dO_i   (P^T from TMEM, query half kk/4 at kColPT + kPtHalf*(kk/4); dO_i M/N-major)
+      auto issue_dv = [&](int ko, bool first) {
+        const uint64_t ddo = ptx::desc_advance(dring_mn, slot_off(ko));
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          ptx::mma_ts(tmem + C::kColDV, tmem + C::kColPT + (kk / 4) * C::kPtHalf + (kk % 4) * 8,
+                      ptx::desc_advance(ddo, kk * 2048), id_dv, (!first || kk > 0) ? 1u : 0u);
+        ptx::mma_commit(slot_empty(ko));  // dO_i no longer needed
+      };
+      // dK += dS^T Q_i  (dS^T K-major in shared memory, Q_i M/N-major)
+      auto issue_dk = [&](int kq, bool first) {
+        const uint64_t dq = ptx::desc_advance(dring_mn, slot_off(kq));
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          ptx::mma_ss(tmem + C::kColDK, ptx::desc_advance(dds_k, kstep(kk)), ptx::desc_advance(dq, kk * 2048), id_dv,
+                      (!first || kk > 0) ? 1u : 0u);
+        ptx::mma_commit(slot_empty(kq));  // Q_i (and its LSE2/D rows) no longer needed
+      };
+      // dQ_i = dS K_j  (dS read M-major from the dS^T tile)
+      auto issue_dq = [&]() {
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          ptx::mma_ss(tmem + C::kColDQ, ptx::desc_advance(dds_mn, kk * 2048), ptx::desc_advance(dk_mn, kk * 2048),
+                      id_dq, kk > 0 ? 1u : 0u);
+        ptx::mma_commit(ptx::smem_addr(&bar_dq_full));
       };
       bool ok = true;
       int i;
@@ -317,60 +368,62 @@ __global__ void __launch_bounds__(512, 1)
         ok = wait_or_abort(ptx::smem_addr(&bar_kv), 0, args.budget_ns, abortp);
         ptx::tc_fence_after();
         if (ok) ok = issue_s(0);
+        if (ok && C::kDqOwnCols) ok = issue_dp(1);
       }
       int iter = 0;
-      while (ok && have) {
-        const int kq = 2 * iter, ko = 2 * iter + 1;
-        const uint32_t q_base = slot_base(kq), do_base = slot_base(ko);
-        const uint32_t ph = iter & 1, ph_prev = (iter - 1) & 1;
-        // dP^T = V dO_i^T (for d = 128 its columns hold dQ_{i-1} until the drain warps have read it)
-        if (!(ok = wait_or_abort(slot_full(ko), slot_phase(ko), args.budget_ns, abortp))) break;
-        if (!C::kDqOwnCols && iter > 0 &&
-            !(ok = wait_or_abort(ptx::smem_addr(&bar_dq_free), ph_prev, args.budget_ns, abortp)))
-          break;
-        ptx::tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk / 4) * 16384 + (kk % 4) * 32;
-          ptx::mma_ss(tmem + C::kColDP, ptx::sw128_desc(v_base + off, 16, 1024),
-                      ptx::sw128_desc(do_base + off, 16, 1024), id_sq, kk > 0 ? 1u : 0u);
+      if constexpr (C::kDqOwnCols) {
+        // d = 64.  Per Q tile i:  [P^T_i published] S^T_{i+1}, dV_i  [dS^T_i published] dP^T_{i+1}, dK_i, dQ_i.
+        // The next tile's S^T and dP^T are issued as soon as their TMEM columns have been read, so the P^T/dS^T
+        // warps find them complete when they get there.
+        while (ok && have) {
+          const int kq = 2 * iter, ko = 2 * iter + 1;
+          const uint32_t ph = iter & 1, ph_prev = (iter - 1) & 1;
+          if (!(ok = wait_or_abort(ptx::smem_addr(&bar_p), ph, args.budget_ns, abortp))) break;
+          ptx::tc_fence_after();
+          int inext;
+          const bool have_next = it.next(inext);
+          if (have_next && !(ok = issue_s(kq + 2))) break;
+          issue_dv(ko, iter == 0);
+          ptx::mma_commit(ptx::smem_addr(&bar_pt_free));
+          if (!(ok = wait_or_abort(ptx::smem_addr(&bar_ds), ph, args.budget_ns, abortp))) break;
+          ptx::tc_fence_after();
+          if (have_next && !(ok = issue_dp(ko + 2))) break;
+          issue_dk(kq, iter == 0);
+          if (iter > 0 && !(ok = wait_or_abort(ptx::smem_addr(&bar_dq_free), ph_prev, args.budget_ns, abortp)))
+            break;
+          ptx::tc_fence_after();
+          issue_dq();
+          ptx::mma_commit(ptx::smem_addr(&bar_ds_free));
+          ++iter;
+          have = have_next;
+          i = inext;
         }
-        ptx::mma_commit(ptx::smem_addr(&bar_dp));
-        // dV += P^T dO_i   (P^T from TMEM; dO_i M/N-major)
-        if (!(ok = wait_or_abort(ptx::smem_addr(&bar_p), ph, args.budget_ns, abortp))) break;
-        ptx::tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk)  // queries 16kk..16kk+15: P^T half kk/4 at column 64*(kk/4)
-          ptx::mma_ts(tmem + C::kColDV, tmem + C::kColS + (kk / 4) * 64 + (kk % 4) * 8,
-                      ptx::sw128_desc(do_base + kk * 2048, 16384, 1024), id_dv, (iter > 0 || kk > 0) ? 1u : 0u);
-        ptx::mma_commit(slot_empty(ko));  // dO_i no longer needed
-        // next tile's scores (P^T_i has been consumed by dV_i, which precedes it in the MMA pipe)
-        int inext;
-        const bool have_next = it.next(inext);
-        if (have_next && !(ok = issue_s(kq + 2))) break;
-        // dK += dS^T Q_i and dQ_i = dS K_j  (dS^T in shared memory)
-        if (!(ok = wait_or_abort(ptx::smem_addr(&bar_ds), ph, args.budget_ns, abortp))) break;
-        ptx::tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk) {
-          const uint32_t off = (kk / 4) * 16384 + (kk % 4) * 32;
-          ptx::mma_ss(tmem + C::kColDK, ptx::sw128_desc(ds_base + off, 16, 1024),
-                      ptx::sw128_desc(q_base + kk * 2048, 16384, 1024), id_dv, (iter > 0 || kk > 0) ? 1u : 0u);
+      } else {
+        // d = 128.  Per Q tile i: dP^T_i, dV_i, S^T_{i+1}, dQ_i, dK_i.  dQ_i occupies the dP^T columns, so dP^T_i
+        // waits until the drain warps have read dQ_{i-1}; dQ_i goes before dK_i to start that drain sooner.
+        // S^T_{i+1} overwrites P^T_i only after dV_i (MMA order).
+        while (ok && have) {
+          const int kq = 2 * iter, ko = 2 * iter + 1;
+          const uint32_t ph = iter & 1, ph_prev = (iter - 1) & 1;
+          if (iter > 0 && !(ok = wait_or_abort(ptx::smem_addr(&bar_dq_free), ph_prev, args.budget_ns, abortp)))
+            break;
+          ptx::tc_fence_after();
+          if (!(ok = issue_dp(ko))) break;
+          if (!(ok = wait_or_abort(ptx::smem_addr(&bar_p), ph, args.budget_ns, abortp))) break;
+          ptx::tc_fence_after();
+          issue_dv(ko, iter == 0);
+          int inext;
+          const bool have_next = it.next(inext);
+          if (have_next && !(ok = issue_s(kq + 2))) break;
+          if (!(ok = wait_or_abort(ptx::smem_addr(&bar_ds), ph, args.budget_ns, abortp))) break;
+          ptx::tc_fence_after();
+          issue_dq();
+          issue_dk(kq, iter == 0);
+          ptx::mma_commit(ptx::smem_addr(&bar_ds_free));
+          ++iter;
+          have = have_next;
+          i = inext;
         }
-        ptx::mma_commit(slot_empty(kq));  // Q_i (and its LSE2/D rows) no longer needed
-        if (C::kDqOwnCols && iter > 0 &&
-            !(ok = wait_or_abort(ptx::smem_addr(&bar_dq_free), ph_prev, args.budget_ns, abortp)))
-          break;
-        ptx::tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk)
-          ptx::mma_ss(tmem + C::kColDQ, ptx::sw128_desc(ds_base + kk * 2048, 16384, 1024),
-                      ptx::sw128_desc(k_base + kk * 2048, 16384, 1024), id_dq, kk > 0 ? 1u : 0u);
-        ptx::mma_commit(ptx::smem_addr(&bar_dq_full));
-        ptx::mma_commit(ptx::smem_addr(&bar_ds_free));
-        ++iter;
-        have = have_next;
-        i = inext;
       }
       if (ok) ptx::mma_commit(ptx::smem_addr(&bar_done));
       ptx::mma_commit(ptx::smem_addr(&bar_drain));
@@ -422,9 +475,16 @@ __global__ void __launch_bounds__(512, 1)
           pk[16 * h + u] = ptx::pack2<kBF16>(p0, p1);
         }
       }
-      // P^T of this half (2 queries per 32-bit column) goes to columns [64g, 64g+32): inside the S^T columns this
-      // warpgroup has just read, never over columns the other warpgroup may still be reading
-      ptx::tmem_st32(tmem + lane_base + C::kColS + 64 * g, pk);
+      // P^T of this half (2 queries per 32-bit column) goes to kColPT + kPtHalf*g.  d = 128: inside the S^T columns
+      // this warpgroup has just read, never over columns the other warpgroup may still be reading.  d = 64: its own
+      // columns, free once dV_{i-1} has read P^T_{i-1}.
+      if (C::kDqOwnCols && iter > 0) {
+        ok = __all_sync(0xffffffffu, wait_or_abort(ptx::smem_addr(&bar_pt_free), (iter - 1) & 1, args.budget_ns,
+                                                    abortp));
+        if (!ok) break;
+        ptx::tc_fence_after();
+      }
+      ptx::tmem_st32(tmem + lane_base + C::kColPT + C::kPtHalf * g, pk);
       ptx::tmem_st_wait();
       ptx::tc_fence_before();
       ptx::mbar_arrive(ptx::smem_addr(&bar_p));
@@ -503,8 +563,8 @@ __global__ void __launch_bounds__(512, 1)
     // ------------------------------------------------------------------------------------------ dQ drain warps
     // Each warp owns 32 query rows (its TMEM lanes).  Per 32-column chunk it writes a 32 x 32 fp32 box into its
     // staging buffer in the 128-byte-swizzled layout of the dq_acc tensor map (16-byte chunk k of row r lands at
-    // k ^ (r % 8): conflict-free), then one lane issues a TMA reduce-add of that box into dq_acc.  Columns are read
-    // out of TMEM 64 at a time; the TMEM region is released as soon as the last columns are in registers.
+    // k ^ (r % 8): conflict-free), then one lane issues a TMA reduce-add of that box into dq_acc.  The TMEM region
+    // is released as soon as the last columns are in registers.
     const int wq = warp - kWarpDrain;
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
     uint8_t* stage = sStage + wq * 4096;
@@ -516,31 +576,43 @@ __global__ void __launch_bounds__(512, 1)
       if (!ok) break;
       ptx::tc_fence_after();
       const int row0 = (int)((size_t)bh * Npad + (size_t)i * kTile) + wq * 32;
+      // one 32 x 32 fp32 box: staging buffer (after the previous box has been read out of it) -> TMA reduce-add
+      auto reduce_box = [&](const uint32_t (&r)[32], int col) {
+        if (lane == 0) ptx::bulk_wait_group_read<0>();
+        __syncwarp();
 #pragma unroll
-      for (int half = 0; half < D / 64; ++half) {
-        uint32_t r[2][32];
-        ptx::tmem_ld32(tmem + lane_base + C::kColDQ + 64 * half, r[0]);
-        ptx::tmem_ld32(tmem + lane_base + C::kColDQ + 64 * half + 32, r[1]);
+        for (int k = 0; k < 8; ++k)
+          *reinterpret_cast<uint4*>(stage + lane * 128 + ((k ^ (lane & 7)) * 16)) =
+              make_uint4(r[4 * k], r[4 * k + 1], r[4 * k + 2], r[4 * k + 3]);
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          ptx::tma_reduce_add_2d(&map_dq, col, row0, stage_addr);
+          ptx::bulk_commit_group();
+        }
+      };
+      uint32_t ra[32], rb[32];
+      ptx::tmem_ld32(tmem + lane_base + C::kColDQ, ra);
+      ptx::tmem_ld32(tmem + lane_base + C::kColDQ + 32, rb);
+      ptx::tmem_ld_wait();
+      if constexpr (D == 64) {
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(ptx::smem_addr(&bar_dq_free));  // TMEM columns may now be overwritten
+        reduce_box(ra, 0);
+        reduce_box(rb, 32);
+      } else {
+        // d = 128: the columns are the next dP^T's, so all four chunks leave TMEM before any wait on the staging
+        // buffer (registers hold up to three chunks)
+        reduce_box(ra, 0);
+        uint32_t rc[32], rd[32];
+        ptx::tmem_ld32(tmem + lane_base + C::kColDQ + 64, rc);
+        ptx::tmem_ld32(tmem + lane_base + C::kColDQ + 96, rd);
         ptx::tmem_ld_wait();
-        if (half == D / 64 - 1) {
-          ptx::tc_fence_before();
-          ptx::mbar_arrive(ptx::smem_addr(&bar_dq_free));  // TMEM columns may now be overwritten
-        }
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          if (lane == 0) ptx::bulk_wait_group_read<0>();  // previous box has been read out of the staging buffer
-          __syncwarp();
-#pragma unroll
-          for (int k = 0; k < 8; ++k)
-            *reinterpret_cast<uint4*>(stage + lane * 128 + ((k ^ (lane & 7)) * 16)) =
-                make_uint4(r[cc][4 * k], r[cc][4 * k + 1], r[cc][4 * k + 2], r[cc][4 * k + 3]);
-          ptx::fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            ptx::tma_reduce_add_2d(&map_dq, 64 * half + 32 * cc, row0, stage_addr);
-            ptx::bulk_commit_group();
-          }
-        }
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(ptx::smem_addr(&bar_dq_free));
+        reduce_box(rb, 32);
+        reduce_box(rc, 64);
+        reduce_box(rd, 96);
       }
       ++iter;
     }

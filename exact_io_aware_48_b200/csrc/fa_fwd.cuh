@@ -153,7 +153,10 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
     if (lane == 0) {
       constexpr uint32_t idesc_s = ptx::idesc_f16(kBF16, false, false, 128, 128);
       constexpr uint32_t idesc_o = ptx::idesc_f16(kBF16, false, true, 128, D);
-      const uint32_t q_base = ptx::smem_addr(sQ), kv_base = ptx::smem_addr(sKV);
+      // descriptors built once and advanced by constants per MMA (one add each)
+      const uint64_t dq0 = ptx::sw128_desc(ptx::smem_addr(sQ), 16, 1024);        // Q tiles, K-major
+      const uint64_t dkv_k = ptx::sw128_desc(ptx::smem_addr(sKV), 16, 1024);     // K tiles, K-major
+      const uint64_t dkv_mn = ptx::sw128_desc(ptx::smem_addr(sKV), 16384, 1024); // V tiles, M/N-major
       bool ok = wait_or_abort(ptx::smem_addr(&bar_q), 0, args.budget_ns, abortp);
       ptx::tc_fence_after();
       int n = 0, j, fl;
@@ -164,23 +167,22 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
 
       // O_t += P_t V  (A = P_t from TMEM, B = V tile, M/N-major, 128-byte swizzle)
       auto issue_pv = [&](int t, int slot) {
-        const uint32_t v_base = kv_base + slot * C::kSlotBytes;
+        const uint64_t dv = ptx::desc_advance(dkv_mn, slot * C::kSlotBytes);
 #pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk) {
-          const uint64_t bdesc = ptx::sw128_desc(v_base + kk * 2048, 16384, 1024);
-          ptx::mma_ts(tmem + C::kColO + t * D, tmem + t * 128 + kk * 8, bdesc, idesc_o,
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          ptx::mma_ts(tmem + C::kColO + t * D, tmem + t * 128 + kk * 8, ptx::desc_advance(dv, kk * 2048), idesc_o,
                       (pv_count[t] > 0 || kk > 0) ? 1u : 0u);
-        }
         ++pv_count[t];
       };
       // S_t = Q_t K^T  (both K-major, 128-byte swizzle, K = D in steps of 16)
       auto issue_s = [&](int t, int slot) {
-        const uint32_t qa = q_base + t * C::kSlotBytes, kb = kv_base + slot * C::kSlotBytes;
+        const uint64_t dqa = ptx::desc_advance(dq0, t * C::kSlotBytes);
+        const uint64_t dkb = ptx::desc_advance(dkv_k, slot * C::kSlotBytes);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * 16384 + (kk % 4) * 32;
-          ptx::mma_ss(tmem + t * 128, ptx::sw128_desc(qa + off, 16, 1024), ptx::sw128_desc(kb + off, 16, 1024),
-                      idesc_s, kk > 0 ? 1u : 0u);
+          ptx::mma_ss(tmem + t * 128, ptx::desc_advance(dqa, off), ptx::desc_advance(dkb, off), idesc_s,
+                      kk > 0 ? 1u : 0u);
         }
       };
       // Issue the pending P V of the previous visible tile for tile t (waits for its P).

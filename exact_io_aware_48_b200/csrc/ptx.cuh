@@ -208,6 +208,11 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo_byte
   return d;
 }
 
+// The descriptor of the operand `bytes` further on (a multiple of 16).  Only the 14-bit start-address field
+// (address / 16) changes, and it cannot carry into the next field because shared-memory addresses stay below 2^18.
+// One add instead of rebuilding the descriptor: the MMA-issuing thread shares its issue slots with busy warps.
+__device__ __forceinline__ uint64_t desc_advance(uint64_t desc, uint32_t bytes) { return desc + (bytes >> 4); }
+
 // Instruction descriptor for kind::f16 with fp32 accumulation.
 //   is_bf16: operand format (1 = bf16, 0 = fp16); a_mn / b_mn: 1 if that operand is M/N-major.
 __host__ __device__ constexpr uint32_t idesc_f16(bool is_bf16, bool a_mn, bool b_mn, int M, int N) {
