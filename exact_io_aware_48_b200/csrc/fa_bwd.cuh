@@ -10,7 +10,8 @@
 //   bwd_pre_kernel   D_r = sum_j dO_rj O_rj (fp32) and LSE in base 2 for every row of a 128-padded row space
 //                    (padded rows and rows with no visible key get +inf, so their recomputed P is exactly 0);
 //                    zeroes the fp32 dQ accumulator.  HBM-bound.
-//   bwd_kernel       one CTA per 128-key tile j of one (b, h); loops over the visible 128-row Q tiles i.
+//   bwd_kernel       persistent, at most one CTA per SM; each CTA walks a share of the units (128-key tile j of
+//                    one (b, h)) and, per unit, loops over the visible 128-row Q tiles i.
 //                    Five tcgen05 GEMMs per (i, j): S^T = K Q^T and dP^T = V dO^T (recompute), dV += P^T dO (P^T read
 //                    from TMEM), dK += dS^T Q and dQ_i = dS K (dS^T staged in shared memory, used K-major for dK and
 //                    M-major for dQ).  dK, dV accumulate in TMEM for the whole loop.  Each dQ_i partial leaves
@@ -20,7 +21,9 @@
 //
 // Roles in bwd_kernel (512 threads): warps 0-7 recompute P^T and dS^T (thread = key row = TMEM lane; warpgroup g
 // takes queries [64g, 64g+64), so every SM sub-partition interleaves two such warps), warps 8-11 drain dQ_i
-// (thread = query row), warp 12 issues MMAs, warp 13 issues TMA loads, warps 14-15 only pad the fourth warpgroup.
+// (thread = query row) and write each unit's dK, dV, warp 12 issues MMAs, warp 13 issues TMA loads, warps 14-15
+// only pad the fourth warpgroup.  At d = 64 the K/V tiles are double-buffered, so the next unit's load overlaps
+// the current unit's last tiles; the epilogue overlaps the next unit's first scores.
 // MMA order per Q tile i, so that the P^T warps recompute P_{i+1} while the tensor core finishes tile i:
 //   d = 64:  [P^T_i] S^T_{i+1}, dV_i  [dS^T_i] dP^T_{i+1}, dK_i, dQ_i
 //   d = 128: dP^T_i [P^T_i] dV_i, S^T_{i+1} [dS^T_i] dQ_i, dK_i      ([X] = wait until X is published)
@@ -41,7 +44,8 @@ struct BwdCfg {
   static constexpr int kNumSlots = D == 128 ? 3 : 6;
   static constexpr int kDsBytes = kTile * kTile * 2;      // dS^T, 128 keys x 128 queries
   static constexpr int kStageBytes = 4 * 4096;             // dQ staging: one 32 x 32 fp32 box per drain warp
-  static constexpr int kSmemBytes = 2 * kTileBytes + kDsBytes + kNumSlots * kSlotBytes + kStageBytes + 1024;
+  static constexpr int kKvBufs = D == 64 ? 2 : 1;           // K/V tile buffers: d = 64 prefetches the next unit's
+  static constexpr int kSmemBytes = kKvBufs * 2 * kTileBytes + kDsBytes + kNumSlots * kSlotBytes + kStageBytes + 1024;
   static constexpr int kThreads = 512;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
@@ -191,41 +195,76 @@ __global__ void __launch_bounds__(256) bwd_dq_kernel(const float* __restrict__ d
 }
 
 // ------------------------------------------------------------------------------------------------ main kernel
+// Units of work are (K/V tile j, head bh), ordered j-major so that the longest causal columns come first.  The
+// kernel is persistent: CTA c of G takes, in round r, unit r*G + c (r even) or r*G + G-1-c (r odd); this zigzag
+// evens out the per-CTA work about as well as a greedy longest-first queue, without a global counter.
+struct UnitSeq {
+  int c, G, total, r;
+  __device__ __forceinline__ void init(int total_units) {
+    c = blockIdx.x;
+    G = gridDim.x;
+    total = total_units;
+    r = 0;
+  }
+  __device__ __forceinline__ bool next(int& L) {
+    while (r * G < total) {
+      L = r * G + ((r & 1) ? G - 1 - c : c);
+      ++r;
+      if (L < total) return true;  // the last round may be partial
+    }
+    return false;
+  }
+};
+
+struct BwdUnit {
+  int j, bh, kv_lim;
+  bool visible;  // some key of the tile is visible to someone
+};
+
+__device__ __forceinline__ BwdUnit bwd_unit(int L, const BwdArgs& a) {
+  BwdUnit u;
+  u.j = L / a.BH;
+  u.bh = L % a.BH;
+  u.kv_lim = key_limit(a.key_lens, u.bh / a.H, a.N);
+  u.visible = u.j * kTile < u.kv_lim;
+  return u;
+}
+
 template <int D, bool kBF16>
 __global__ void __launch_bounds__(512, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_do,
                const __grid_constant__ CUtensorMap map_dq, const BwdArgs args) {
   using C = BwdCfg<D>;
-  constexpr int NS = C::kNumSlots;
+  constexpr int NS = C::kNumSlots, KB = C::kKvBufs;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sK = smem;
-  uint8_t* sV = smem + C::kTileBytes;
-  uint8_t* sDS = smem + 2 * C::kTileBytes;
+  uint8_t* sKV = smem;                               // KB x (K tile, V tile)
+  uint8_t* sDS = smem + KB * 2 * C::kTileBytes;
   uint8_t* sRing = sDS + C::kDsBytes;
   uint8_t* sStage = sRing + NS * C::kSlotBytes;  // 1024-aligned: slot bytes are multiples of 1024
+  auto sK = [&](int kb) { return sKV + kb * 2 * C::kTileBytes; };
+  auto sV = [&](int kb) { return sKV + kb * 2 * C::kTileBytes + C::kTileBytes; };
 
-  __shared__ __align__(8) uint64_t bar_kv, bar_full[NS], bar_empty[NS], bar_s, bar_dp, bar_p, bar_ds, bar_dq_full,
-      bar_dq_free, bar_ds_free, bar_pt_free, bar_done, bar_drain;
+  __shared__ __align__(8) uint64_t bar_kv[KB], bar_kv_free[KB], bar_full[NS], bar_empty[NS], bar_s, bar_dp, bar_p,
+      bar_ds, bar_dq_full, bar_dq_free, bar_ds_free, bar_pt_free, bar_done, bar_acc_free, bar_drain;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
   volatile int* abortp = &abort_flag;
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  // warps 0-7: P^T/dS^T (two warpgroups, one per 64-query half), 8-11: dQ drain, 12: MMA, 13: TMA, 14-15: idle
+  // warps 0-7: P^T/dS^T (two warpgroups, one per 64-query half), 8-11: dQ drain and the dK/dV epilogue,
+  // 12: MMA, 13: TMA, 14-15: idle
   constexpr int kWarpDrain = 8, kWarpMma = 12, kWarpLoad = 13;
-  const int L = blockIdx.x;
-  const int j = L / args.BH;  // K/V tile; ascending j = longest causal work first
-  const int bh = L % args.BH;
-  const int b = bh / args.H;
   const bool causal = args.causal != 0;
-  const int kv_lim = key_limit(args.key_lens, b, args.N);
-  const bool visible = j * kTile < kv_lim;  // some key of this tile is visible to someone
   const int Npad = args.nT * kTile;
+  const int total_units = args.nT * args.BH;
 
   if (threadIdx.x == 0) {
-    ptx::mbar_init(ptx::smem_addr(&bar_kv), 1);
+    for (int k = 0; k < KB; ++k) {
+      ptx::mbar_init(ptx::smem_addr(&bar_kv[k]), 1);
+      ptx::mbar_init(ptx::smem_addr(&bar_kv_free[k]), 1);
+    }
     for (int s = 0; s < NS; ++s) {
       ptx::mbar_init(ptx::smem_addr(&bar_full[s]), 1);
       ptx::mbar_init(ptx::smem_addr(&bar_empty[s]), 1);
@@ -239,6 +278,7 @@ __global__ void __launch_bounds__(512, 1)
     ptx::mbar_init(ptx::smem_addr(&bar_ds_free), 1);
     ptx::mbar_init(ptx::smem_addr(&bar_pt_free), 1);
     ptx::mbar_init(ptx::smem_addr(&bar_done), 1);
+    ptx::mbar_init(ptx::smem_addr(&bar_acc_free), 128);
     ptx::mbar_init(ptx::smem_addr(&bar_drain), 1);
     abort_flag = 0;
     ptx::fence_barrier_init();
@@ -252,42 +292,65 @@ __global__ void __launch_bounds__(512, 1)
   ptx::tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
 
-  ColTileIter it;
-  it.init(args.col_ptr, args.row_idx, j, args.nT, causal ? j : 0, visible);
-  const int n_iters = it.count();
+  // Every role walks the same unit sequence and, per unit, the same Q-tile list; counters that index barrier
+  // phases and ring slots run on across units.  Units without a visible Q tile load and compute nothing (the
+  // epilogue writes zero dK, dV for them).
+  UnitSeq us;
+  us.init(total_units);
+  int L;
 
   if (warp == kWarpLoad) {
     // ------------------------------------------------------------------------------------------ TMA producer
-    if (lane == 0 && n_iters > 0) {
+    if (lane == 0) {
       ptx::prefetch_tensormap(&map_q);
       ptx::prefetch_tensormap(&map_do);
-      const uint32_t bkv = ptx::smem_addr(&bar_kv);
-      ptx::mbar_arrive_expect_tx(bkv, 2 * C::kTileBytes);
-      for (int c = 0; c < C::kSubTiles; ++c) {
-        ptx::tma_load_3d(ptx::smem_addr(sK + c * 16384), &map_k, 64 * c, j * kTile, bh, bkv);
-        ptx::tma_load_3d(ptx::smem_addr(sV + c * 16384), &map_v, 64 * c, j * kTile, bh, bkv);
-      }
-      int n = 0, i;
+      ptx::prefetch_tensormap(&map_k);
+      ptx::prefetch_tensormap(&map_v);
+      int n = 0, ku = 0;
       bool ok = true;
-      while (ok && it.next(i)) {
-        for (int u = 0; u < 2; ++u) {  // u = 0: Q_i (+ LSE2, D rows), u = 1: dO_i
-          const int s = n % NS;
-          const uint32_t ph = (n / NS) & 1;
-          if (!wait_or_abort(ptx::smem_addr(&bar_empty[s]), ph ^ 1, args.budget_ns, abortp)) { ok = false; break; }
-          const uint32_t bf = ptx::smem_addr(&bar_full[s]);
-          uint8_t* slot = sRing + s * C::kSlotBytes;
-          ptx::mbar_arrive_expect_tx(bf, C::kTileBytes + (u == 0 ? 1024 : 0));
-          for (int c = 0; c < C::kSubTiles; ++c)
-            ptx::tma_load_3d(ptx::smem_addr(slot + c * 16384), u == 0 ? &map_q : &map_do, 64 * c, i * kTile, bh, bf);
-          if (u == 0) {
-            const size_t row0 = (size_t)bh * Npad + (size_t)i * kTile;
-            ptx::bulk_load(ptx::smem_addr(slot + C::kTileBytes), args.lse2 + row0, 512, bf);
-            ptx::bulk_load(ptx::smem_addr(slot + C::kTileBytes + 512), args.Dv + row0, 512, bf);
-          }
-          ++n;
+      while (ok && us.next(L)) {
+        const BwdUnit u = bwd_unit(L, args);
+        ColTileIter it;
+        it.init(args.col_ptr, args.row_idx, u.j, args.nT, causal ? u.j : 0, u.visible);
+        if (it.count() == 0) continue;
+        const int kb = ku % KB;
+        // the buffer's previous K/V tiles must have been read by every MMA of their unit
+        if (ku >= KB &&
+            !wait_or_abort(ptx::smem_addr(&bar_kv_free[kb]), ((ku / KB) - 1) & 1, args.budget_ns, abortp)) {
+          ok = false;
+          break;
         }
+        const uint32_t bkv = ptx::smem_addr(&bar_kv[kb]);
+        ptx::mbar_arrive_expect_tx(bkv, 2 * C::kTileBytes);
+        for (int c = 0; c < C::kSubTiles; ++c) {
+          ptx::tma_load_3d(ptx::smem_addr(sK(kb) + c * 16384), &map_k, 64 * c, u.j * kTile, u.bh, bkv);
+          ptx::tma_load_3d(ptx::smem_addr(sV(kb) + c * 16384), &map_v, 64 * c, u.j * kTile, u.bh, bkv);
+        }
+        int i;
+        while (ok && it.next(i)) {
+          for (int v = 0; v < 2; ++v) {  // v = 0: Q_i (+ LSE2, D rows), v = 1: dO_i
+            const int s = n % NS;
+            const uint32_t ph = (n / NS) & 1;
+            if (!wait_or_abort(ptx::smem_addr(&bar_empty[s]), ph ^ 1, args.budget_ns, abortp)) { ok = false; break; }
+            const uint32_t bf = ptx::smem_addr(&bar_full[s]);
+            uint8_t* slot = sRing + s * C::kSlotBytes;
+            ptx::mbar_arrive_expect_tx(bf, C::kTileBytes + (v == 0 ? 1024 : 0));
+            for (int c = 0; c < C::kSubTiles; ++c)
+              ptx::tma_load_3d(ptx::smem_addr(slot + c * 16384), v == 0 ? &map_q : &map_do, 64 * c, i * kTile, u.bh,
+                               bf);
+            if (v == 0) {
+              const size_t row0 = (size_t)u.bh * Npad + (size_t)i * kTile;
+              ptx::bulk_load(ptx::smem_addr(slot + C::kTileBytes), args.lse2 + row0, 512, bf);
+              ptx::bulk_load(ptx::smem_addr(slot + C::kTileBytes + 512), args.Dv + row0, 512, bf);
+            }
+            ++n;
+          }
+        }
+        ++ku;
       }
-      ptx::mbar_wait(bkv, 0, args.budget_ns);
+      // Let every copy this thread issued land before the CTA can exit (immediate in the normal path).
+      for (int k = (ku > KB ? ku - KB : 0); k < ku; ++k)
+        ptx::mbar_wait(ptx::smem_addr(&bar_kv[k % KB]), (k / KB) & 1, args.budget_ns);
       for (int k = (n > NS ? n - NS : 0); k < n; ++k)
         ptx::mbar_wait(ptx::smem_addr(&bar_full[k % NS]), (k / NS) & 1, args.budget_ns);
     }
@@ -299,10 +362,7 @@ __global__ void __launch_bounds__(512, 1)
       constexpr uint32_t id_dq = ptx::idesc_f16(kBF16, true, true, 128, D);      // dQ
       // Operand descriptors are built once; each MMA advances one by a constant (K-major: +32 B per 16-element K
       // step inside a 64-element sub-tile, +16 KB per sub-tile; M/N-major: +2 KB per 16-row K step).
-      const uint64_t dk_k = ptx::sw128_desc(ptx::smem_addr(sK), 16, 1024);      // K_j, K-major (S^T)
-      const uint64_t dk_mn = ptx::sw128_desc(ptx::smem_addr(sK), 16384, 1024);  // K_j, M/N-major (dQ)
-      const uint64_t dv_k = ptx::sw128_desc(ptx::smem_addr(sV), 16, 1024);      // V_j, K-major (dP^T)
-      const uint64_t dds_k = ptx::sw128_desc(ptx::smem_addr(sDS), 16, 1024);    // dS^T, K-major (dK)
+      const uint64_t dds_k = ptx::sw128_desc(ptx::smem_addr(sDS), 16, 1024);      // dS^T, K-major (dK)
       const uint64_t dds_mn = ptx::sw128_desc(ptx::smem_addr(sDS), 16384, 1024);  // dS, M-major (dQ)
       const uint64_t dring_k = ptx::sw128_desc(ptx::smem_addr(sRing), 16, 1024);
       const uint64_t dring_mn = ptx::sw128_desc(ptx::smem_addr(sRing), 16384, 1024);
@@ -311,6 +371,7 @@ __global__ void __launch_bounds__(512, 1)
       auto slot_empty = [&](int k) { return ptx::smem_addr(&bar_empty[k % NS]); };
       auto slot_phase = [&](int k) { return (uint32_t)((k / NS) & 1); };
       constexpr auto kstep = [](int kk) { return (uint32_t)((kk / 4) * 16384 + (kk % 4) * 32); };
+      uint64_t dk_k = 0, dk_mn = 0, dv_k = 0;  // K_j (K-major for S^T, M/N-major for dQ), V_j (K-major for dP^T)
       // S^T = K Q^T for the Q tile in ring position kq
       auto issue_s = [&](int kq) -> bool {
         if (!wait_or_abort(slot_full(kq), slot_phase(kq), args.budget_ns, abortp)) return false;
@@ -361,71 +422,94 @@ __global__ void __launch_bounds__(512, 1)
                       id_dq, kk > 0 ? 1u : 0u);
         ptx::mma_commit(ptx::smem_addr(&bar_dq_full));
       };
+      int gi = 0, ku = 0;  // Q tiles and non-empty units processed so far
       bool ok = true;
-      int i;
-      bool have = it.next(i);
-      if (have) {
-        ok = wait_or_abort(ptx::smem_addr(&bar_kv), 0, args.budget_ns, abortp);
+      while (ok && us.next(L)) {
+        const BwdUnit u = bwd_unit(L, args);
+        ColTileIter it;
+        it.init(args.col_ptr, args.row_idx, u.j, args.nT, causal ? u.j : 0, u.visible);
+        if (it.count() == 0) continue;
+        const int kb = ku % KB;
+        dk_k = ptx::sw128_desc(ptx::smem_addr(sK(kb)), 16, 1024);
+        dk_mn = ptx::sw128_desc(ptx::smem_addr(sK(kb)), 16384, 1024);
+        dv_k = ptx::sw128_desc(ptx::smem_addr(sV(kb)), 16, 1024);
+        // dV and dK start over in TMEM: the epilogue must have read the previous unit's
+        auto acc_ready = [&]() -> bool {
+          if (ku == 0) return true;
+          if (!wait_or_abort(ptx::smem_addr(&bar_acc_free), (ku - 1) & 1, args.budget_ns, abortp)) return false;
+          ptx::tc_fence_after();
+          return true;
+        };
+        if (!(ok = wait_or_abort(ptx::smem_addr(&bar_kv[kb]), (ku / KB) & 1, args.budget_ns, abortp))) break;
         ptx::tc_fence_after();
-        if (ok) ok = issue_s(0);
-        if (ok && C::kDqOwnCols) ok = issue_dp(1);
-      }
-      int iter = 0;
-      if constexpr (C::kDqOwnCols) {
-        // d = 64.  Per Q tile i:  [P^T_i published] S^T_{i+1}, dV_i  [dS^T_i published] dP^T_{i+1}, dK_i, dQ_i.
-        // The next tile's S^T and dP^T are issued as soon as their TMEM columns have been read, so the P^T/dS^T
-        // warps find them complete when they get there.
-        while (ok && have) {
-          const int kq = 2 * iter, ko = 2 * iter + 1;
-          const uint32_t ph = iter & 1, ph_prev = (iter - 1) & 1;
-          if (!(ok = wait_or_abort(ptx::smem_addr(&bar_p), ph, args.budget_ns, abortp))) break;
-          ptx::tc_fence_after();
-          int inext;
-          const bool have_next = it.next(inext);
-          if (have_next && !(ok = issue_s(kq + 2))) break;
-          issue_dv(ko, iter == 0);
-          ptx::mma_commit(ptx::smem_addr(&bar_pt_free));
-          if (!(ok = wait_or_abort(ptx::smem_addr(&bar_ds), ph, args.budget_ns, abortp))) break;
-          ptx::tc_fence_after();
-          if (have_next && !(ok = issue_dp(ko + 2))) break;
-          issue_dk(kq, iter == 0);
-          if (iter > 0 && !(ok = wait_or_abort(ptx::smem_addr(&bar_dq_free), ph_prev, args.budget_ns, abortp)))
-            break;
-          ptx::tc_fence_after();
-          issue_dq();
-          ptx::mma_commit(ptx::smem_addr(&bar_ds_free));
-          ++iter;
-          have = have_next;
-          i = inext;
+        int i, li = 0;
+        bool have = it.next(i);
+        if constexpr (C::kDqOwnCols) {
+          // d = 64.  Per Q tile i:  [P^T_i published] S^T_{i+1}, dV_i  [dS^T_i published] dP^T_{i+1}, dK_i, dQ_i.
+          // The next tile's S^T and dP^T are issued as soon as their TMEM columns have been read, so the P^T/dS^T
+          // warps find them complete when they get there.
+          if (!(ok = issue_s(2 * gi))) break;
+          if (!(ok = issue_dp(2 * gi + 1))) break;
+          while (ok && have) {
+            const int kq = 2 * gi, ko = 2 * gi + 1;
+            const uint32_t ph = gi & 1, ph_prev = (gi - 1) & 1;
+            if (!(ok = wait_or_abort(ptx::smem_addr(&bar_p), ph, args.budget_ns, abortp))) break;
+            ptx::tc_fence_after();
+            int inext;
+            const bool have_next = it.next(inext);
+            if (have_next && !(ok = issue_s(kq + 2))) break;
+            if (li == 0 && !(ok = acc_ready())) break;
+            issue_dv(ko, li == 0);
+            ptx::mma_commit(ptx::smem_addr(&bar_pt_free));
+            if (!(ok = wait_or_abort(ptx::smem_addr(&bar_ds), ph, args.budget_ns, abortp))) break;
+            ptx::tc_fence_after();
+            if (have_next && !(ok = issue_dp(ko + 2))) break;
+            issue_dk(kq, li == 0);
+            if (gi > 0 && !(ok = wait_or_abort(ptx::smem_addr(&bar_dq_free), ph_prev, args.budget_ns, abortp)))
+              break;
+            ptx::tc_fence_after();
+            issue_dq();
+            ptx::mma_commit(ptx::smem_addr(&bar_ds_free));
+            ++gi;
+            ++li;
+            have = have_next;
+            i = inext;
+          }
+        } else {
+          // d = 128.  Per Q tile i: dP^T_i, dV_i, S^T_{i+1}, dQ_i, dK_i.  dQ_i occupies the dP^T columns, so dP^T_i
+          // waits until the drain warps have read dQ_{i-1}; dQ_i goes before dK_i to start that drain sooner.
+          // S^T_{i+1} overwrites P^T_i only after dV_i (MMA order).
+          if (!(ok = issue_s(2 * gi))) break;
+          while (ok && have) {
+            const int kq = 2 * gi, ko = 2 * gi + 1;
+            const uint32_t ph = gi & 1, ph_prev = (gi - 1) & 1;
+            if (gi > 0 && !(ok = wait_or_abort(ptx::smem_addr(&bar_dq_free), ph_prev, args.budget_ns, abortp)))
+              break;
+            ptx::tc_fence_after();
+            if (!(ok = issue_dp(ko))) break;
+            if (!(ok = wait_or_abort(ptx::smem_addr(&bar_p), ph, args.budget_ns, abortp))) break;
+            ptx::tc_fence_after();
+            if (li == 0 && !(ok = acc_ready())) break;
+            issue_dv(ko, li == 0);
+            int inext;
+            const bool have_next = it.next(inext);
+            if (have_next && !(ok = issue_s(kq + 2))) break;
+            if (!(ok = wait_or_abort(ptx::smem_addr(&bar_ds), ph, args.budget_ns, abortp))) break;
+            ptx::tc_fence_after();
+            issue_dq();
+            issue_dk(kq, li == 0);
+            ptx::mma_commit(ptx::smem_addr(&bar_ds_free));
+            ++gi;
+            ++li;
+            have = have_next;
+            i = inext;
+          }
         }
-      } else {
-        // d = 128.  Per Q tile i: dP^T_i, dV_i, S^T_{i+1}, dQ_i, dK_i.  dQ_i occupies the dP^T columns, so dP^T_i
-        // waits until the drain warps have read dQ_{i-1}; dQ_i goes before dK_i to start that drain sooner.
-        // S^T_{i+1} overwrites P^T_i only after dV_i (MMA order).
-        while (ok && have) {
-          const int kq = 2 * iter, ko = 2 * iter + 1;
-          const uint32_t ph = iter & 1, ph_prev = (iter - 1) & 1;
-          if (iter > 0 && !(ok = wait_or_abort(ptx::smem_addr(&bar_dq_free), ph_prev, args.budget_ns, abortp)))
-            break;
-          ptx::tc_fence_after();
-          if (!(ok = issue_dp(ko))) break;
-          if (!(ok = wait_or_abort(ptx::smem_addr(&bar_p), ph, args.budget_ns, abortp))) break;
-          ptx::tc_fence_after();
-          issue_dv(ko, iter == 0);
-          int inext;
-          const bool have_next = it.next(inext);
-          if (have_next && !(ok = issue_s(kq + 2))) break;
-          if (!(ok = wait_or_abort(ptx::smem_addr(&bar_ds), ph, args.budget_ns, abortp))) break;
-          ptx::tc_fence_after();
-          issue_dq();
-          issue_dk(kq, iter == 0);
-          ptx::mma_commit(ptx::smem_addr(&bar_ds_free));
-          ++iter;
-          have = have_next;
-          i = inext;
-        }
+        if (!ok) break;
+        ptx::mma_commit(ptx::smem_addr(&bar_done));        // dK, dV of this unit are final
+        ptx::mma_commit(ptx::smem_addr(&bar_kv_free[kb]));  // K_j, V_j no longer read
+        ++ku;
       }
-      if (ok) ptx::mma_commit(ptx::smem_addr(&bar_done));
       ptx::mma_commit(ptx::smem_addr(&bar_drain));
       ptx::mbar_wait(ptx::smem_addr(&bar_drain), 0, args.budget_ns);
     }
@@ -433,188 +517,213 @@ __global__ void __launch_bounds__(512, 1)
     // ------------------------------------------------------------------------------------------ P^T / dS^T warps
     // Warpgroup g handles queries [64g, 64g+64) of every key row; the 4 warps of a group cover the 128 key rows.
     const int g = warp / 4, quarter = warp % 4;
-    const int c = quarter * 32 + lane;         // key row within the tile == TMEM lane
-    const int gc = j * kTile + c;              // key index in the sequence
+    const int c = quarter * 32 + lane;  // key row within the tile == TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const float sl2 = args.scale_log2, sc = args.scale;
-    int n = 0, iter = 0, i;
+    int n = 0, gi = 0;
     bool ok = true;
-    while (it.next(i)) {
-      const int sq = n % NS;
-      const uint32_t phq = (n / NS) & 1;
-      n += 2;
-      const float* lse2 = reinterpret_cast<const float*>(sRing + sq * C::kSlotBytes + C::kTileBytes) + 64 * g;
-      const float* Drow = lse2 + 128;
-      const uint32_t ph = iter & 1;
-      // the LSE2/D rows came in by bulk copy with Q_i: observe that copy's barrier before reading them (the slot
-      // cannot be refilled before this iteration's dS^T is published, so the phase is stable)
-      ok = __all_sync(0xffffffffu, wait_or_abort(ptx::smem_addr(&bar_full[sq]), phq, args.budget_ns, abortp));
-      if (ok) ok = __all_sync(0xffffffffu, wait_or_abort(ptx::smem_addr(&bar_s), ph, args.budget_ns, abortp));
-      if (!ok) break;
-      ptx::tc_fence_after();
-      const bool masked = (causal && i == j) || (j + 1) * kTile > kv_lim;
-      // visible queries of key gc: r >= gc (causal) and the key itself below the key limit
-      const int rmin = causal ? gc - i * kTile - 64 * g : 0;  // first visible query column within this half
-      const bool key_ok = gc < kv_lim;
-      uint32_t pk[32];  // P^T of this half, 16-bit pairs
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t sr[32];
-        ptx::tmem_ld32(tmem + lane_base + C::kColS + 64 * g + 32 * h, sr);
-        ptx::tmem_ld_wait();
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const int r0 = 32 * h + 2 * u;
-          const float2 l2 = *reinterpret_cast<const float2*>(lse2 + r0);
-          float p0 = ptx::ex2(fmaf(__uint_as_float(sr[2 * u]), sl2, -l2.x));
-          float p1 = ptx::ex2(fmaf(__uint_as_float(sr[2 * u + 1]), sl2, -l2.y));
-          if (masked) {
-            if (!key_ok || r0 < rmin) p0 = 0.f;
-            if (!key_ok || r0 + 1 < rmin) p1 = 0.f;
-          }
-          pk[16 * h + u] = ptx::pack2<kBF16>(p0, p1);
-        }
-      }
-      // P^T of this half (2 queries per 32-bit column) goes to kColPT + kPtHalf*g.  d = 128: inside the S^T columns
-      // this warpgroup has just read, never over columns the other warpgroup may still be reading.  d = 64: its own
-      // columns, free once dV_{i-1} has read P^T_{i-1}.
-      if (C::kDqOwnCols && iter > 0) {
-        ok = __all_sync(0xffffffffu, wait_or_abort(ptx::smem_addr(&bar_pt_free), (iter - 1) & 1, args.budget_ns,
-                                                    abortp));
+    while (ok && us.next(L)) {
+      const BwdUnit u = bwd_unit(L, args);
+      ColTileIter it;
+      it.init(args.col_ptr, args.row_idx, u.j, args.nT, causal ? u.j : 0, u.visible);
+      const int j = u.j, kv_lim = u.kv_lim;
+      const int gc = j * kTile + c;  // key index in the sequence
+      int i;
+      while (it.next(i)) {
+        const int sq = n % NS;
+        const uint32_t phq = (n / NS) & 1;
+        n += 2;
+        const float* lse2 = reinterpret_cast<const float*>(sRing + sq * C::kSlotBytes + C::kTileBytes) + 64 * g;
+        const float* Drow = lse2 + 128;
+        const uint32_t ph = gi & 1;
+        // the LSE2/D rows came in by bulk copy with Q_i: observe that copy's barrier before reading them (the slot
+        // cannot be refilled before this iteration's dS^T is published, so the phase is stable)
+        ok = __all_sync(0xffffffffu, wait_or_abort(ptx::smem_addr(&bar_full[sq]), phq, args.budget_ns, abortp));
+        if (ok) ok = __all_sync(0xffffffffu, wait_or_abort(ptx::smem_addr(&bar_s), ph, args.budget_ns, abortp));
         if (!ok) break;
         ptx::tc_fence_after();
-      }
-      ptx::tmem_st32(tmem + lane_base + C::kColPT + C::kPtHalf * g, pk);
-      ptx::tmem_st_wait();
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(ptx::smem_addr(&bar_p));
-      // dS^T = P^T * (dP^T - D) * scale, written 16-bit into sub-tile g of the swizzled dS^T tile
-      ok = __all_sync(0xffffffffu, wait_or_abort(ptx::smem_addr(&bar_dp), ph, args.budget_ns, abortp));
-      if (ok && iter > 0)
-        ok = __all_sync(0xffffffffu, wait_or_abort(ptx::smem_addr(&bar_ds_free), (iter - 1) & 1, args.budget_ns,
-                                                    abortp));
-      if (!ok) break;
-      ptx::tc_fence_after();
-      uint8_t* rowp = sDS + g * 16384 + c * 128;
+        const bool masked = (causal && i == j) || (j + 1) * kTile > kv_lim;
+        // visible queries of key gc: r >= gc (causal) and the key itself below the key limit
+        const int rmin = causal ? gc - i * kTile - 64 * g : 0;  // first visible query column within this half
+        const bool key_ok = gc < kv_lim;
+        uint32_t pk[32];  // P^T of this half, 16-bit pairs
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t dr[32];
-        ptx::tmem_ld32(tmem + lane_base + C::kColDP + 64 * g + 32 * h, dr);
-        ptx::tmem_ld_wait();
-        uint32_t o[16];
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const int r0 = 32 * h + 2 * u;
-          const float2 dd = *reinterpret_cast<const float2*>(Drow + r0);
-          float p0, p1;
-          if constexpr (kBF16) {
-            p0 = __uint_as_float(pk[16 * h + u] << 16);
-            p1 = __uint_as_float(pk[16 * h + u] & 0xffff0000u);
-          } else {
-            p0 = __half2float(__ushort_as_half((unsigned short)(pk[16 * h + u] & 0xffff)));
-            p1 = __half2float(__ushort_as_half((unsigned short)(pk[16 * h + u] >> 16)));
-          }
-          const float ds0 = p0 * (__uint_as_float(dr[2 * u]) - dd.x) * sc;
-          const float ds1 = p1 * (__uint_as_float(dr[2 * u + 1]) - dd.y) * sc;
-          o[u] = ptx::pack2<kBF16>(ds0, ds1);
-        }
-        // queries 32h .. 32h+31 of this half: 16-byte chunks 4h .. 4h+3 of row c (128-byte swizzle)
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          const int chunk = (4 * h + v) ^ (c & 7);
-          *reinterpret_cast<uint4*>(rowp + chunk * 16) = make_uint4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
-        }
-      }
-      ptx::fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(ptx::smem_addr(&bar_ds));
-      ++iter;
-    }
-    // ------------------------------------------------------------------------------------------ dK, dV epilogue
-    // warpgroup 0 writes dV, warpgroup 1 writes dK (dK already carries the softmax scale through dS)
-    if (ok && n_iters > 0)
-      ok = __all_sync(0xffffffffu, wait_or_abort(ptx::smem_addr(&bar_done), 0, args.budget_ns, abortp));
-    if (ok) {
-      ptx::tc_fence_after();
-      const bool row_ok = gc < args.N;
-      uint8_t* dst_row = reinterpret_cast<uint8_t*>(g == 0 ? args.dv : args.dk) + ((size_t)bh * args.N + gc) * D * 2;
-      const uint32_t col = g == 0 ? C::kColDV : C::kColDK;
-#pragma unroll 1
-      for (int ch = 0; ch < D / 32; ++ch) {
-        uint32_t r[32];
-        if (n_iters > 0) {
-          ptx::tmem_ld32(tmem + lane_base + col + ch * 32, r);
+        for (int h = 0; h < 2; ++h) {
+          uint32_t sr[32];
+          ptx::tmem_ld32(tmem + lane_base + C::kColS + 64 * g + 32 * h, sr);
           ptx::tmem_ld_wait();
-        } else {
 #pragma unroll
-          for (int u = 0; u < 32; ++u) r[u] = 0u;  // no visible query: zero gradient
+          for (int v = 0; v < 16; ++v) {
+            const int r0 = 32 * h + 2 * v;
+            const float2 l2 = *reinterpret_cast<const float2*>(lse2 + r0);
+            float p0 = ptx::ex2(fmaf(__uint_as_float(sr[2 * v]), sl2, -l2.x));
+            float p1 = ptx::ex2(fmaf(__uint_as_float(sr[2 * v + 1]), sl2, -l2.y));
+            if (masked) {
+              if (!key_ok || r0 < rmin) p0 = 0.f;
+              if (!key_ok || r0 + 1 < rmin) p1 = 0.f;
+            }
+            pk[16 * h + v] = ptx::pack2<kBF16>(p0, p1);
+          }
         }
-        uint32_t pkd[16];
-#pragma unroll
-        for (int u = 0; u < 16; ++u) pkd[u] = ptx::pack2<kBF16>(__uint_as_float(r[2 * u]), __uint_as_float(r[2 * u + 1]));
-        if (row_ok) {
-          uint4* dst = reinterpret_cast<uint4*>(dst_row + ch * 64);
-#pragma unroll
-          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pkd[4 * v], pkd[4 * v + 1], pkd[4 * v + 2], pkd[4 * v + 3]);
+        // P^T of this half (2 queries per 32-bit column) goes to kColPT + kPtHalf*g.  d = 128: inside the S^T
+        // columns this warpgroup has just read, never over columns the other warpgroup may still be reading.
+        // d = 64: its own columns, free once dV_{i-1} has read P^T_{i-1}.
+        if (C::kDqOwnCols && gi > 0) {
+          ok = __all_sync(0xffffffffu, wait_or_abort(ptx::smem_addr(&bar_pt_free), (gi - 1) & 1, args.budget_ns,
+                                                      abortp));
+          if (!ok) break;
+          ptx::tc_fence_after();
         }
+        ptx::tmem_st32(tmem + lane_base + C::kColPT + C::kPtHalf * g, pk);
+        ptx::tmem_st_wait();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(ptx::smem_addr(&bar_p));
+        // dS^T = P^T * (dP^T - D) * scale, written 16-bit into sub-tile g of the swizzled dS^T tile
+        ok = __all_sync(0xffffffffu, wait_or_abort(ptx::smem_addr(&bar_dp), ph, args.budget_ns, abortp));
+        if (ok && gi > 0)
+          ok = __all_sync(0xffffffffu, wait_or_abort(ptx::smem_addr(&bar_ds_free), (gi - 1) & 1, args.budget_ns,
+                                                      abortp));
+        if (!ok) break;
+        ptx::tc_fence_after();
+        uint8_t* rowp = sDS + g * 16384 + c * 128;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t dr[32];
+          ptx::tmem_ld32(tmem + lane_base + C::kColDP + 64 * g + 32 * h, dr);
+          ptx::tmem_ld_wait();
+          uint32_t o[16];
+#pragma unroll
+          for (int v = 0; v < 16; ++v) {
+            const int r0 = 32 * h + 2 * v;
+            const float2 dd = *reinterpret_cast<const float2*>(Drow + r0);
+            float p0, p1;
+            if constexpr (kBF16) {
+              p0 = __uint_as_float(pk[16 * h + v] << 16);
+              p1 = __uint_as_float(pk[16 * h + v] & 0xffff0000u);
+            } else {
+              p0 = __half2float(__ushort_as_half((unsigned short)(pk[16 * h + v] & 0xffff)));
+              p1 = __half2float(__ushort_as_half((unsigned short)(pk[16 * h + v] >> 16)));
+            }
+            const float ds0 = p0 * (__uint_as_float(dr[2 * v]) - dd.x) * sc;
+            const float ds1 = p1 * (__uint_as_float(dr[2 * v + 1]) - dd.y) * sc;
+            o[v] = ptx::pack2<kBF16>(ds0, ds1);
+          }
+          // queries 32h .. 32h+31 of this half: 16-byte chunks 4h .. 4h+3 of row c (128-byte swizzle)
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const int chunk = (4 * h + v) ^ (c & 7);
+            *reinterpret_cast<uint4*>(rowp + chunk * 16) =
+                make_uint4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+          }
+        }
+        ptx::fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(ptx::smem_addr(&bar_ds));
+        ++gi;
       }
     }
   } else if (warp < kWarpMma) {
-    // ------------------------------------------------------------------------------------------ dQ drain warps
-    // Each warp owns 32 query rows (its TMEM lanes).  Per 32-column chunk it writes a 32 x 32 fp32 box into its
-    // staging buffer in the 128-byte-swizzled layout of the dq_acc tensor map (16-byte chunk k of row r lands at
+    // ------------------------------------------------------------------------------------------ drain warps
+    // dQ_i: each warp owns 32 query rows (its TMEM lanes).  Per 32-column chunk it writes a 32 x 32 fp32 box into
+    // its staging buffer in the 128-byte-swizzled layout of the dq_acc tensor map (16-byte chunk k of row r lands at
     // k ^ (r % 8): conflict-free), then one lane issues a TMA reduce-add of that box into dq_acc.  The TMEM region
     // is released as soon as the last columns are in registers.
+    // dK, dV epilogue: after a unit's last MMA each warp reads its 32 key rows of dV and dK (dK already carries
+    // the softmax scale through dS), releases the accumulators to the next unit, and stores them 16-bit.
     const int wq = warp - kWarpDrain;
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
     uint8_t* stage = sStage + wq * 4096;
     const uint32_t stage_addr = ptx::smem_addr(stage);
-    int iter = 0, i;
-    while (it.next(i)) {
-      const bool ok = __all_sync(0xffffffffu, wait_or_abort(ptx::smem_addr(&bar_dq_full), iter & 1, args.budget_ns,
-                                                            abortp));
-      if (!ok) break;
-      ptx::tc_fence_after();
-      const int row0 = (int)((size_t)bh * Npad + (size_t)i * kTile) + wq * 32;
-      // one 32 x 32 fp32 box: staging buffer (after the previous box has been read out of it) -> TMA reduce-add
-      auto reduce_box = [&](const uint32_t (&r)[32], int col) {
-        if (lane == 0) ptx::bulk_wait_group_read<0>();
-        __syncwarp();
+    int gi = 0, ku = 0;
+    bool ok = true;
+    while (ok && us.next(L)) {
+      const BwdUnit u = bwd_unit(L, args);
+      ColTileIter it;
+      it.init(args.col_ptr, args.row_idx, u.j, args.nT, causal ? u.j : 0, u.visible);
+      const int n_iters = it.count();
+      int i;
+      while (it.next(i)) {
+        ok = __all_sync(0xffffffffu, wait_or_abort(ptx::smem_addr(&bar_dq_full), gi & 1, args.budget_ns, abortp));
+        if (!ok) break;
+        ptx::tc_fence_after();
+        const int row0 = (int)((size_t)u.bh * Npad + (size_t)i * kTile) + wq * 32;
+        // one 32 x 32 fp32 box: staging buffer (after the previous box has been read out of it) -> TMA reduce-add
+        auto reduce_box = [&](const uint32_t (&r)[32], int col) {
+          if (lane == 0) ptx::bulk_wait_group_read<0>();
+          __syncwarp();
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-          *reinterpret_cast<uint4*>(stage + lane * 128 + ((k ^ (lane & 7)) * 16)) =
-              make_uint4(r[4 * k], r[4 * k + 1], r[4 * k + 2], r[4 * k + 3]);
-        ptx::fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          ptx::tma_reduce_add_2d(&map_dq, col, row0, stage_addr);
-          ptx::bulk_commit_group();
-        }
-      };
-      uint32_t ra[32], rb[32];
-      ptx::tmem_ld32(tmem + lane_base + C::kColDQ, ra);
-      ptx::tmem_ld32(tmem + lane_base + C::kColDQ + 32, rb);
-      ptx::tmem_ld_wait();
-      if constexpr (D == 64) {
-        ptx::tc_fence_before();
-        ptx::mbar_arrive(ptx::smem_addr(&bar_dq_free));  // TMEM columns may now be overwritten
-        reduce_box(ra, 0);
-        reduce_box(rb, 32);
-      } else {
-        // d = 128: the columns are the next dP^T's, so all four chunks leave TMEM before any wait on the staging
-        // buffer (registers hold up to three chunks)
-        reduce_box(ra, 0);
-        uint32_t rc[32], rd[32];
-        ptx::tmem_ld32(tmem + lane_base + C::kColDQ + 64, rc);
-        ptx::tmem_ld32(tmem + lane_base + C::kColDQ + 96, rd);
+          for (int k = 0; k < 8; ++k)
+            *reinterpret_cast<uint4*>(stage + lane * 128 + ((k ^ (lane & 7)) * 16)) =
+                make_uint4(r[4 * k], r[4 * k + 1], r[4 * k + 2], r[4 * k + 3]);
+          ptx::fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            ptx::tma_reduce_add_2d(&map_dq, col, row0, stage_addr);
+            ptx::bulk_commit_group();
+          }
+        };
+        uint32_t ra[32], rb[32];
+        ptx::tmem_ld32(tmem + lane_base + C::kColDQ, ra);
+        ptx::tmem_ld32(tmem + lane_base + C::kColDQ + 32, rb);
         ptx::tmem_ld_wait();
-        ptx::tc_fence_before();
-        ptx::mbar_arrive(ptx::smem_addr(&bar_dq_free));
-        reduce_box(rb, 32);
-        reduce_box(rc, 64);
-        reduce_box(rd, 96);
+        if constexpr (D == 64) {
+          ptx::tc_fence_before();
+          ptx::mbar_arrive(ptx::smem_addr(&bar_dq_free));  // TMEM columns may now be overwritten
+          reduce_box(ra, 0);
+          reduce_box(rb, 32);
+        } else {
+          // d = 128: the columns are the next dP^T's, so all four chunks leave TMEM before any wait on the
+          // staging buffer (registers hold up to three chunks)
+          reduce_box(ra, 0);
+          uint32_t rc[32], rd[32];
+          ptx::tmem_ld32(tmem + lane_base + C::kColDQ + 64, rc);
+          ptx::tmem_ld32(tmem + lane_base + C::kColDQ + 96, rd);
+          ptx::tmem_ld_wait();
+          ptx::tc_fence_before();
+          ptx::mbar_arrive(ptx::smem_addr(&bar_dq_free));
+          reduce_box(rb, 32);
+          reduce_box(rc, 64);
+          reduce_box(rd, 96);
+        }
+        ++gi;
       }
-      ++iter;
+      if (!ok) break;
+      // ---- dK, dV epilogue of this unit
+      const int gc = u.j * kTile + wq * 32 + lane;  // key row
+      const bool row_ok = gc < args.N;
+      uint8_t* dv_row = reinterpret_cast<uint8_t*>(args.dv) + ((size_t)u.bh * args.N + gc) * D * 2;
+      uint8_t* dk_row = reinterpret_cast<uint8_t*>(args.dk) + ((size_t)u.bh * args.N + gc) * D * 2;
+      if (n_iters > 0) {
+        ok = __all_sync(0xffffffffu, wait_or_abort(ptx::smem_addr(&bar_done), ku & 1, args.budget_ns, abortp));
+        if (!ok) break;
+        ptx::tc_fence_after();
+      }
+#pragma unroll 1
+      for (int ch = 0; ch < 2 * (D / 32); ++ch) {  // chunks of 32 columns: dV then dK
+        const bool is_dk = ch >= D / 32;
+        const int cc = is_dk ? ch - D / 32 : ch;
+        uint32_t r[32];
+        if (n_iters > 0) {
+          ptx::tmem_ld32(tmem + lane_base + (is_dk ? C::kColDK : C::kColDV) + cc * 32, r);
+          ptx::tmem_ld_wait();
+          if (ch == 2 * (D / 32) - 1) {
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(ptx::smem_addr(&bar_acc_free));  // the next unit may overwrite dK, dV
+          }
+        } else {
+#pragma unroll
+          for (int v = 0; v < 32; ++v) r[v] = 0u;  // no visible query: zero gradient
+        }
+        uint32_t pkd[16];
+#pragma unroll
+        for (int v = 0; v < 16; ++v) pkd[v] = ptx::pack2<kBF16>(__uint_as_float(r[2 * v]), __uint_as_float(r[2 * v + 1]));
+        if (row_ok) {
+          uint4* dst = reinterpret_cast<uint4*>((is_dk ? dk_row : dv_row) + cc * 64);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pkd[4 * v], pkd[4 * v + 1], pkd[4 * v + 2], pkd[4 * v + 3]);
+        }
+      }
+      if (n_iters > 0) ++ku;
     }
     if (lane == 0) ptx::bulk_wait_group<0>();  // all reductions performed before the CTA retires
     __syncwarp();
@@ -651,8 +760,17 @@ cudaError_t launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
     if (e != cudaSuccess) return e;
     smem_set.fetch_or(1ull << (dev & 63));
   }
+  // persistent: one CTA per SM at most (each walks its share of the units)
+  static std::atomic<int> sm_count[64];
+  int sms = sm_count[dev & 63].load();
+  if (sms == 0) {
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    sm_count[dev & 63].store(sms);
+  }
+  const long long units = (long long)a.nT * a.BH;
+  const unsigned grid = (unsigned)std::min<long long>(units, sms);
   if (ev_start && (e = cudaEventRecord(ev_start, st)) != cudaSuccess) return e;
-  bwd_kernel<D, BF><<<(unsigned)(a.nT * a.BH), C::kThreads, C::kSmemBytes, st>>>(mq, mk, mv, mdo, mdq, a);
+  bwd_kernel<D, BF><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mk, mv, mdo, mdq, a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (ev_stop && (e = cudaEventRecord(ev_stop, st)) != cudaSuccess) return e;
   const long long total_vec8 = (long long)a.BH * a.N * D / 8;
