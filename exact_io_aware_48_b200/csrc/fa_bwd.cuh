@@ -195,27 +195,8 @@ __global__ void __launch_bounds__(256) bwd_dq_kernel(const float* __restrict__ d
 }
 
 // ------------------------------------------------------------------------------------------------ main kernel
-// Units of work are (K/V tile j, head bh), ordered j-major so that the longest causal columns come first.  The
-// kernel is persistent: CTA c of G takes, in round r, unit r*G + c (r even) or r*G + G-1-c (r odd); this zigzag
-// evens out the per-CTA work about as well as a greedy longest-first queue, without a global counter.
-struct UnitSeq {
-  int c, G, total, r;
-  __device__ __forceinline__ void init(int total_units) {
-    c = blockIdx.x;
-    G = gridDim.x;
-    total = total_units;
-    r = 0;
-  }
-  __device__ __forceinline__ bool next(int& L) {
-    while (r * G < total) {
-      L = r * G + ((r & 1) ? G - 1 - c : c);
-      ++r;
-      if (L < total) return true;  // the last round may be partial
-    }
-    return false;
-  }
-};
-
+// Units of work are (K/V tile j, head bh), ordered j-major so that the longest causal columns come first; the
+// kernel is persistent and walks them with UnitSeq.
 struct BwdUnit {
   int j, bh, kv_lim;
   bool visible;  // some key of the tile is visible to someone
@@ -761,12 +742,8 @@ cudaError_t launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
     smem_set.fetch_or(1ull << (dev & 63));
   }
   // persistent: one CTA per SM at most (each walks its share of the units)
-  static std::atomic<int> sm_count[64];
-  int sms = sm_count[dev & 63].load();
-  if (sms == 0) {
-    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    sm_count[dev & 63].store(sms);
-  }
+  int sms = 0;
+  if ((e = device_sm_count(dev, &sms)) != cudaSuccess) return e;
   const long long units = (long long)a.nT * a.BH;
   const unsigned grid = (unsigned)std::min<long long>(units, sms);
   if (ev_start && (e = cudaEventRecord(ev_start, st)) != cudaSuccess) return e;

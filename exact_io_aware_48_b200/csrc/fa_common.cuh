@@ -112,4 +112,38 @@ struct PairTileIter {
   __device__ __forceinline__ int count(int t) const { return len[t]; }
 };
 
+// Persistent kernels: CTA c of G takes, in round r, unit r*G + c (r even) or r*G + G-1-c (r odd).  With units
+// ordered longest first, this zigzag evens out the per-CTA work about as well as a greedy longest-first queue,
+// without a global counter.
+struct UnitSeq {
+  int c, G, total, r;
+  __device__ __forceinline__ void init(int total_units) {
+    c = blockIdx.x;
+    G = gridDim.x;
+    total = total_units;
+    r = 0;
+  }
+  __device__ __forceinline__ bool next(int& L) {
+    while (r * G < total) {
+      L = r * G + ((r & 1) ? G - 1 - c : c);
+      ++r;
+      if (L < total) return true;  // the last round may be partial
+    }
+    return false;
+  }
+};
+
+// Number of SMs of the current device (cached per device).
+inline cudaError_t device_sm_count(int dev, int* sms) {
+  static std::atomic<int> cache[64];
+  int v = cache[dev & 63].load();
+  if (v == 0) {
+    const cudaError_t e = cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    cache[dev & 63].store(v);
+  }
+  *sms = v;
+  return cudaSuccess;
+}
+
 }  // namespace fa

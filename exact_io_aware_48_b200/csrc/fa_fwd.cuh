@@ -58,6 +58,33 @@ struct FwdArgs {
   uint64_t budget_ns;
 };
 
+// One unit of work: kTiles consecutive 128-row Q tiles of one (b, h).  Units are ordered longest first (latest Q
+// tiles first under the causal mask); the kernel is persistent and walks them with UnitSeq.
+struct FwdUnit {
+  int qt0, bh, kv_lim, end0, end1;
+  bool has1;
+};
+
+__device__ __forceinline__ FwdUnit fwd_unit(int L, const FwdArgs& a, int tiles) {
+  FwdUnit u;
+  const int pair = a.npairs - 1 - L / a.BH;
+  u.bh = L % a.BH;
+  u.qt0 = tiles * pair;
+  u.has1 = tiles == 2 && u.qt0 + 1 < a.nT;
+  u.kv_lim = key_limit(a.key_lens, u.bh / a.H, a.N);
+  const bool causal = a.causal != 0;
+  u.end0 = kv_tile_end(u.qt0, u.kv_lim, causal);
+  u.end1 = u.has1 ? kv_tile_end(u.qt0 + 1, u.kv_lim, causal) : 0;
+  return u;
+}
+
+__device__ __forceinline__ void fwd_tiles(PairTileIter& it, const FwdUnit& u, const FwdArgs& a) {
+  if (a.row_ptr != nullptr)
+    it.init_sparse(a.row_ptr, a.col_idx, u.qt0, a.nT, u.end0, u.end1);
+  else
+    it.init_dense(u.end0, u.end1);
+}
+
 template <int D, bool kBF16, int kTiles>
 __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
     fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
@@ -69,25 +96,19 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
   uint8_t* sQ = smem;
   uint8_t* sKV = smem + C::kQBytes;
 
-  __shared__ __align__(8) uint64_t bar_q, bar_full[NS], bar_empty[NS], bar_s[2], bar_p[2], bar_o[2], bar_drain;
+  __shared__ __align__(8) uint64_t bar_q, bar_q_free, bar_full[NS], bar_empty[NS], bar_s[2], bar_p[2], bar_o[2],
+      bar_o_free[2], bar_drain;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
   volatile int* abortp = &abort_flag;
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int L = blockIdx.x;
-  const int pair = args.npairs - 1 - L / args.BH;  // longest (latest) Q tiles first: causal load balance
-  const int bh = L % args.BH;
-  const int b = bh / args.H;
-  const int qt0 = kTiles * pair;
-  const bool has1 = kTiles == 2 && qt0 + 1 < args.nT;
   const bool causal = args.causal != 0;
-  const int kv_lim = key_limit(args.key_lens, b, args.N);
-  const int end0 = kv_tile_end(qt0, kv_lim, causal);
-  const int end1 = has1 ? kv_tile_end(qt0 + 1, kv_lim, causal) : 0;
+  const int total_units = args.npairs * args.BH;
 
   if (threadIdx.x == 0) {
     ptx::mbar_init(ptx::smem_addr(&bar_q), 1);
+    ptx::mbar_init(ptx::smem_addr(&bar_q_free), 1);
     for (int s = 0; s < NS; ++s) {
       ptx::mbar_init(ptx::smem_addr(&bar_full[s]), 1);
       ptx::mbar_init(ptx::smem_addr(&bar_empty[s]), 1);
@@ -96,6 +117,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
       ptx::mbar_init(ptx::smem_addr(&bar_s[t]), 1);
       ptx::mbar_init(ptx::smem_addr(&bar_p[t]), 128);
       ptx::mbar_init(ptx::smem_addr(&bar_o[t]), 1);
+      ptx::mbar_init(ptx::smem_addr(&bar_o_free[t]), 128);
     }
     ptx::mbar_init(ptx::smem_addr(&bar_drain), 1);
     abort_flag = 0;
@@ -110,11 +132,11 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
   ptx::tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
 
-  PairTileIter it;
-  if (args.row_ptr != nullptr)
-    it.init_sparse(args.row_ptr, args.col_idx, qt0, args.nT, end0, end1);
-  else
-    it.init_dense(end0, end1);
+  // Every role walks the same unit sequence and, per unit, the same K/V tile list; barrier phases and ring
+  // positions run on across units.
+  UnitSeq us;
+  us.init(total_units);
+  int L;
 
   if (warp == C::kWarpLoad) {
     // ------------------------------------------------------------------------------------------ TMA producer
@@ -123,28 +145,36 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
       ptx::prefetch_tensormap(&map_k);
       ptx::prefetch_tensormap(&map_v);
       const uint32_t bq = ptx::smem_addr(&bar_q);
-      ptx::mbar_arrive_expect_tx(bq, (has1 ? 2 : 1) * C::kSlotBytes);
-      for (int t = 0; t < (has1 ? 2 : 1); ++t)
-        for (int c = 0; c < C::kSubTiles; ++c)
-          ptx::tma_load_3d(ptx::smem_addr(sQ + t * C::kSlotBytes + c * 16384), &map_q, 64 * c, (qt0 + t) * kTile,
-                           bh, bq);
-      int n = 0, j, fl;
+      int n = 0, ku = 0, j, fl;
       bool ok = true;
-      while (ok && it.next(j, fl)) {
-        for (int kv = 0; kv < 2; ++kv) {
-          const int s = n % NS;
-          const uint32_t ph = (n / NS) & 1;
-          if (!wait_or_abort(ptx::smem_addr(&bar_empty[s]), ph ^ 1, args.budget_ns, abortp)) { ok = false; break; }
-          const uint32_t bf = ptx::smem_addr(&bar_full[s]);
-          ptx::mbar_arrive_expect_tx(bf, C::kSlotBytes);
-          const CUtensorMap* map = kv == 0 ? &map_k : &map_v;
+      while (ok && us.next(L)) {
+        const FwdUnit u = fwd_unit(L, args, kTiles);
+        PairTileIter it;
+        fwd_tiles(it, u, args);
+        // the Q buffer is free once every S MMA of the previous unit has completed
+        if (ku > 0 && !wait_or_abort(ptx::smem_addr(&bar_q_free), (ku - 1) & 1, args.budget_ns, abortp)) break;
+        ptx::mbar_arrive_expect_tx(bq, (u.has1 ? 2 : 1) * C::kSlotBytes);
+        for (int t = 0; t < (u.has1 ? 2 : 1); ++t)
           for (int c = 0; c < C::kSubTiles; ++c)
-            ptx::tma_load_3d(ptx::smem_addr(sKV + s * C::kSlotBytes + c * 16384), map, 64 * c, j * kTile, bh, bf);
-          ++n;
+            ptx::tma_load_3d(ptx::smem_addr(sQ + t * C::kSlotBytes + c * 16384), &map_q, 64 * c,
+                             (u.qt0 + t) * kTile, u.bh, bq);
+        while (ok && it.next(j, fl)) {
+          for (int kv = 0; kv < 2; ++kv) {
+            const int s = n % NS;
+            const uint32_t ph = (n / NS) & 1;
+            if (!wait_or_abort(ptx::smem_addr(&bar_empty[s]), ph ^ 1, args.budget_ns, abortp)) { ok = false; break; }
+            const uint32_t bf = ptx::smem_addr(&bar_full[s]);
+            ptx::mbar_arrive_expect_tx(bf, C::kSlotBytes);
+            const CUtensorMap* map = kv == 0 ? &map_k : &map_v;
+            for (int c = 0; c < C::kSubTiles; ++c)
+              ptx::tma_load_3d(ptx::smem_addr(sKV + s * C::kSlotBytes + c * 16384), map, 64 * c, j * kTile, u.bh, bf);
+            ++n;
+          }
         }
+        ++ku;
       }
       // Let every copy this thread issued land before the CTA can exit (immediate in the normal path).
-      ptx::mbar_wait(bq, 0, args.budget_ns);
+      if (ku > 0) ptx::mbar_wait(bq, (ku - 1) & 1, args.budget_ns);
       for (int k = (n > NS ? n - NS : 0); k < n; ++k)
         ptx::mbar_wait(ptx::smem_addr(&bar_full[k % NS]), (k / NS) & 1, args.budget_ns);
     }
@@ -157,9 +187,8 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
       const uint64_t dq0 = ptx::sw128_desc(ptx::smem_addr(sQ), 16, 1024);        // Q tiles, K-major
       const uint64_t dkv_k = ptx::sw128_desc(ptx::smem_addr(sKV), 16, 1024);     // K tiles, K-major
       const uint64_t dkv_mn = ptx::sw128_desc(ptx::smem_addr(sKV), 16384, 1024); // V tiles, M/N-major
-      bool ok = wait_or_abort(ptx::smem_addr(&bar_q), 0, args.budget_ns, abortp);
-      ptx::tc_fence_after();
-      int n = 0, j, fl;
+      bool ok = true;
+      int n = 0, ku = 0, j, fl;
       int pend_slot = 0, pend_flags = 0;
       uint32_t pend_phase = 0;
       uint32_t p_phase[2] = {0, 0};
@@ -185,7 +214,8 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
                       kk > 0 ? 1u : 0u);
         }
       };
-      // Issue the pending P V of the previous visible tile for tile t (waits for its P).
+      // Issue the pending P V of the previous visible tile for tile t (waits for its P).  The first P V of a unit
+      // overwrites O_t, so it also waits until the epilogue has read the previous unit's O_t.
       bool v_ready = false;
       auto flush_pv = [&](int t) -> bool {
         if (!(pend_flags & (1 << t))) return true;
@@ -195,51 +225,64 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
           if (!wait_or_abort(ptx::smem_addr(&bar_full[pend_slot]), pend_phase, args.budget_ns, abortp)) return false;
           v_ready = true;
         }
+        if (pv_count[t] == 0 && ku > 0 &&
+            !wait_or_abort(ptx::smem_addr(&bar_o_free[t]), (ku - 1) & 1, args.budget_ns, abortp))
+          return false;
         ptx::tc_fence_after();
         issue_pv(t, pend_slot);
         return true;
       };
 
-      while (ok && it.next(j, fl)) {
-        const int sK = n % NS;
-        const uint32_t phK = (n / NS) & 1;
-        ++n;
-        const int sV = n % NS;
-        const uint32_t phV = (n / NS) & 1;
-        ++n;
-        bool k_ready = false;
+      while (ok && us.next(L)) {
+        const FwdUnit u = fwd_unit(L, args, kTiles);
+        PairTileIter it;
+        fwd_tiles(it, u, args);
+        if (!(ok = wait_or_abort(ptx::smem_addr(&bar_q), ku & 1, args.budget_ns, abortp))) break;
+        ptx::tc_fence_after();
+        pend_flags = 0;
+        pv_count[0] = pv_count[1] = 0;
+        v_ready = false;
+        while (ok && it.next(j, fl)) {
+          const int sK = n % NS;
+          const uint32_t phK = (n / NS) & 1;
+          ++n;
+          const int sV = n % NS;
+          const uint32_t phV = (n / NS) & 1;
+          ++n;
+          bool k_ready = false;
 #pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          if (ok) ok = flush_pv(t);
-          if (ok && (fl & (1 << t))) {
-            if (!k_ready) {
-              ok = wait_or_abort(ptx::smem_addr(&bar_full[sK]), phK, args.budget_ns, abortp);
-              ptx::tc_fence_after();
-              k_ready = true;
-            }
-            if (ok) {
-              issue_s(t, sK);
-              ptx::mma_commit(ptx::smem_addr(&bar_s[t]));
+          for (int t = 0; t < 2; ++t) {
+            if (ok) ok = flush_pv(t);
+            if (ok && (fl & (1 << t))) {
+              if (!k_ready) {
+                ok = wait_or_abort(ptx::smem_addr(&bar_full[sK]), phK, args.budget_ns, abortp);
+                ptx::tc_fence_after();
+                k_ready = true;
+              }
+              if (ok) {
+                issue_s(t, sK);
+                ptx::mma_commit(ptx::smem_addr(&bar_s[t]));
+              }
             }
           }
+          if (!ok) break;
+          if (pend_flags) ptx::mma_commit(ptx::smem_addr(&bar_empty[pend_slot]));  // previous V consumed
+          ptx::mma_commit(ptx::smem_addr(&bar_empty[sK]));                          // this K consumed
+          pend_slot = sV;
+          pend_phase = phV;
+          pend_flags = fl;
+          v_ready = false;
         }
         if (!ok) break;
-        if (pend_flags) ptx::mma_commit(ptx::smem_addr(&bar_empty[pend_slot]));  // previous V consumed
-        ptx::mma_commit(ptx::smem_addr(&bar_empty[sK]));                          // this K consumed
-        pend_slot = sV;
-        pend_phase = phV;
-        pend_flags = fl;
-        v_ready = false;
-      }
-      if (ok) {
+        ptx::mma_commit(ptx::smem_addr(&bar_q_free));  // every S of this unit issued: Q may be replaced
 #pragma unroll
         for (int t = 0; t < 2; ++t)
           if (ok) ok = flush_pv(t);
-        if (ok && pend_flags) ptx::mma_commit(ptx::smem_addr(&bar_empty[pend_slot]));
-        if (ok) {
-          ptx::mma_commit(ptx::smem_addr(&bar_o[0]));
-          ptx::mma_commit(ptx::smem_addr(&bar_o[1]));
-        }
+        if (!ok) break;
+        if (pend_flags) ptx::mma_commit(ptx::smem_addr(&bar_empty[pend_slot]));
+        ptx::mma_commit(ptx::smem_addr(&bar_o[0]));
+        ptx::mma_commit(ptx::smem_addr(&bar_o[1]));
+        ++ku;
       }
       // No MMA may still be running when the tensor memory is released.
       ptx::mma_commit(ptx::smem_addr(&bar_drain));
@@ -249,109 +292,122 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
     // ------------------------------------------------------------------------------------------ softmax warps
     const int t = warp / 4;
     const int quarter = warp % 4;
-    const int qt = qt0 + t;
     const int row = quarter * 32 + lane;  // row within the Q tile == TMEM lane
-    const int grow = qt * kTile + row;    // row within the sequence
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t tS = tmem + lane_base + t * 128;
     const uint32_t tO = tmem + lane_base + C::kColO + t * D;
     const float scale_log2 = args.scale_log2;
-    float m_ref = -INFINITY;
-    ptx::f32x2 lacc[2] = {{0.f, 0.f}, {0.f, 0.f}};  // running denominator l, as four partial sums
     uint32_t s_phase = 0;
-    int kidx = 0;
+    int ku = 0;
     bool ok = true;
-    int j, fl;
-    while (it.next(j, fl)) {
-      if (!(fl & (1 << t))) continue;
-      // every lane waits; the verdict is made warp-uniform before any warp-collective TMEM access
-      ok = __all_sync(0xffffffffu, wait_or_abort(ptx::smem_addr(&bar_s[t]), s_phase, args.budget_ns, abortp));
-      if (!ok) break;
-      s_phase ^= 1;
-      ptx::tc_fence_after();
-      uint32_t sr[128];
-      ptx::tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-      ptx::tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-      ptx::tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
-      ptx::tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
-      ptx::tmem_ld_wait();
-      float* s = reinterpret_cast<float*>(sr);
-      // element masks only on tiles that straddle the diagonal or the key limit
-      if ((causal && j >= qt) || (j + 1) * kTile > kv_lim) {
-        const int c0 = j * kTile;
-        const int lim = causal ? min(kv_lim, grow + 1) : kv_lim;  // keys c < lim are visible
+    while (ok && us.next(L)) {
+      const FwdUnit u = fwd_unit(L, args, kTiles);
+      PairTileIter it;
+      fwd_tiles(it, u, args);
+      const int qt = u.qt0 + t;
+      const int grow = qt * kTile + row;  // row within the sequence
+      const int kv_lim = u.kv_lim;
+      float m_ref = -INFINITY;
+      ptx::f32x2 lacc[2] = {{0.f, 0.f}, {0.f, 0.f}};  // running denominator l, as four partial sums
+      int kidx = 0;
+      int j, fl;
+      while (it.next(j, fl)) {
+        if (!(fl & (1 << t))) continue;
+        // every lane waits; the verdict is made warp-uniform before any warp-collective TMEM access
+        ok = __all_sync(0xffffffffu, wait_or_abort(ptx::smem_addr(&bar_s[t]), s_phase, args.budget_ns, abortp));
+        if (!ok) break;
+        s_phase ^= 1;
+        ptx::tc_fence_after();
+        uint32_t sr[128];
+        ptx::tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+        ptx::tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+        ptx::tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+        ptx::tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+        ptx::tmem_ld_wait();
+        float* s = reinterpret_cast<float*>(sr);
+        // element masks only on tiles that straddle the diagonal or the key limit
+        if ((causal && j >= qt) || (j + 1) * kTile > kv_lim) {
+          const int c0 = j * kTile;
+          const int lim = causal ? min(kv_lim, grow + 1) : kv_lim;  // keys c < lim are visible
 #pragma unroll
-        for (int i = 0; i < 128; ++i)
-          if (c0 + i >= lim) s[i] = -INFINITY;
-      }
-      // row max: 8 independent partial maxima with 3-input max (two new elements per instruction), then a tree
-      float pm[8];
-#pragma unroll
-      for (int a = 0; a < 8; ++a) pm[a] = fmaxf(s[a], s[a + 8]);
-#pragma unroll
-      for (int i = 16; i < 128; i += 16)
-#pragma unroll
-        for (int a = 0; a < 8; ++a) pm[a] = ptx::max3(pm[a], s[i + a], s[i + 8 + a]);
-      const float mx = ptx::max3(ptx::max3(pm[0], pm[1], pm[2]), ptx::max3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
-      const float m_tile = mx * scale_log2;
-      const bool need = m_tile > m_ref + 8.0f;
-      float alpha = 1.0f;
-      if (need) {
-        alpha = ptx::ex2(m_ref - m_tile);  // 0 when nothing was visible before
-        m_ref = m_tile;
-      }
-      const float m_use = (m_ref == -INFINITY) ? 0.0f : m_ref;
-      if (need) {  // the running partial sums follow the reference max
-        lacc[0].x *= alpha; lacc[0].y *= alpha; lacc[1].x *= alpha; lacc[1].y *= alpha;
-      }
-      const ptx::f32x2 sc2{scale_log2, scale_log2}, nm2{-m_use, -m_use};
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const ptx::f32x2 x = ptx::fma2({s[h * 64 + 2 * i], s[h * 64 + 2 * i + 1]}, sc2, nm2);
-          // one pair in kExpFmaEvery goes through the FMA-pipe exp2 so the MUFU pipe is not the only exp unit
-          const bool emu = kExpFmaEvery > 0 && (i % (kExpFmaEvery > 0 ? kExpFmaEvery : 1)) == kExpFmaEvery - 1;
-          const float p0 = emu ? ptx::exp2_fma(x.x) : ptx::ex2(x.x);
-          const float p1 = emu ? ptx::exp2_fma(x.y) : ptx::ex2(x.y);
-          pk[i] = ptx::pack2<kBF16>(p0, p1);
-          // l sums the rounded P that P V multiplies, so O stays a convex mix of V rows
-          lacc[i & 1] = ptx::add2(lacc[i & 1], ptx::unpack2<kBF16>(pk[i]));
+          for (int i = 0; i < 128; ++i)
+            if (c0 + i >= lim) s[i] = -INFINITY;
         }
-        ptx::tmem_st32(tS + h * 32, pk);
-      }
-      // rescale the running output (only if some row of this warp moved its reference max)
-      if (kidx > 0 && __any_sync(0xffffffffu, need)) {
+        // row max: 8 independent partial maxima with 3-input max (two new elements per instruction), then a tree
+        float pm[8];
+#pragma unroll
+        for (int a = 0; a < 8; ++a) pm[a] = fmaxf(s[a], s[a + 8]);
+#pragma unroll
+        for (int i = 16; i < 128; i += 16)
+#pragma unroll
+          for (int a = 0; a < 8; ++a) pm[a] = ptx::max3(pm[a], s[i + a], s[i + 8 + a]);
+        const float mx =
+            ptx::max3(ptx::max3(pm[0], pm[1], pm[2]), ptx::max3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
+        const float m_tile = mx * scale_log2;
+        const bool need = m_tile > m_ref + 8.0f;
+        float alpha = 1.0f;
+        if (need) {
+          alpha = ptx::ex2(m_ref - m_tile);  // 0 when nothing was visible before
+          m_ref = m_tile;
+        }
+        const float m_use = (m_ref == -INFINITY) ? 0.0f : m_ref;
+        if (need) {  // the running partial sums follow the reference max
+          lacc[0].x *= alpha; lacc[0].y *= alpha; lacc[1].x *= alpha; lacc[1].y *= alpha;
+        }
+        const ptx::f32x2 sc2{scale_log2, scale_log2}, nm2{-m_use, -m_use};
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const ptx::f32x2 x = ptx::fma2({s[h * 64 + 2 * i], s[h * 64 + 2 * i + 1]}, sc2, nm2);
+            // one pair in kExpFmaEvery goes through the FMA-pipe exp2 so the MUFU pipe is not the only exp unit
+            const bool emu = kExpFmaEvery > 0 && (i % (kExpFmaEvery > 0 ? kExpFmaEvery : 1)) == kExpFmaEvery - 1;
+            const float p0 = emu ? ptx::exp2_fma(x.x) : ptx::ex2(x.x);
+            const float p1 = emu ? ptx::exp2_fma(x.y) : ptx::ex2(x.y);
+            pk[i] = ptx::pack2<kBF16>(p0, p1);
+            // l sums the rounded P that P V multiplies, so O stays a convex mix of V rows
+            lacc[i & 1] = ptx::add2(lacc[i & 1], ptx::unpack2<kBF16>(pk[i]));
+          }
+          ptx::tmem_st32(tS + h * 32, pk);
+        }
+        // rescale the running output (only if some row of this warp moved its reference max)
+        if (kidx > 0 && __any_sync(0xffffffffu, need)) {
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t orr[32];
-          ptx::tmem_ld32(tO + c * 32, orr);
-          ptx::tmem_ld_wait();
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t orr[32];
+            ptx::tmem_ld32(tO + c * 32, orr);
+            ptx::tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) orr[i] = __float_as_uint(__uint_as_float(orr[i]) * alpha);
-          ptx::tmem_st32(tO + c * 32, orr);
+            for (int i = 0; i < 32; ++i) orr[i] = __float_as_uint(__uint_as_float(orr[i]) * alpha);
+            ptx::tmem_st32(tO + c * 32, orr);
+          }
         }
+        ptx::tmem_st_wait();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(ptx::smem_addr(&bar_p[t]));
+        ++kidx;
       }
-      ptx::tmem_st_wait();
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(ptx::smem_addr(&bar_p[t]));
-      ++kidx;
-    }
-    // ------------------------------------------------------------------------------------------ epilogue
-    if (ok) ok = __all_sync(0xffffffffu, wait_or_abort(ptx::smem_addr(&bar_o[t]), 0, args.budget_ns, abortp));
-    if (ok) {
+      if (!ok) break;
+      // ---------------------------------------------------------------------------------------- epilogue
+      // O_t is read out of TMEM and released to the next unit's first P V before it is normalised and stored.
+      ok = __all_sync(0xffffffffu, wait_or_abort(ptx::smem_addr(&bar_o[t]), ku & 1, args.budget_ns, abortp));
+      if (!ok) break;
       ptx::tc_fence_after();
-      const bool row_ok = grow < args.N && (t == 0 || has1);
+      const bool row_ok = grow < args.N && (t == 0 || u.has1);
       const float l_sum = (lacc[0].x + lacc[0].y) + (lacc[1].x + lacc[1].y);
       const bool nonempty = l_sum > 0.f;
       const float inv = nonempty ? 1.0f / l_sum : 0.0f;
-      uint8_t* orow = reinterpret_cast<uint8_t*>(args.o) + ((size_t)bh * args.N + grow) * D * 2;
+      uint8_t* orow = reinterpret_cast<uint8_t*>(args.o) + ((size_t)u.bh * args.N + grow) * D * 2;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t orr[32];
         ptx::tmem_ld32(tO + c * 32, orr);
         ptx::tmem_ld_wait();
+        if (c == D / 32 - 1) {
+          ptx::tc_fence_before();
+          ptx::mbar_arrive(ptx::smem_addr(&bar_o_free[t]));
+        }
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
@@ -366,8 +422,9 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
         }
       }
       if (row_ok)
-        args.lse[(size_t)bh * args.N + grow] = nonempty ? (m_ref + __log2f(l_sum)) * 0.69314718055994530942f
-                                                        : -INFINITY;
+        args.lse[(size_t)u.bh * args.N + grow] = nonempty ? (m_ref + __log2f(l_sum)) * 0.69314718055994530942f
+                                                          : -INFINITY;
+      ++ku;
     }
   }
 

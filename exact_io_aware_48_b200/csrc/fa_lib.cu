@@ -131,7 +131,12 @@ cudaError_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   cudaError_t e = ensure_smem(fa::fwd_kernel<D, BF, T>, C::kSmemBytes, smem_set);
   if (e != cudaSuccess) return e;
   a.npairs = (a.nT + T - 1) / T;  // work units (groups of T Q tiles) per (b, h)
-  const unsigned grid = (unsigned)a.BH * (unsigned)a.npairs;
+  // persistent: as many CTAs as fit at once (3 - T per SM), each walking its share of the units
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = fa::device_sm_count(dev, &sms)) != cudaSuccess) return e;
+  const long long units = (long long)a.BH * a.npairs;
+  const unsigned grid = (unsigned)std::min<long long>(units, (long long)sms * (3 - T));
   if ((e = mark(FA_KERNEL_FWD, 0, st)) != cudaSuccess) return e;
   fa::fwd_kernel<D, BF, T><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mk, mv, a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
