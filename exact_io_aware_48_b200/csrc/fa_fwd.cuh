@@ -42,9 +42,12 @@ struct FwdCfg {
 };
 
 // Every kExpFmaEvery-th pair of probabilities is exponentiated on the FMA pipe (see ptx::exp2_fma); 0 = never.
-// Measured on B200: sending 1 pair in 4 to the FMA pipe lowered long-context forward throughput by 6-7% (the
-// softmax warps are issue/latency bound, not MUFU bound), so it is off.
-constexpr int kExpFmaEvery = 0;
+// Measured on B200 (same box, interleaved runs): 1 pair in 16 gains 1-5% (GPT-2 shape 286 -> 299 TFLOP/s,
+// N = 4096 800 -> 819, N = 16384 1109 -> 1122); 1 in 8 gains nothing and 1 in 4 loses 6%.
+#ifndef FA_FWD_EXP_FMA_EVERY
+#define FA_FWD_EXP_FMA_EVERY 16
+#endif
+constexpr int kExpFmaEvery = FA_FWD_EXP_FMA_EVERY;
 
 struct FwdArgs {
   void* o;
