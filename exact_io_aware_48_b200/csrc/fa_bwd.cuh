@@ -7,9 +7,9 @@
 //     dQ = scale * dS K,  dK = scale * dS^T Q.
 //
 // Three launches:
-//   bwd_pre_kernel   D_r = sum_j dO_rj O_rj (fp32) and LSE in base 2 for every row of a 128-padded row space
-//                    (padded rows and rows with no visible key get +inf, so their recomputed P is exactly 0);
-//                    zeroes the fp32 dQ accumulator.  HBM-bound.
+//   bwd_pre_kernel   D_r = sum_j dO_rj O_rj (fp32) and LSE in base 2 for every row of a 128-padded row space,
+//                    stored as -scale * D_r and -LSE2_r (padded rows and rows with no visible key get -LSE2 = -inf,
+//                    so their recomputed P is exactly 0); zeroes the fp32 dQ accumulator.  HBM-bound.
 //   bwd_kernel       persistent, at most one CTA per SM; each CTA walks a share of the units (128-key tile j of
 //                    one (b, h)) and, per unit, loops over the visible 128-row Q tiles i.
 //                    Five tcgen05 GEMMs per (i, j): S^T = K Q^T and dP^T = V dO^T (recompute), dV += P^T dO (P^T read
@@ -64,7 +64,8 @@ struct BwdCfg {
   static constexpr uint32_t kPtHalf = kDqOwnCols ? 32 : 64;  // column distance between the two query halves
 };
 
-// Workspace layout: dq_acc [BH][Npad][D] fp32 | lse2 [BH][Npad] fp32 | Dv [BH][Npad] fp32 (each 256-B aligned)
+// Workspace layout: dq_acc [BH][Npad][D] fp32 | nlse2 [BH][Npad] fp32 (-LSE in base 2) | nDv [BH][Npad] fp32
+// (-softmax_scale * D), each 256-B aligned
 inline size_t bwd_workspace_bytes(int BH, int nT, int d) {
   const size_t npad = (size_t)nT * kTile;
   auto al = [](size_t x) { return (x + 255) / 256 * 256; };
@@ -75,8 +76,8 @@ struct BwdArgs {
   void* dk;
   void* dv;
   float* dq_acc;
-  const float* lse2;
-  const float* Dv;
+  const float* lse2;  // -LSE2 per padded row
+  const float* Dv;    // -scale * D per padded row
   const int32_t* key_lens;
   const int32_t* col_ptr;  // CSC of the block mask (nullptr: dense)
   const int32_t* row_idx;
@@ -134,7 +135,7 @@ template <int D, bool kBF16>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const void* __restrict__ o, const void* __restrict__ dout,
                                                       const float* __restrict__ lse, float* __restrict__ dq_acc,
                                                       float* __restrict__ lse2, float* __restrict__ Dv, int N,
-                                                      int Npad, long long rows) {
+                                                      int Npad, long long rows, float scale) {
   constexpr int kLanesPerRow = D / 8;          // 8 or 16
   constexpr int kRowsPerWarp = 32 / kLanesPerRow;  // 4 or 2
   const int lane = threadIdx.x % 32;
@@ -166,13 +167,13 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const void* __restrict__ o
       acc[2 * l] = make_float4(0.f, 0.f, 0.f, 0.f);
       acc[2 * l + 1] = make_float4(0.f, 0.f, 0.f, 0.f);
       if (l == 0) {
-        float l2 = INFINITY;  // padded row or no visible key: recomputed P = exp2(x - inf) = 0
+        float nl2 = -INFINITY;  // padded row or no visible key: recomputed P = exp2(x - inf) = 0
         if (r < N) {
           const float lv = lse[(size_t)bh * N + r];
-          if (lv != -INFINITY) l2 = lv * 1.4426950408889634f;
+          if (lv != -INFINITY) nl2 = -lv * 1.4426950408889634f;
         }
-        lse2[row] = l2;
-        Dv[row] = dsum;
+        lse2[row] = nl2;
+        Dv[row] = -scale * dsum;
       }
     }
   }
@@ -507,7 +508,7 @@ __global__ void __launch_bounds__(512, 1)
     const int g = warp / 4, quarter = warp % 4;
     const int c = quarter * 32 + lane;  // key row within the tile == TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    const float sl2 = args.scale_log2, sc = args.scale;
+    const ptx::f32x2 sl2v{args.scale_log2, args.scale_log2}, sc2{args.scale, args.scale};
     int n = 0, gi = 0;
     bool ok = true;
     while (ok && us.next(L)) {
@@ -521,8 +522,9 @@ __global__ void __launch_bounds__(512, 1)
         const int sq = n % NS;
         const uint32_t phq = (n / NS) & 1;
         n += 2;
-        const float* lse2 = reinterpret_cast<const float*>(sRing + sq * C::kSlotBytes + C::kTileBytes) + 64 * g;
-        const float* Drow = lse2 + 128;
+        // -LSE2 and -scale*D of this half's 64 queries (16-byte aligned: read four at a time, all lanes alike)
+        const float* nlse2 = reinterpret_cast<const float*>(sRing + sq * C::kSlotBytes + C::kTileBytes) + 64 * g;
+        const float* nDrow = nlse2 + 128;
         const uint32_t ph = gi & 1;
         // the LSE2/D rows came in by bulk copy with Q_i: observe that copy's barrier before reading them (the slot
         // cannot be refilled before this iteration's dS^T is published, so the phase is stable)
@@ -543,12 +545,13 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
           for (int v = 0; v < 16; ++v) {
             const int r0 = 32 * h + 2 * v;
-            const float2 l2 = *reinterpret_cast<const float2*>(lse2 + r0);
+            const float4 nl4 = *reinterpret_cast<const float4*>(nlse2 + (r0 & ~3));
+            const ptx::f32x2 nl = (v & 1) ? ptx::f32x2{nl4.z, nl4.w} : ptx::f32x2{nl4.x, nl4.y};
             const bool emu = kBwdExpFmaEvery > 0 && v % (kBwdExpFmaEvery > 0 ? kBwdExpFmaEvery : 1) == 0;
-            const float x0 = fmaf(__uint_as_float(sr[2 * v]), sl2, -l2.x);
-            const float x1 = fmaf(__uint_as_float(sr[2 * v + 1]), sl2, -l2.y);
-            float p0 = emu ? ptx::exp2_fma(x0) : ptx::ex2(x0);
-            float p1 = emu ? ptx::exp2_fma(x1) : ptx::ex2(x1);
+            const ptx::f32x2 x =
+                ptx::fma2({__uint_as_float(sr[2 * v]), __uint_as_float(sr[2 * v + 1])}, sl2v, nl);  // S*scale - LSE
+            float p0 = emu ? ptx::exp2_fma(x.x) : ptx::ex2(x.x);
+            float p1 = emu ? ptx::exp2_fma(x.y) : ptx::ex2(x.y);
             if (masked) {
               if (!key_ok || r0 < rmin) p0 = 0.f;
               if (!key_ok || r0 + 1 < rmin) p1 = 0.f;
@@ -586,18 +589,13 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
           for (int v = 0; v < 16; ++v) {
             const int r0 = 32 * h + 2 * v;
-            const float2 dd = *reinterpret_cast<const float2*>(Drow + r0);
-            float p0, p1;
-            if constexpr (kBF16) {
-              p0 = __uint_as_float(pk[16 * h + v] << 16);
-              p1 = __uint_as_float(pk[16 * h + v] & 0xffff0000u);
-            } else {
-              p0 = __half2float(__ushort_as_half((unsigned short)(pk[16 * h + v] & 0xffff)));
-              p1 = __half2float(__ushort_as_half((unsigned short)(pk[16 * h + v] >> 16)));
-            }
-            const float ds0 = p0 * (__uint_as_float(dr[2 * v]) - dd.x) * sc;
-            const float ds1 = p1 * (__uint_as_float(dr[2 * v + 1]) - dd.y) * sc;
-            o[v] = ptx::pack2<kBF16>(ds0, ds1);
+            const float4 nd4 = *reinterpret_cast<const float4*>(nDrow + (r0 & ~3));
+            const ptx::f32x2 nd = (v & 1) ? ptx::f32x2{nd4.z, nd4.w} : ptx::f32x2{nd4.x, nd4.y};
+            // dS = P * (dP - D) * scale = P * (dP * scale + (-scale * D)), P as the 16-bit values dV used
+            const ptx::f32x2 t =
+                ptx::fma2({__uint_as_float(dr[2 * v]), __uint_as_float(dr[2 * v + 1])}, sc2, nd);
+            const ptx::f32x2 ds = ptx::mul2(ptx::unpack2<kBF16>(pk[16 * h + v]), t);
+            o[v] = ptx::pack2<kBF16>(ds.x, ds.y);
           }
           // queries 32h .. 32h+31 of this half: 16-byte chunks 4h .. 4h+3 of row c (128-byte swizzle)
 #pragma unroll
@@ -740,7 +738,7 @@ cudaError_t launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   const long long pre_warps = (rows + (256 / D) - 1) / (256 / D);  // rows per warp pass: 4 (d=64) or 2 (d=128)
   const unsigned pre_blocks = (unsigned)std::min<long long>((pre_warps + 7) / 8, 148LL * 16);
   bwd_pre_kernel<D, BF><<<pre_blocks, 256, 0, st>>>(o, dout, lse, a.dq_acc, const_cast<float*>(a.lse2),
-                                                     const_cast<float*>(a.Dv), a.N, Npad, rows);
+                                                     const_cast<float*>(a.Dv), a.N, Npad, rows, a.scale);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   static std::atomic<uint64_t> smem_set{0};

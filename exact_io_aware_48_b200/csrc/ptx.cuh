@@ -281,6 +281,16 @@ __device__ __forceinline__ f32x2 add2(f32x2 a, f32x2 b) {
   return d;
 }
 
+__device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b) {
+  uint64_t ra, rb, rd;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(ra) : "f"(a.x), "f"(a.y));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(rb) : "f"(b.x), "f"(b.y));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(rd) : "l"(ra), "l"(rb));
+  f32x2 d;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(d.x), "=f"(d.y) : "l"(rd));
+  return d;
+}
+
 // The two 16-bit values packed by pack2, widened to fp32 (exactly the values the tensor core multiplies).
 template <bool kBF16>
 __device__ __forceinline__ f32x2 unpack2(uint32_t v) {
