@@ -13,7 +13,8 @@ from . import _lib
 from ._lib import (FA_BF16, FA_FP16, FA_OK, FA_ERR_CUDA, FA_ERR_INVALID_ARG, FA_ERR_TIMEOUT, FA_ERR_UNSUPPORTED,
                    FA_ERR_WORKSPACE)
 
-__all__ = ["attention_fwd", "attention_bwd", "blockmask_lists", "FAError", "FA_BF16", "FA_FP16"]
+__all__ = ["attention_fwd", "attention_bwd", "attention_fwd_varlen", "attention_bwd_varlen", "blockmask_lists",
+           "FAError", "FA_BF16", "FA_FP16"]
 
 
 class FAError(RuntimeError):
@@ -101,3 +102,39 @@ def blockmask_lists(mask, stream=None):
 def last_device_status(stream=None) -> int:
     """Synchronise and return (then clear) the device status word: FA_OK or FA_ERR_TIMEOUT."""
     return _lib.fa_last_device_status(stream)
+
+
+def attention_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, causal=False,
+                         softmax_scale=None, stream=None):
+    """O, LSE of a packed variable-length batch: q [total_q, H, d], k, v [total_k, H, d] CUDA tensors (bf16 or
+    fp16), cu_seqlens_* int32 CUDA tensors [B+1].  Returns O [total_q, H, d] and LSE [H, total_q] (fp32)."""
+    import torch
+    _require_cuda(q, k, v, cu_seqlens_q, cu_seqlens_k)
+    total_q, H, d = q.shape
+    total_k = k.shape[0]
+    B = cu_seqlens_q.numel() - 1
+    scale = softmax_scale if softmax_scale is not None else 1.0 / math.sqrt(d)
+    o = torch.empty_like(q)
+    lse = torch.empty((H, total_q), device=q.device, dtype=torch.float32)
+    _check(_lib.fa_fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, H, max_seqlen_q, max_seqlen_k, total_q,
+                              total_k, d, scale, causal, _dtype_code(q), stream), "fa_fwd_varlen")
+    return o, lse
+
+
+def attention_bwd_varlen(q, k, v, o, dout, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
+                         causal=False, softmax_scale=None, stream=None):
+    """dQ, dK, dV of sum(O * dout) for attention_fwd_varlen with the same arguments."""
+    import torch
+    _require_cuda(q, k, v, o, dout, lse, cu_seqlens_q, cu_seqlens_k)
+    total_q, H, d = q.shape
+    total_k = k.shape[0]
+    B = cu_seqlens_q.numel() - 1
+    scale = softmax_scale if softmax_scale is not None else 1.0 / math.sqrt(d)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws_bytes = _lib.fa_bwd_varlen_workspace_size(B, H, max_seqlen_q, d)
+    ws = torch.empty(ws_bytes, device=q.device, dtype=torch.uint8)
+    _check(_lib.fa_bwd_varlen(q, k, v, o, dout, lse, dq, dk, dv, cu_seqlens_q, cu_seqlens_k, B, H, max_seqlen_q,
+                              max_seqlen_k, total_q, total_k, d, scale, causal, ws, ws_bytes, _dtype_code(q), stream),
+           "fa_bwd_varlen")
+    return dq, dk, dv
+

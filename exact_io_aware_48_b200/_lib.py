@@ -35,6 +35,10 @@ SIGNATURES = {
     "fa_selftest_exp2": ([_P, _P, _P, _I, _P], _I),
     "fa_set_fwd_tiles_per_cta": ([_I], _I),
     "fa_bwd_noalloc": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P, _P, _I, _P], _I),
+    "fa_fwd_varlen": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P], _I),
+    "fa_bwd_varlen_workspace_size": ([_I, _I, _I, _I], _SZ),
+    "fa_bwd_varlen": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P, _SZ, _I,
+                       _P], _I),
 }
 FA_NOALLOC_SCRATCH_BYTES = 32 << 20
 FA_KERNEL_FWD, FA_KERNEL_BWD_MAIN = 0, 1
@@ -159,3 +163,20 @@ def fa_selftest_exp2(x, out_fma, out_mufu, n, stream=None) -> int:
 
 def fa_set_fwd_tiles_per_cta(tiles) -> int:
     return load().fa_set_fwd_tiles_per_cta(int(tiles))
+
+
+def fa_fwd_varlen(q, k, v, o, lse, cu_q, cu_k, B, H, max_q, max_k, total_q, total_k, d, softmax_scale, causal, dtype,
+                  stream=None) -> int:
+    return load().fa_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(cu_q), _ptr(cu_k), B, H, max_q,
+                                max_k, total_q, total_k, d, softmax_scale, int(causal), dtype, _stream(stream))
+
+
+def fa_bwd_varlen_workspace_size(B, H, max_q, d) -> int:
+    return load().fa_bwd_varlen_workspace_size(B, H, max_q, d)
+
+
+def fa_bwd_varlen(q, k, v, o, dout, lse, dq, dk, dv, cu_q, cu_k, B, H, max_q, max_k, total_q, total_k, d,
+                  softmax_scale, causal, workspace, workspace_bytes, dtype, stream=None) -> int:
+    return load().fa_bwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
+                                _ptr(dv), _ptr(cu_q), _ptr(cu_k), B, H, max_q, max_k, total_q, total_k, d,
+                                softmax_scale, int(causal), _ptr(workspace), workspace_bytes, dtype, _stream(stream))

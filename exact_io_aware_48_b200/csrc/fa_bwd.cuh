@@ -81,7 +81,11 @@ struct BwdArgs {
   const int32_t* key_lens;
   const int32_t* col_ptr;  // CSC of the block mask (nullptr: dense)
   const int32_t* row_idx;
-  int H, N, nT, BH;
+  const int32_t* cu_q;  // packed variable-length batch: cumulative sequence lengths (nullptr: dense [B,H,N,d])
+  const int32_t* cu_k;
+  int total_q, total_k;  // packed: token counts; dK, dV are [total_k, H, d]
+  int H, N, nT, BH;  // nT = Q tiles of the padded row space (packed: of the longest query sequence)
+  int Nk, nTk;       // key rows and K/V tiles per head (packed: of the longest key sequence)
   int causal;
   float scale;       // softmax scale
   float scale_log2;  // softmax scale * log2(e)
@@ -130,12 +134,15 @@ struct ColTileIter {
 // ------------------------------------------------------------------------------------------------ preprocess
 // Row r of a head needs D/8 lanes (16-byte loads of 8 16-bit values), so a warp covers 32*8/D rows per pass; the
 // lanes of a row reduce with xor-shuffles inside their group.  Every padded row's dQ accumulator is zeroed with
-// 16-byte stores.  Grid-stride over all padded rows of all heads.
+// 16-byte stores.  Grid-stride over all padded rows of all heads.  Packed variable-length batches (cu_q non-null):
+// O, dO are [total_q, H, d] and LSE [H, total_q]; the padded row space stays per (b, h), rows past the sequence's
+// length get -LSE2 = -inf like padding.
 template <int D, bool kBF16>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const void* __restrict__ o, const void* __restrict__ dout,
                                                       const float* __restrict__ lse, float* __restrict__ dq_acc,
                                                       float* __restrict__ lse2, float* __restrict__ Dv, int N,
-                                                      int Npad, long long rows, float scale) {
+                                                      int Npad, long long rows, float scale,
+                                                      const int32_t* __restrict__ cu_q, int total_q, int H) {
   constexpr int kLanesPerRow = D / 8;          // 8 or 16
   constexpr int kRowsPerWarp = 32 / kLanesPerRow;  // 4 or 2
   const int lane = threadIdx.x % 32;
@@ -147,9 +154,12 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const void* __restrict__ o
     const bool in = row < rows;
     const long long bh = in ? row / Npad : 0;
     const int r = in ? (int)(row % Npad) : 0;
+    const SeqGeom g = seq_geom(cu_q, cu_q, nullptr, (int)(bh / H), N, N, total_q, total_q);
+    const bool valid = r < g.lq;
+    const size_t prow = cu_q ? (size_t)(g.q0 + r) * H + (size_t)(bh % H) : (size_t)bh * N + r;  // row of O, dO
     float dsum = 0.f;
-    if (in && r < N) {
-      const size_t off = ((size_t)bh * N + r) * D + (size_t)l * 8;
+    if (in && valid) {
+      const size_t off = prow * D + (size_t)l * 8;
       const uint4 a = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(o) + off);
       const uint4 c = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(dout) + off);
       const uint32_t va[4] = {a.x, a.y, a.z, a.w}, vc[4] = {c.x, c.y, c.z, c.w};
@@ -168,8 +178,8 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const void* __restrict__ o
       acc[2 * l + 1] = make_float4(0.f, 0.f, 0.f, 0.f);
       if (l == 0) {
         float nl2 = -INFINITY;  // padded row or no visible key: recomputed P = exp2(x - inf) = 0
-        if (r < N) {
-          const float lv = lse[(size_t)bh * N + r];
+        if (valid) {
+          const float lv = lse[cu_q ? (size_t)(bh % H) * total_q + g.q0 + r : (size_t)bh * N + r];
           if (lv != -INFINITY) nl2 = -lv * 1.4426950408889634f;
         }
         lse2[row] = nl2;
@@ -180,17 +190,25 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const void* __restrict__ o
 }
 
 // ------------------------------------------------------------------------------------------------ dQ convert
-// Each thread converts 8 consecutive elements (two 16-byte loads, one 16-byte store) of the N-row output.
+// Each thread converts 8 consecutive elements (two 16-byte loads, one 16-byte store).  Dense: over the N-row
+// output.  Packed variable-length: over the padded rows, writing those inside their sequence to [total_q, H, d].
 template <int D, bool kBF16>
 __global__ void __launch_bounds__(256) bwd_dq_kernel(const float* __restrict__ dq_acc, void* __restrict__ dq, int N,
-                                                     int Npad, long long total_vec8) {
+                                                     int Npad, long long total_vec8, const int32_t* __restrict__ cu_q,
+                                                     int total_q, int H) {
   for (long long v = (long long)blockIdx.x * blockDim.x + threadIdx.x; v < total_vec8;
        v += (long long)gridDim.x * blockDim.x) {
     const long long e = v * 8;
-    const long long row = e / D;  // bh * N + r
+    const long long row = e / D;  // dense: bh * N + r; packed: bh * Npad + r
     const int c = (int)(e % D);
-    const long long bh = row / N;
-    const int r = (int)(row % N);
+    const long long bh = row / (cu_q ? Npad : N);
+    const int r = (int)(row % (cu_q ? Npad : N));
+    size_t out_e = (size_t)e;
+    if (cu_q) {
+      const SeqGeom g = seq_geom(cu_q, cu_q, nullptr, (int)(bh / H), N, N, total_q, total_q);
+      if (r >= g.lq) continue;
+      out_e = ((size_t)(g.q0 + r) * H + (size_t)(bh % H)) * D + c;
+    }
     const float4* src = reinterpret_cast<const float4*>(dq_acc + ((size_t)bh * Npad + r) * D + c);
     const float4 a = src[0], b = src[1];
     uint4 out;
@@ -198,7 +216,7 @@ __global__ void __launch_bounds__(256) bwd_dq_kernel(const float* __restrict__ d
     out.y = ptx::pack2<kBF16>(a.z, a.w);
     out.z = ptx::pack2<kBF16>(b.x, b.y);
     out.w = ptx::pack2<kBF16>(b.z, b.w);
-    *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(dq) + e) = out;
+    *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(dq) + out_e) = out;
   }
 }
 
@@ -206,7 +224,8 @@ __global__ void __launch_bounds__(256) bwd_dq_kernel(const float* __restrict__ d
 // Units of work are (K/V tile j, head bh), ordered j-major so that the longest causal columns come first; the
 // kernel is persistent and walks them with UnitSeq.
 struct BwdUnit {
-  int j, bh, kv_lim;
+  int j, bh, h, kv_lim, nTq;
+  SeqGeom g;
   bool visible;  // some key of the tile is visible to someone
 };
 
@@ -214,8 +233,11 @@ __device__ __forceinline__ BwdUnit bwd_unit(int L, const BwdArgs& a) {
   BwdUnit u;
   u.j = L / a.BH;
   u.bh = L % a.BH;
-  u.kv_lim = key_limit(a.key_lens, u.bh / a.H, a.N);
-  u.visible = u.j * kTile < u.kv_lim;
+  u.h = u.bh % a.H;
+  u.g = seq_geom(a.cu_q, a.cu_k, a.key_lens, u.bh / a.H, a.N, a.Nk, a.total_q, a.total_k);
+  u.kv_lim = u.g.lk;
+  u.nTq = (u.g.lq + kTile - 1) / kTile;
+  u.visible = u.j * kTile < u.kv_lim && u.nTq > 0;
   return u;
 }
 
@@ -247,7 +269,8 @@ __global__ void __launch_bounds__(512, 1)
   constexpr int kWarpDrain = 8, kWarpMma = 12, kWarpLoad = 13;
   const bool causal = args.causal != 0;
   const int Npad = args.nT * kTile;
-  const int total_units = args.nT * args.BH;
+  const int total_units = args.nTk * args.BH;
+  const bool packed = args.cu_q != nullptr;
 
   if (threadIdx.x == 0) {
     for (int k = 0; k < KB; ++k) {
@@ -300,7 +323,7 @@ __global__ void __launch_bounds__(512, 1)
       while (ok && us.next(L)) {
         const BwdUnit u = bwd_unit(L, args);
         ColTileIter it;
-        it.init(args.col_ptr, args.row_idx, u.j, args.nT, causal ? u.j : 0, u.visible);
+        it.init(args.col_ptr, args.row_idx, u.j, u.nTq, causal ? u.j : 0, u.visible);
         if (it.count() == 0) continue;
         const int kb = ku % KB;
         // the buffer's previous K/V tiles must have been read by every MMA of their unit
@@ -312,8 +335,8 @@ __global__ void __launch_bounds__(512, 1)
         const uint32_t bkv = ptx::smem_addr(&bar_kv[kb]);
         ptx::mbar_arrive_expect_tx(bkv, 2 * C::kTileBytes);
         for (int c = 0; c < C::kSubTiles; ++c) {
-          ptx::tma_load_3d(ptx::smem_addr(sK(kb) + c * 16384), &map_k, 64 * c, u.j * kTile, u.bh, bkv);
-          ptx::tma_load_3d(ptx::smem_addr(sV(kb) + c * 16384), &map_v, 64 * c, u.j * kTile, u.bh, bkv);
+          tma_rows(ptx::smem_addr(sK(kb) + c * 16384), &map_k, c, u.j * kTile, u.g.k0, u.bh, u.h, packed, bkv);
+          tma_rows(ptx::smem_addr(sV(kb) + c * 16384), &map_v, c, u.j * kTile, u.g.k0, u.bh, u.h, packed, bkv);
         }
         int i;
         while (ok && it.next(i)) {
@@ -325,8 +348,8 @@ __global__ void __launch_bounds__(512, 1)
             uint8_t* slot = sRing + s * C::kSlotBytes;
             ptx::mbar_arrive_expect_tx(bf, C::kTileBytes + (v == 0 ? 1024 : 0));
             for (int c = 0; c < C::kSubTiles; ++c)
-              ptx::tma_load_3d(ptx::smem_addr(slot + c * 16384), v == 0 ? &map_q : &map_do, 64 * c, i * kTile, u.bh,
-                               bf);
+              tma_rows(ptx::smem_addr(slot + c * 16384), v == 0 ? &map_q : &map_do, c, i * kTile, u.g.q0, u.bh, u.h,
+                       packed, bf);
             if (v == 0) {
               const size_t row0 = (size_t)u.bh * Npad + (size_t)i * kTile;
               ptx::bulk_load(ptx::smem_addr(slot + C::kTileBytes), args.lse2 + row0, 512, bf);
@@ -416,7 +439,7 @@ __global__ void __launch_bounds__(512, 1)
       while (ok && us.next(L)) {
         const BwdUnit u = bwd_unit(L, args);
         ColTileIter it;
-        it.init(args.col_ptr, args.row_idx, u.j, args.nT, causal ? u.j : 0, u.visible);
+        it.init(args.col_ptr, args.row_idx, u.j, u.nTq, causal ? u.j : 0, u.visible);
         if (it.count() == 0) continue;
         const int kb = ku % KB;
         dk_k = ptx::sw128_desc(ptx::smem_addr(sK(kb)), 16, 1024);
@@ -514,7 +537,7 @@ __global__ void __launch_bounds__(512, 1)
     while (ok && us.next(L)) {
       const BwdUnit u = bwd_unit(L, args);
       ColTileIter it;
-      it.init(args.col_ptr, args.row_idx, u.j, args.nT, causal ? u.j : 0, u.visible);
+      it.init(args.col_ptr, args.row_idx, u.j, u.nTq, causal ? u.j : 0, u.visible);
       const int j = u.j, kv_lim = u.kv_lim;
       const int gc = j * kTile + c;  // key index in the sequence
       int i;
@@ -628,7 +651,7 @@ __global__ void __launch_bounds__(512, 1)
     while (ok && us.next(L)) {
       const BwdUnit u = bwd_unit(L, args);
       ColTileIter it;
-      it.init(args.col_ptr, args.row_idx, u.j, args.nT, causal ? u.j : 0, u.visible);
+      it.init(args.col_ptr, args.row_idx, u.j, u.nTq, causal ? u.j : 0, u.visible);
       const int n_iters = it.count();
       int i;
       while (it.next(i)) {
@@ -679,9 +702,11 @@ __global__ void __launch_bounds__(512, 1)
       if (!ok) break;
       // ---- dK, dV epilogue of this unit
       const int gc = u.j * kTile + wq * 32 + lane;  // key row
-      const bool row_ok = gc < args.N;
-      uint8_t* dv_row = reinterpret_cast<uint8_t*>(args.dv) + ((size_t)u.bh * args.N + gc) * D * 2;
-      uint8_t* dk_row = reinterpret_cast<uint8_t*>(args.dk) + ((size_t)u.bh * args.N + gc) * D * 2;
+      // dense: every row of the head (keys past a key length get zero); packed: the sequence's own keys only
+      const bool row_ok = packed ? gc < u.g.lk : gc < args.N;
+      const size_t krow = packed ? (size_t)(u.g.k0 + gc) * args.H + u.h : (size_t)u.bh * args.N + gc;
+      uint8_t* dv_row = reinterpret_cast<uint8_t*>(args.dv) + krow * D * 2;
+      uint8_t* dk_row = reinterpret_cast<uint8_t*>(args.dk) + krow * D * 2;
       if (n_iters > 0) {
         ok = __all_sync(0xffffffffu, wait_or_abort(ptx::smem_addr(&bar_done), ku & 1, args.budget_ns, abortp));
         if (!ok) break;
@@ -738,7 +763,8 @@ cudaError_t launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   const long long pre_warps = (rows + (256 / D) - 1) / (256 / D);  // rows per warp pass: 4 (d=64) or 2 (d=128)
   const unsigned pre_blocks = (unsigned)std::min<long long>((pre_warps + 7) / 8, 148LL * 16);
   bwd_pre_kernel<D, BF><<<pre_blocks, 256, 0, st>>>(o, dout, lse, a.dq_acc, const_cast<float*>(a.lse2),
-                                                     const_cast<float*>(a.Dv), a.N, Npad, rows, a.scale);
+                                                     const_cast<float*>(a.Dv), a.N, Npad, rows, a.scale, a.cu_q,
+                                                     a.total_q, a.H);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   static std::atomic<uint64_t> smem_set{0};
@@ -752,15 +778,15 @@ cudaError_t launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   // persistent: one CTA per SM at most (each walks its share of the units)
   int sms = 0;
   if ((e = device_sm_count(dev, &sms)) != cudaSuccess) return e;
-  const long long units = (long long)a.nT * a.BH;
+  const long long units = (long long)a.nTk * a.BH;
   const unsigned grid = (unsigned)std::min<long long>(units, sms);
   if (ev_start && (e = cudaEventRecord(ev_start, st)) != cudaSuccess) return e;
   bwd_kernel<D, BF><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mk, mv, mdo, mdq, a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (ev_stop && (e = cudaEventRecord(ev_stop, st)) != cudaSuccess) return e;
-  const long long total_vec8 = (long long)a.BH * a.N * D / 8;
+  const long long total_vec8 = (long long)a.BH * (a.cu_q ? Npad : a.N) * D / 8;
   const unsigned blocks = (unsigned)std::min<long long>((total_vec8 + 255) / 256, 148LL * 16);
-  bwd_dq_kernel<D, BF><<<blocks, 256, 0, st>>>(a.dq_acc, dq, a.N, Npad, total_vec8);
+  bwd_dq_kernel<D, BF><<<blocks, 256, 0, st>>>(a.dq_acc, dq, a.N, Npad, total_vec8, a.cu_q, a.total_q, a.H);
   return cudaGetLastError();
 }
 
@@ -769,7 +795,10 @@ inline cudaError_t run_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const C
                            void* dk, void* dv, int B, int H, int N, int d, float scale, bool causal,
                            const int32_t* key_lens, const int32_t* col_ptr, const int32_t* row_idx, void* workspace,
                            bool bf16, uint64_t budget_ns, cudaStream_t st, cudaEvent_t ev_start,
-                           cudaEvent_t ev_stop) {
+                           cudaEvent_t ev_stop, const int32_t* cu_q = nullptr, const int32_t* cu_k = nullptr,
+                           int total_q = 0, int total_k = 0, int Nk = 0) {
+  // packed variable-length batches: N / Nk are the longest query / key sequences; dense: Nk = N
+  if (Nk <= 0) Nk = N;
   const int nT = (N + kTile - 1) / kTile;
   const int BH = B * H;
   const size_t npad = (size_t)nT * kTile;
@@ -784,9 +813,15 @@ inline cudaError_t run_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const C
   a.key_lens = key_lens;
   a.col_ptr = col_ptr;
   a.row_idx = row_idx;
+  a.cu_q = cu_q;
+  a.cu_k = cu_k;
+  a.total_q = total_q;
+  a.total_k = total_k;
   a.H = H;
   a.N = N;
   a.nT = nT;
+  a.Nk = Nk;
+  a.nTk = (Nk + kTile - 1) / kTile;
   a.BH = BH;
   a.causal = causal ? 1 : 0;
   a.scale = scale;

@@ -112,6 +112,44 @@ struct PairTileIter {
   __device__ __forceinline__ int count(int t) const { return len[t]; }
 };
 
+// Where the rows of one (b, h) live.  Dense [B, H, N, d]: rows 0..N-1 of plane b*H+h, keys limited by key_lens.
+// Packed variable-length [total, H, d]: tokens cu[b] .. cu[b+1]-1 of head h, for queries and keys separately
+// (the caller's cu_seqlens; values are clamped to [0, total] and lengths to the stated maximum, so a bad array
+// cannot move an access out of range).  Positions r, c below are always relative to the sequence start.
+struct SeqGeom {
+  int q0, k0;  // first row (dense: 0) / token (packed) of the sequence
+  int lq, lk;  // query rows, visible keys
+};
+
+__device__ __forceinline__ SeqGeom seq_geom(const int32_t* cu_q, const int32_t* cu_k, const int32_t* key_lens, int b,
+                                            int N, int Nk, int total_q, int total_k) {
+  SeqGeom g;
+  if (cu_q != nullptr) {
+    const int a = min(max(cu_q[b], 0), total_q), e = min(max(cu_q[b + 1], a), total_q);
+    const int ak = min(max(cu_k[b], 0), total_k), ek = min(max(cu_k[b + 1], ak), total_k);
+    g.q0 = a;
+    g.lq = min(e - a, N);
+    g.k0 = ak;
+    g.lk = min(ek - ak, Nk);
+  } else {
+    g.q0 = 0;
+    g.k0 = 0;
+    g.lq = N;
+    g.lk = key_limit(key_lens, b, N);
+  }
+  return g;
+}
+
+// One 128-row x 64-column box of a 16-bit tensor into shared memory.  Dense maps are {d, N, B*H} (row, plane);
+// packed maps are {d, H, total} with a {64, 1, 128} box (head, token): both land as 128 rows of 128 bytes.
+__device__ __forceinline__ void tma_rows(uint32_t dst, const CUtensorMap* map, int c, int row, int base, int bh, int h,
+                                         bool packed, uint32_t bar) {
+  if (packed)
+    ptx::tma_load_3d(dst, map, 64 * c, h, base + row, bar);
+  else
+    ptx::tma_load_3d(dst, map, 64 * c, row, bh, bar);
+}
+
 // Persistent kernels: CTA c of G takes, in round r, unit r*G + c (r even) or r*G + G-1-c (r odd).  With units
 // ordered longest first, this zigzag evens out the per-CTA work about as well as a greedy longest-first queue,
 // without a global counter.

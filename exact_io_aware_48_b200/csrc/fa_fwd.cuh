@@ -55,7 +55,11 @@ struct FwdArgs {
   const int32_t* key_lens;
   const int32_t* row_ptr;  // CSR of the block mask (nullptr: dense)
   const int32_t* col_idx;
-  int H, N, nT, npairs, BH;
+  const int32_t* cu_q;  // packed variable-length batch: cumulative sequence lengths (nullptr: dense [B,H,N,d])
+  const int32_t* cu_k;
+  int total_q, total_k;  // packed: token counts; O is [total_q, H, d], LSE [H, total_q]
+  int H, N, nT, npairs, BH;  // packed: N = the longest query sequence, Nk the longest key sequence
+  int Nk;
   int causal;
   float scale_log2;  // softmax_scale * log2(e)
   uint64_t budget_ns;
@@ -64,7 +68,8 @@ struct FwdArgs {
 // One unit of work: kTiles consecutive 128-row Q tiles of one (b, h).  Units are ordered longest first (latest Q
 // tiles first under the causal mask); the kernel is persistent and walks them with UnitSeq.
 struct FwdUnit {
-  int qt0, bh, kv_lim, end0, end1;
+  int qt0, bh, h, kv_lim, end0, end1;
+  SeqGeom g;
   bool has1;
 };
 
@@ -72,11 +77,14 @@ __device__ __forceinline__ FwdUnit fwd_unit(int L, const FwdArgs& a, int tiles) 
   FwdUnit u;
   const int pair = a.npairs - 1 - L / a.BH;
   u.bh = L % a.BH;
+  u.h = u.bh % a.H;
   u.qt0 = tiles * pair;
-  u.has1 = tiles == 2 && u.qt0 + 1 < a.nT;
-  u.kv_lim = key_limit(a.key_lens, u.bh / a.H, a.N);
+  u.g = seq_geom(a.cu_q, a.cu_k, a.key_lens, u.bh / a.H, a.N, a.Nk, a.total_q, a.total_k);
+  const int nTq = (u.g.lq + kTile - 1) / kTile;  // Q tiles of this sequence
+  u.has1 = tiles == 2 && u.qt0 + 1 < nTq;
+  u.kv_lim = u.g.lk;
   const bool causal = a.causal != 0;
-  u.end0 = kv_tile_end(u.qt0, u.kv_lim, causal);
+  u.end0 = u.qt0 < nTq ? kv_tile_end(u.qt0, u.kv_lim, causal) : 0;  // a tile past the sequence sees nothing
   u.end1 = u.has1 ? kv_tile_end(u.qt0 + 1, u.kv_lim, causal) : 0;
   return u;
 }
@@ -107,6 +115,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const bool causal = args.causal != 0;
+  const bool packed = args.cu_q != nullptr;
   const int total_units = args.npairs * args.BH;
 
   if (threadIdx.x == 0) {
@@ -159,8 +168,8 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
         ptx::mbar_arrive_expect_tx(bq, (u.has1 ? 2 : 1) * C::kSlotBytes);
         for (int t = 0; t < (u.has1 ? 2 : 1); ++t)
           for (int c = 0; c < C::kSubTiles; ++c)
-            ptx::tma_load_3d(ptx::smem_addr(sQ + t * C::kSlotBytes + c * 16384), &map_q, 64 * c,
-                             (u.qt0 + t) * kTile, u.bh, bq);
+            tma_rows(ptx::smem_addr(sQ + t * C::kSlotBytes + c * 16384), &map_q, c, (u.qt0 + t) * kTile, u.g.q0, u.bh,
+                     u.h, packed, bq);
         while (ok && it.next(j, fl)) {
           for (int kv = 0; kv < 2; ++kv) {
             const int s = n % NS;
@@ -170,7 +179,8 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
             ptx::mbar_arrive_expect_tx(bf, C::kSlotBytes);
             const CUtensorMap* map = kv == 0 ? &map_k : &map_v;
             for (int c = 0; c < C::kSubTiles; ++c)
-              ptx::tma_load_3d(ptx::smem_addr(sKV + s * C::kSlotBytes + c * 16384), map, 64 * c, j * kTile, u.bh, bf);
+              tma_rows(ptx::smem_addr(sKV + s * C::kSlotBytes + c * 16384), map, c, j * kTile, u.g.k0, u.bh, u.h,
+                       packed, bf);
             ++n;
           }
         }
@@ -397,11 +407,12 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
       ok = __all_sync(0xffffffffu, wait_or_abort(ptx::smem_addr(&bar_o[t]), ku & 1, args.budget_ns, abortp));
       if (!ok) break;
       ptx::tc_fence_after();
-      const bool row_ok = grow < args.N && (t == 0 || u.has1);
+      const bool row_ok = grow < u.g.lq && (t == 0 || u.has1);
       const float l_sum = (lacc[0].x + lacc[0].y) + (lacc[1].x + lacc[1].y);
       const bool nonempty = l_sum > 0.f;
       const float inv = nonempty ? 1.0f / l_sum : 0.0f;
-      uint8_t* orow = reinterpret_cast<uint8_t*>(args.o) + ((size_t)u.bh * args.N + grow) * D * 2;
+      const size_t orow_idx = packed ? (size_t)(u.g.q0 + grow) * args.H + u.h : (size_t)u.bh * args.N + grow;
+      uint8_t* orow = reinterpret_cast<uint8_t*>(args.o) + orow_idx * D * 2;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t orr[32];
@@ -424,9 +435,10 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
           for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
         }
       }
-      if (row_ok)
-        args.lse[(size_t)u.bh * args.N + grow] = nonempty ? (m_ref + __log2f(l_sum)) * 0.69314718055994530942f
-                                                          : -INFINITY;
+      if (row_ok) {
+        const size_t li = packed ? (size_t)u.h * args.total_q + u.g.q0 + grow : (size_t)u.bh * args.N + grow;
+        args.lse[li] = nonempty ? (m_ref + __log2f(l_sum)) * 0.69314718055994530942f : -INFINITY;
+      }
       ++ku;
     }
   }

@@ -15,7 +15,7 @@
 
 namespace {
 
-constexpr int kVersion = 10000;  // 1.0.0
+constexpr int kVersion = 10100;  // 1.1.0: packed variable-length batches
 constexpr int kMaxN = 1 << 20;
 constexpr long long kMaxElems = 1LL << 34;
 
@@ -88,6 +88,29 @@ int make_map(CUtensorMap* m, const void* ptr, int BH, int N, int d, int dtype) {
   return FA_OK;
 }
 
+// {d, H, total} view of a packed [total, H, d] tensor with a {64, 1, 128} box: 128 consecutive tokens of one head,
+// 64 columns (128 bytes), 128-byte swizzle -- the same shared-memory image as the dense box.  Tokens past `total`
+// read as zero.
+int make_map_packed(CUtensorMap* m, const void* ptr, int total, int H, int d, int dtype) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) {
+    t_last_error = "cuTensorMapEncodeTiled unavailable";
+    return FA_ERR_CUDA;
+  }
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)total};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2};
+  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = enc(m, dtype == FA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+                   const_cast<void*>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    t_last_error = "cuTensorMapEncodeTiled (packed) failed with CUresult " + std::to_string((int)r);
+    return FA_ERR_CUDA;
+  }
+  return FA_OK;
+}
+
 // 2-D fp32 view {cols, rows} of the dQ accumulator for TMA reduce-add: box 32 columns (128 bytes) x 32 rows,
 // 128-byte swizzle (matches the drain warps' staging layout).
 int make_map_f32(CUtensorMap* m, void* ptr, long long rows, int cols) {
@@ -152,20 +175,38 @@ int fwd_tiles_for(int d) {
   return d == 64 ? 1 : 2;
 }
 
+// Packed variable-length batch description (all null / zero for the dense [B, H, N, d] layout).
+struct Packed {
+  const int32_t* cu_q = nullptr;
+  const int32_t* cu_k = nullptr;
+  int total_q = 0, total_k = 0, Nk = 0;
+};
+
 int run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
             float scale, int causal, const int32_t* key_lens, const int32_t* row_ptr, const int32_t* col_idx,
-            int dtype, cudaStream_t st) {
+            int dtype, cudaStream_t st, const Packed& pk = Packed()) {
   CUtensorMap mq, mk, mv;
   int rc;
-  if ((rc = make_map(&mq, q, B * H, N, d, dtype)) != FA_OK) return rc;
-  if ((rc = make_map(&mk, k, B * H, N, d, dtype)) != FA_OK) return rc;
-  if ((rc = make_map(&mv, v, B * H, N, d, dtype)) != FA_OK) return rc;
+  if (pk.cu_q) {
+    if ((rc = make_map_packed(&mq, q, pk.total_q, H, d, dtype)) != FA_OK) return rc;
+    if ((rc = make_map_packed(&mk, k, pk.total_k, H, d, dtype)) != FA_OK) return rc;
+    if ((rc = make_map_packed(&mv, v, pk.total_k, H, d, dtype)) != FA_OK) return rc;
+  } else {
+    if ((rc = make_map(&mq, q, B * H, N, d, dtype)) != FA_OK) return rc;
+    if ((rc = make_map(&mk, k, B * H, N, d, dtype)) != FA_OK) return rc;
+    if ((rc = make_map(&mv, v, B * H, N, d, dtype)) != FA_OK) return rc;
+  }
   fa::FwdArgs a;
   a.o = o;
   a.lse = lse;
   a.key_lens = key_lens;
   a.row_ptr = row_ptr;
   a.col_idx = col_idx;
+  a.cu_q = pk.cu_q;
+  a.cu_k = pk.cu_k;
+  a.total_q = pk.total_q;
+  a.total_k = pk.total_k;
+  a.Nk = pk.cu_q ? pk.Nk : N;
   a.H = H;
   a.N = N;
   a.nT = (N + fa::kTile - 1) / fa::kTile;
@@ -316,6 +357,74 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
   cudaError_t e = fa::run_bwd(mq, mk, mv, mdo, mdq, o, dout, lse, dq, dk, dv, B, H, N, d, softmax_scale, causal != 0,
                               key_lens, col_ptr, row_idx, workspace, dtype == FA_BF16, g_budget_ns.load(), st,
                               t_events[FA_KERNEL_BWD_MAIN][0], t_events[FA_KERNEL_BWD_MAIN][1]);
+  return e == cudaSuccess ? FA_OK : cuda_fail(e);
+}
+
+// ------------------------------------------------------------------------------------------ packed batches
+int check_packed(const void* q, const void* k, const void* v, const int32_t* cu_q, const int32_t* cu_k, int B, int H,
+                 int max_q, int max_k, int total_q, int total_k, int d, float scale, int dtype) {
+  if (!q || !k || !v || !cu_q || !cu_k) return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(cu_q, 4) || !aligned(cu_k, 4))
+    return FA_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || max_q < 1 || max_k < 1 || max_q > kMaxN || max_k > kMaxN) return FA_ERR_INVALID_ARG;
+  if (total_q < 1 || total_k < 1) return FA_ERR_INVALID_ARG;
+  if (dtype != FA_BF16 && dtype != FA_FP16) return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.0f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  const long long npad = (long long)(max_q + fa::kTile - 1) / fa::kTile * fa::kTile;
+  if ((long long)total_q * H * d > kMaxElems || (long long)total_k * H * d > kMaxElems ||
+      (long long)B * H * npad * d > kMaxElems)
+    return FA_ERR_INVALID_ARG;
+  return FA_OK;
+}
+
+int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int32_t* cu_seqlens_q,
+                  const int32_t* cu_seqlens_k, int B, int H, int max_seqlen_q, int max_seqlen_k, int total_q,
+                  int total_k, int d, float softmax_scale, int causal, int dtype, void* stream) {
+  int rc = check_packed(q, k, v, cu_seqlens_q, cu_seqlens_k, B, H, max_seqlen_q, max_seqlen_k, total_q, total_k, d,
+                        softmax_scale, dtype);
+  if (rc != FA_OK) return rc;
+  if (!o || !lse || !aligned(o, 16) || !aligned(lse, 4)) return FA_ERR_INVALID_ARG;
+  Packed pk;
+  pk.cu_q = cu_seqlens_q;
+  pk.cu_k = cu_seqlens_k;
+  pk.total_q = total_q;
+  pk.total_k = total_k;
+  pk.Nk = max_seqlen_k;
+  return run_fwd(q, k, v, o, lse, B, H, max_seqlen_q, d, softmax_scale, causal, nullptr, nullptr, nullptr, dtype,
+                 static_cast<cudaStream_t>(stream), pk);
+}
+
+size_t fa_bwd_varlen_workspace_size(int B, int H, int max_seqlen_q, int d) {
+  if (B < 1 || H < 1 || max_seqlen_q < 1 || max_seqlen_q > kMaxN || (d != 64 && d != 128)) return 0;
+  return fa::bwd_workspace_bytes(B * H, (max_seqlen_q + fa::kTile - 1) / fa::kTile, d);
+}
+
+int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                  void* dq, void* dk, void* dv, const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int B, int H,
+                  int max_seqlen_q, int max_seqlen_k, int total_q, int total_k, int d, float softmax_scale, int causal,
+                  void* workspace, size_t workspace_bytes, int dtype, void* stream) {
+  int rc = check_packed(q, k, v, cu_seqlens_q, cu_seqlens_k, B, H, max_seqlen_q, max_seqlen_k, total_q, total_k, d,
+                        softmax_scale, dtype);
+  if (rc != FA_OK) return rc;
+  if (!o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  if (!aligned(o, 16) || !aligned(dout, 16) || !aligned(lse, 4) || !aligned(dq, 16) || !aligned(dk, 16) ||
+      !aligned(dv, 16))
+    return FA_ERR_INVALID_ARG;
+  const size_t need = fa_bwd_varlen_workspace_size(B, H, max_seqlen_q, d);
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < need) return FA_ERR_WORKSPACE;
+  CUtensorMap mq, mk, mv, mdo, mdq;
+  if ((rc = make_map_packed(&mq, q, total_q, H, d, dtype)) != FA_OK) return rc;
+  if ((rc = make_map_packed(&mk, k, total_k, H, d, dtype)) != FA_OK) return rc;
+  if ((rc = make_map_packed(&mv, v, total_k, H, d, dtype)) != FA_OK) return rc;
+  if ((rc = make_map_packed(&mdo, dout, total_q, H, d, dtype)) != FA_OK) return rc;
+  const int nTq = (max_seqlen_q + fa::kTile - 1) / fa::kTile;
+  if ((rc = make_map_f32(&mdq, workspace, (long long)B * H * nTq * fa::kTile, d)) != FA_OK) return rc;
+  cudaError_t e = fa::run_bwd(mq, mk, mv, mdo, mdq, o, dout, lse, dq, dk, dv, B, H, max_seqlen_q, d, softmax_scale,
+                              causal != 0, nullptr, nullptr, nullptr, workspace, dtype == FA_BF16, g_budget_ns.load(),
+                              static_cast<cudaStream_t>(stream), t_events[FA_KERNEL_BWD_MAIN][0],
+                              t_events[FA_KERNEL_BWD_MAIN][1], cu_seqlens_q, cu_seqlens_k, total_q, total_k,
+                              max_seqlen_k);
   return e == cudaSuccess ? FA_OK : cuda_fail(e);
 }
 

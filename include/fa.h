@@ -91,8 +91,9 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d, int has_block_mask);
  * Backward (review page claim C7: P is recomputed tile by tile from the saved LSE; the N x N matrix never exists
  * in HBM).  Inputs q, k, v, o, dO [B,H,N,d] and lse [B,H,N] from fa_fwd with the same mask arguments; outputs
  * dq, dk, dv [B,H,N,d] (fully overwritten).  block_mask may be NULL.  Runs a preprocessing kernel (D = rowsum(dO*O),
- * zeroed dQ accumulator), the main kernel (one CTA per 128-key tile, looping over the visible Q tiles; dK, dV
- * accumulate on chip, dQ by fp32 atomics into the workspace) and a conversion kernel for dQ.
+ * zeroed dQ accumulator), the main kernel (persistent CTAs, each walking 128-key tiles and, per tile, the visible
+ * Q tiles; dK, dV accumulate on chip, dQ partial sums go into the fp32 accumulator in the workspace by bulk
+ * reduce-add) and a conversion kernel for dQ.
  */
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
            void* dq, void* dk, void* dv, int B, int H, int N, int d, float softmax_scale, int causal,
@@ -107,6 +108,34 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
  */
 int fa_blockmask_lists(const uint8_t* mask, int nT, int32_t* row_ptr, int32_t* col_idx, int32_t* col_ptr,
                        int32_t* row_idx, void* stream);
+
+/*
+ * Packed variable-length batches.  The pages give no interface for this (it generalises the key-length masking
+ * they describe for padded BERT batches, explainer page, block-sparse and masking section): B sequences of
+ * different lengths are stored back to back without padding.
+ *   Layout      q, o, dO, dq: [total_q, H, d]; k, v, dk, dv: [total_k, H, d] (token-major, d innermost, 16-bit);
+ *               lse: [H, total_q] fp32 (natural log, -inf for a row with no visible key).
+ *               cu_seqlens_q [B+1], cu_seqlens_k [B+1]: int32 device arrays, cu[0] = 0, non-decreasing,
+ *               cu[B] = total; sequence b is tokens cu[b] .. cu[b+1]-1.  len_q(b) <= max_seqlen_q and
+ *               len_k(b) <= max_seqlen_k (both <= 2^20).  Values outside these rules are clamped into range on the
+ *               device (no access leaves the tensors) but the results for such sequences are unspecified.
+ *   Visibility  Key c of sequence b is visible from its query r (positions within the sequence) iff
+ *               c < len_k(b) && (causal == 0 || c <= r).  For len_q == len_k this is ordinary causal self-attention.
+ *   Shapes      total_q, total_k >= 1; total*H*d and B*H*ceil(max_seqlen_q/128)*128*d <= 2^34; d in {64, 128}.
+ * Everything else (pointers, execution, errors) is as for fa_fwd / fa_bwd.  No block mask, no key_lens.
+ */
+int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int32_t* cu_seqlens_q,
+                  const int32_t* cu_seqlens_k, int B, int H, int max_seqlen_q, int max_seqlen_k, int total_q,
+                  int total_k, int d, float softmax_scale, int causal, int dtype, void* stream);
+
+/* Bytes of workspace fa_bwd_varlen needs (fp32 dQ accumulator and per-row LSE/D over B*H padded sequences). */
+size_t fa_bwd_varlen_workspace_size(int B, int H, int max_seqlen_q, int d);
+
+/* Backward of fa_fwd_varlen: dq [total_q,H,d], dk, dv [total_k,H,d] (fully overwritten); same kernels as fa_bwd. */
+int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                  void* dq, void* dk, void* dv, const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int B, int H,
+                  int max_seqlen_q, int max_seqlen_k, int total_q, int total_k, int d, float softmax_scale, int causal,
+                  void* workspace, size_t workspace_bytes, int dtype, void* stream);
 
 /*
  * Synchronises `stream`, then returns and clears the current device's status word: FA_OK, or FA_ERR_TIMEOUT if a

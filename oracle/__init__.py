@@ -175,6 +175,70 @@ def attn_bwd_keys(q, k, v, do, scale, sel_bh, sel_c, causal=False, key_lens=None
     return dk, dv
 
 
+def _varlen_slices(cu_q, cu_k):
+    cu_q = np.asarray(cu_q, dtype=np.int64)
+    cu_k = np.asarray(cu_k, dtype=np.int64)
+    if cu_q.shape != cu_k.shape or cu_q.ndim != 1 or cu_q.size < 2:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must be 1-D of the same length B+1 >= 2")
+    for b in range(cu_q.size - 1):
+        yield int(cu_q[b]), int(cu_q[b + 1]), int(cu_k[b]), int(cu_k[b + 1])
+
+
+def _pad_seq(x, a, e, n):
+    """Tokens a..e-1 of a [total, H, d] array as a [1, H, n, d] problem, zero rows after e-a."""
+    t = np.zeros((1, x.shape[1], n, x.shape[2]))
+    t[0, :, :e - a] = x[a:e].transpose(1, 0, 2)
+    return t
+
+
+def attn_fwd_varlen(q, k, v, cu_q, cu_k, scale, causal=False):
+    """Packed variable-length batch (q [total_q,H,d], k, v [total_k,H,d]): sequence b is standard attention of its
+    own queries cu_q[b]..cu_q[b+1]-1 against its own keys cu_k[b]..cu_k[b+1]-1, causal meaning key c <= query r
+    within the sequence.  Each sequence is run through attn_fwd zero-padded to n = max(len_q, len_k) rows with
+    key_lens = [len_k]; the padded query rows are dropped.  Returns (O [total_q,H,d], LSE [H,total_q]) in fp64."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    total_q, H, d = q.shape
+    o = np.zeros((total_q, H, d))
+    lse = np.full((H, total_q), -np.inf)
+    for a, e, ak, ek in _varlen_slices(cu_q, cu_k):
+        lq, lk = e - a, ek - ak
+        if lq <= 0:
+            continue
+        n = max(lq, lk)
+        ob, lb = attn_fwd(_pad_seq(q, a, e, n), _pad_seq(k, ak, ek, n), _pad_seq(v, ak, ek, n), scale, causal=causal,
+                          key_lens=np.array([lk], dtype=np.int32))
+        o[a:e] = ob[0, :, :lq].transpose(1, 0, 2)
+        lse[:, a:e] = lb[0, :, :lq]
+    return o, lse
+
+
+def attn_bwd_varlen(q, k, v, do, cu_q, cu_k, scale, causal=False):
+    """Gradients of sum(O * dO) for attn_fwd_varlen, per sequence through attn_bwd (padded query rows carry dO = 0,
+    so they add nothing).  Returns (dQ [total_q,H,d], dK, dV [total_k,H,d], O, LSE [H,total_q])."""
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    total_q, H, d = q.shape
+    total_k = k.shape[0]
+    dq = np.zeros((total_q, H, d))
+    dk = np.zeros((total_k, H, d))
+    dv = np.zeros((total_k, H, d))
+    o = np.zeros((total_q, H, d))
+    lse = np.full((H, total_q), -np.inf)
+    for a, e, ak, ek in _varlen_slices(cu_q, cu_k):
+        lq, lk = e - a, ek - ak
+        if lq <= 0 and lk <= 0:
+            continue
+        n = max(lq, lk, 1)
+        gq, gk, gv, ob, lb = attn_bwd(_pad_seq(q, a, e, n), _pad_seq(k, ak, ek, n), _pad_seq(v, ak, ek, n),
+                                      _pad_seq(do, a, e, n), scale, causal=causal,
+                                      key_lens=np.array([lk], dtype=np.int32))
+        dq[a:e] = gq[0, :, :lq].transpose(1, 0, 2)
+        dk[ak:ek] = gk[0, :, :lk].transpose(1, 0, 2)
+        dv[ak:ek] = gv[0, :, :lk].transpose(1, 0, 2)
+        o[a:e] = ob[0, :, :lq].transpose(1, 0, 2)
+        lse[:, a:e] = lb[0, :, :lq]
+    return dq, dk, dv, o, lse
+
+
 def blockmask_csr(mask):
     """CSR of a square 0/1 tile mask: (row_ptr [nT+1] int32, col_idx [nnz] int32), ascending columns."""
     m = np.ascontiguousarray(mask, dtype=np.uint8)

@@ -306,3 +306,108 @@ def test_lists_match_brute_force_random_masks():
     empty = np.zeros((4, 4), np.uint8)
     rp, ci = oracle.blockmask_csr(empty)
     assert rp.tolist() == [0] * 5 and ci.size == 0
+
+
+# ----------------------------------------------------------------------------------------------- packed batches
+# The packed variable-length oracle composes the pinned dense oracle with per-sequence slicing and padding; these
+# pins check the composition against the dense batch it must reduce to, against reordering and independence of
+# the sequences, against calculus (finite differences of a cross-length case) and the per-sequence invariants.
+def _packed(x):
+    """[B, H, N, d] -> packed [B*N, H, d] with cu = 0, N, 2N, ..."""
+    B, H, N, d = x.shape
+    return x.transpose(0, 2, 1, 3).reshape(B * N, H, d)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_varlen_equal_lengths_equal_dense_batch(causal):
+    B, H, N, d = 3, 2, 11, 4
+    q, k, v = qkv(B, H, N, d, 160)
+    do = rnd((B, H, N, d), 161)
+    cu = np.arange(B + 1, dtype=np.int32) * N
+    o, lse = oracle.attn_fwd(q, k, v, 0.4, causal=causal)
+    ov, lv = oracle.attn_fwd_varlen(_packed(q), _packed(k), _packed(v), cu, cu, 0.4, causal=causal)
+    np.testing.assert_allclose(ov, _packed(o), rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lv, lse.transpose(1, 0, 2).reshape(H, B * N), rtol=0, atol=1e-13)
+    dq, dk, dv, _, _ = oracle.attn_bwd(q, k, v, do, 0.4, causal=causal)
+    gq, gk, gv, _, _ = oracle.attn_bwd_varlen(_packed(q), _packed(k), _packed(v), _packed(do), cu, cu, 0.4,
+                                              causal=causal)
+    for a, b in ((gq, dq), (gk, dk), (gv, dv)):
+        np.testing.assert_allclose(a, _packed(b), rtol=0, atol=1e-13)
+
+
+def test_varlen_sequences_are_independent_and_order_free():
+    H, d = 2, 4
+    lq, lk = [5, 0, 9, 3], [7, 4, 9, 1]
+    cq, ck = np.concatenate([[0], np.cumsum(lq)]), np.concatenate([[0], np.cumsum(lk)])
+    q, k, v = rnd((cq[-1], H, d), 170), rnd((ck[-1], H, d), 171), rnd((ck[-1], H, d), 172)
+    o, lse = oracle.attn_fwd_varlen(q, k, v, cq, ck, 0.5)
+    # each sequence alone gives the same rows
+    for b in range(4):
+        if lq[b] == 0:
+            continue
+        ob, lb = oracle.attn_fwd_varlen(q[cq[b]:cq[b + 1]], k[ck[b]:ck[b + 1]], v[ck[b]:ck[b + 1]],
+                                        [0, lq[b]], [0, lk[b]], 0.5)
+        np.testing.assert_allclose(ob, o[cq[b]:cq[b + 1]], rtol=0, atol=1e-14)
+        np.testing.assert_allclose(lb, lse[:, cq[b]:cq[b + 1]], rtol=0, atol=1e-14)
+    # reversing the sequence order reverses the blocks
+    perm = [3, 2, 1, 0]
+    q2 = np.concatenate([q[cq[b]:cq[b + 1]] for b in perm])
+    k2 = np.concatenate([k[ck[b]:ck[b + 1]] for b in perm])
+    v2 = np.concatenate([v[ck[b]:ck[b + 1]] for b in perm])
+    cq2 = np.concatenate([[0], np.cumsum([lq[b] for b in perm])])
+    ck2 = np.concatenate([[0], np.cumsum([lk[b] for b in perm])])
+    o2, _ = oracle.attn_fwd_varlen(q2, k2, v2, cq2, ck2, 0.5)
+    np.testing.assert_allclose(o2, np.concatenate([o[cq[b]:cq[b + 1]] for b in perm]), rtol=0, atol=1e-14)
+
+
+def test_varlen_empty_key_sequence_and_key_count_one():
+    H, d = 1, 3
+    q, k, v = rnd((4, H, d), 180), rnd((3, H, d), 181), rnd((3, H, d), 182)
+    # sequence 0: 2 queries, 0 keys -> O = 0, LSE = -inf; sequence 1: 2 queries, 3 keys, causal -> query 0 sees key 0
+    o, lse = oracle.attn_fwd_varlen(q, k, v, [0, 2, 4], [0, 0, 3], 1.0, causal=True)
+    assert np.all(o[:2] == 0) and np.all(np.isneginf(lse[:, :2]))
+    np.testing.assert_allclose(o[2], v[0], rtol=0, atol=1e-15)
+    np.testing.assert_allclose(lse[:, 2], np.sum(q[2] * k[0], axis=-1), atol=1e-15)  # one visible key: LSE = scale*q.k
+
+
+def test_varlen_cross_lengths_match_central_differences():
+    H, d = 1, 3
+    lq, lk = [3, 4], [5, 2]
+    cq, ck = np.array([0, 3, 7]), np.array([0, 5, 7])
+    q, k, v = rnd((7, H, d), 190), rnd((7, H, d), 191), rnd((7, H, d), 192)
+    do = rnd((7, H, d), 193)
+    s = 0.7
+    for causal in (False, True):
+        dq, dk, dv, _, _ = oracle.attn_bwd_varlen(q, k, v, do, cq, ck, s, causal=causal)
+
+        def loss(qq, kk, vv):
+            o, _ = oracle.attn_fwd_varlen(qq, kk, vv, cq, ck, s, causal=causal)
+            return float(np.sum(o * do))
+
+        h = 1e-6
+        for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+            fd = np.zeros_like(x)
+            for idx in np.ndindex(x.shape):
+                xp, xm = x.copy(), x.copy()
+                xp[idx] += h
+                xm[idx] -= h
+                a = {"q": q, "k": k, "v": v}
+                m = dict(a)
+                a[name], m[name] = xp, xm
+                fd[idx] = (loss(a["q"], a["k"], a["v"]) - loss(m["q"], m["k"], m["v"])) / (2 * h)
+            err = np.max(np.abs(fd - g)) / max(np.max(np.abs(g)), 1e-30)
+            assert err <= 1e-6, (causal, name, err)
+
+
+def test_varlen_gradient_invariants_per_sequence():
+    H, d = 2, 5
+    lq, lk = [6, 13, 1], [9, 13, 4]
+    cq, ck = np.concatenate([[0], np.cumsum(lq)]), np.concatenate([[0], np.cumsum(lk)])
+    q, k, v = rnd((cq[-1], H, d), 200), rnd((ck[-1], H, d), 201), rnd((ck[-1], H, d), 202)
+    do = rnd((cq[-1], H, d), 203)
+    dq, dk, dv, o, lse = oracle.attn_bwd_varlen(q, k, v, do, cq, ck, 0.45, causal=True)
+    for b in range(3):
+        ks, qs = slice(ck[b], ck[b + 1]), slice(cq[b], cq[b + 1])
+        np.testing.assert_allclose(dk[ks].sum(axis=0), 0.0, atol=1e-11)
+        nonempty = np.isfinite(lse[:, qs]).T[..., None]
+        np.testing.assert_allclose(dv[ks].sum(axis=0), (do[qs] * nonempty).sum(axis=0), atol=1e-11)
