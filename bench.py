@@ -278,6 +278,67 @@ def measure_targets(stream, flush, peak):
     return out
 
 
+def measure_varlen(stream, flush, peak):
+    """Packed variable-length batch (BERT-large shape: B16 H16 d64 bf16, non-causal, the BERT workload's sequence
+    lengths U[128, 512]) through fa_fwd_varlen / fa_bwd_varlen, next to the same sequences padded to N = 512 with
+    key lengths (the dense entry points).  TFLOP/s count the same visible pairs (sum over sequences of len^2) for
+    both; the padded run also spends time on the padding rows' queries."""
+    import numpy as np
+    import torch
+    from exact_io_aware_48_b200 import _lib, inputs
+    w = inputs.workloads()["bert"]
+    lens = [int(x) for x in w.key_lens_array()]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    total, H, d, B = int(cu[-1]), w.H, w.d, w.B
+    q, k, v, do = (inputs.gaussian((total, H, d), w.seed * 1000 + 50 + t, "bf16").cuda() for t in range(4))
+    o = torch.empty_like(q)
+    lse = torch.empty((H, total), device="cuda", dtype=torch.float32)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    cud = torch.as_tensor(cu).cuda()
+    mx = max(lens)
+    ws_bytes = _lib.fa_bwd_varlen_workspace_size(B, H, mx, d)
+    ws = torch.empty(ws_bytes, device="cuda", dtype=torch.uint8)
+    scale = 1.0 / math.sqrt(d)
+
+    def fwd(st):
+        rc = _lib.fa_fwd_varlen(q, k, v, o, lse, cud, cud, B, H, mx, mx, total, total, d, scale, False, _lib.FA_BF16,
+                                st)
+        if rc:
+            raise RuntimeError(f"fa_fwd_varlen: {_lib.fa_status_string(rc)}")
+
+    def bwd(st):
+        rc = _lib.fa_bwd_varlen(q, k, v, o, do, lse, dq, dk, dv, cud, cud, B, H, mx, mx, total, total, d, scale, False,
+                                ws, ws_bytes, _lib.FA_BF16, st)
+        if rc:
+            raise RuntimeError(f"fa_bwd_varlen: {_lib.fa_status_string(rc)}")
+
+    pairs = H * sum(n * n for n in lens)
+    flops = fwd_flops(d, pairs)
+    for _ in range(3):
+        fwd(stream)
+        bwd(stream)
+    f_ms, _ = time_loop(fwd, 10, stream, flush)
+    b_ms, _ = time_loop(bwd, 10, stream, flush)
+    f, b = statistics.median(f_ms), statistics.median(b_ms)
+    status = _lib.fa_last_device_status(stream)
+    if status:
+        raise RuntimeError(f"packed-batch kernels reported {_lib.fa_status_string(status)}")
+    padded = Problem(w)  # the same shape padded to N with key lengths
+    for _ in range(3):
+        padded.step(stream)
+    pf_ms, _ = time_loop(padded.fwd, 10, stream, flush)
+    pb_ms, _ = time_loop(padded.bwd, 10, stream, flush)
+    pf, pb = statistics.median(pf_ms), statistics.median(pb_ms)
+    out = {"workload": f"packed BERT-large shape B{B} H{H} d{d} bf16, lengths U[128,512], total {total} tokens",
+           "fwd_ms": round(f, 4), "bwd_ms": round(b, 4),
+           "fwd_tflops": round(flops / f / 1e9, 1), "bwd_tflops": round(2.5 * flops / b / 1e9, 1),
+           "fwd_bwd_tflops": round(3.5 * flops / (f + b) / 1e9, 1),
+           "padded_key_lens_fwd_bwd_ms": round(pf + pb, 4), "padded_key_lens_fwd_bwd_tflops":
+           round(3.5 * flops / (pf + pb) / 1e9, 1)}
+    del padded
+    return out
+
+
 def run_ours(args):
     import numpy as np
     import torch
@@ -340,6 +401,7 @@ def run_ours(args):
     e2e = run_e2e(p, stream, args, world) if args.e2e else None
 
     targets = measure_targets(stream, flush, peak) if (args.targets and rank == 0) else None
+    varlen = measure_varlen(stream, flush, peak) if (args.targets and rank == 0) else None
     cpu = cpu_baseline(p.w) if rank == 0 and world == 1 and args.cpu_baseline else None
 
     if rank == 0:
@@ -360,6 +422,7 @@ def run_ours(args):
             "gpu_launches": 4 * args.steps,
             "clocks": clk.summary(),
             "targets": targets,
+            "varlen": varlen,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)

@@ -73,13 +73,14 @@ struct FwdUnit {
   bool has1;
 };
 
+template <bool kPacked>
 __device__ __forceinline__ FwdUnit fwd_unit(int L, const FwdArgs& a, int tiles) {
   FwdUnit u;
   const int pair = a.npairs - 1 - L / a.BH;
   u.bh = L % a.BH;
   u.h = u.bh % a.H;
   u.qt0 = tiles * pair;
-  u.g = seq_geom(a.cu_q, a.cu_k, a.key_lens, u.bh / a.H, a.N, a.Nk, a.total_q, a.total_k);
+  u.g = seq_geom(kPacked ? a.cu_q : nullptr, a.cu_k, a.key_lens, u.bh / a.H, a.N, a.Nk, a.total_q, a.total_k);
   const int nTq = (u.g.lq + kTile - 1) / kTile;  // Q tiles of this sequence
   u.has1 = tiles == 2 && u.qt0 + 1 < nTq;
   u.kv_lim = u.g.lk;
@@ -96,7 +97,9 @@ __device__ __forceinline__ void fwd_tiles(PairTileIter& it, const FwdUnit& u, co
     it.init_dense(u.end0, u.end1);
 }
 
-template <int D, bool kBF16, int kTiles>
+// kPacked: packed variable-length batch (FwdArgs::cu_q set); a separate instantiation so the dense kernels carry
+// none of its state.
+template <int D, bool kBF16, int kTiles, bool kPacked>
 __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
     fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                const __grid_constant__ CUtensorMap map_v, const FwdArgs args) {
@@ -115,7 +118,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const bool causal = args.causal != 0;
-  const bool packed = args.cu_q != nullptr;
+  constexpr bool packed = kPacked;
   const int total_units = args.npairs * args.BH;
 
   if (threadIdx.x == 0) {
@@ -160,7 +163,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
       int n = 0, ku = 0, j, fl;
       bool ok = true;
       while (ok && us.next(L)) {
-        const FwdUnit u = fwd_unit(L, args, kTiles);
+        const FwdUnit u = fwd_unit<kPacked>(L, args, kTiles);
         PairTileIter it;
         fwd_tiles(it, u, args);
         // the Q buffer is free once every S MMA of the previous unit has completed
@@ -247,7 +250,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
       };
 
       while (ok && us.next(L)) {
-        const FwdUnit u = fwd_unit(L, args, kTiles);
+        const FwdUnit u = fwd_unit<kPacked>(L, args, kTiles);
         PairTileIter it;
         fwd_tiles(it, u, args);
         if (!(ok = wait_or_abort(ptx::smem_addr(&bar_q), ku & 1, args.budget_ns, abortp))) break;
@@ -293,6 +296,12 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
           if (ok) ok = flush_pv(t);
         if (!ok) break;
         if (pend_flags) ptx::mma_commit(ptx::smem_addr(&bar_empty[pend_slot]));
+        // A tile that had no P V in this unit did not wait for the previous unit's epilogue; wait now, or two
+        // back-to-back empty units would complete two phases of bar_o before its softmax warps look (ABA).
+        for (int t = 0; t < kTiles && ok; ++t)
+          if (pv_count[t] == 0 && ku > 0)
+            ok = wait_or_abort(ptx::smem_addr(&bar_o_free[t]), (ku - 1) & 1, args.budget_ns, abortp);
+        if (!ok) break;
         ptx::mma_commit(ptx::smem_addr(&bar_o[0]));
         ptx::mma_commit(ptx::smem_addr(&bar_o[1]));
         ++ku;
@@ -314,7 +323,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
     int ku = 0;
     bool ok = true;
     while (ok && us.next(L)) {
-      const FwdUnit u = fwd_unit(L, args, kTiles);
+      FwdUnit u = fwd_unit<kPacked>(L, args, kTiles);
       PairTileIter it;
       fwd_tiles(it, u, args);
       const int qt = u.qt0 + t;
@@ -407,6 +416,9 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
       ok = __all_sync(0xffffffffu, wait_or_abort(ptx::smem_addr(&bar_o[t]), ku & 1, args.budget_ns, abortp));
       if (!ok) break;
       ptx::tc_fence_after();
+      // packed: the unit is worked out again rather than kept in registers through the K/V loop (the softmax
+      // warps are at their register limit and the packed unit carries more state)
+      if constexpr (kPacked) u = fwd_unit<kPacked>(L, args, kTiles);
       const bool row_ok = grow < u.g.lq && (t == 0 || u.has1);
       const float l_sum = (lacc[0].x + lacc[0].y) + (lacc[1].x + lacc[1].y);
       const bool nonempty = l_sum > 0.f;

@@ -146,12 +146,12 @@ cudaError_t ensure_smem(Kernel kernel, int bytes, std::atomic<uint64_t>& done_ma
   return e;
 }
 
-template <int D, bool BF, int T>
-cudaError_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, fa::FwdArgs a,
-                       cudaStream_t st) {
+template <int D, bool BF, int T, bool P>
+cudaError_t launch_fwd_k(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, fa::FwdArgs a,
+                         cudaStream_t st) {
   using C = fa::FwdCfg<D, T>;
   static std::atomic<uint64_t> smem_set{0};
-  cudaError_t e = ensure_smem(fa::fwd_kernel<D, BF, T>, C::kSmemBytes, smem_set);
+  cudaError_t e = ensure_smem(fa::fwd_kernel<D, BF, T, P>, C::kSmemBytes, smem_set);
   if (e != cudaSuccess) return e;
   a.npairs = (a.nT + T - 1) / T;  // work units (groups of T Q tiles) per (b, h)
   // persistent: as many CTAs as fit at once (3 - T per SM), each walking its share of the units
@@ -161,9 +161,15 @@ cudaError_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   const long long units = (long long)a.BH * a.npairs;
   const unsigned grid = (unsigned)std::min<long long>(units, (long long)sms * (3 - T));
   if ((e = mark(FA_KERNEL_FWD, 0, st)) != cudaSuccess) return e;
-  fa::fwd_kernel<D, BF, T><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mk, mv, a);
+  fa::fwd_kernel<D, BF, T, P><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mk, mv, a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   return mark(FA_KERNEL_FWD, 1, st);
+}
+
+template <int D, bool BF, int T>
+cudaError_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const fa::FwdArgs& a,
+                       cudaStream_t st) {
+  return a.cu_q ? launch_fwd_k<D, BF, T, true>(mq, mk, mv, a, st) : launch_fwd_k<D, BF, T, false>(mq, mk, mv, a, st);
 }
 
 // Q tiles per forward CTA for this call (see FwdCfg).  Measured on B200 (bf16, causal): d = 64 prefers one-tile

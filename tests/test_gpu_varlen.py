@@ -72,3 +72,39 @@ def test_varlen_equal_lengths_match_dense_kernels():
     for a, b in ((gq, dq), (gk, dk), (gv, dv)):
         ref = pk(b).float()
         assert float((a.float() - ref).abs().max()) <= 5e-2 * float(ref.abs().max())
+
+
+def test_varlen_many_empty_units_per_cta():
+    """Sixty-four short sequences and one long one: most (Q tile, head) units of the longest-first order are past
+    their sequence's end, so each persistent CTA walks several empty units back to back (a case that once left the
+    forward's per-unit output barrier two phases ahead of its softmax warps)."""
+    lens = [100] * 64 + [512]
+    cq, ck, q, k, v, do, mq, mk = packed_case(lens, None, 16, 64, "bf16", 37)
+    scale = 0.125
+    cqd = torch.as_tensor(cq).cuda()
+    qd, kd, vd, dod = q.cuda(), k.cuda(), v.cuda(), do.cuda()
+    # non-causal: every row averages its whole sequence, so |O| stays well inside the range where the 16-bit
+    # output rounding is far below the 1e-2 bound (rows that see one or two keys of a gaussian V can reach |O| ~ 5,
+    # where one bf16 rounding step alone is ~8e-3); the unit schedule under test does not depend on the mask
+    o, lse = fa.attention_fwd_varlen(qd, kd, vd, cqd, cqd, mq, mk, causal=False, softmax_scale=scale)
+    dq, dk, dv = fa.attention_bwd_varlen(qd, kd, vd, o, dod, lse, cqd, cqd, mq, mk, causal=False, softmax_scale=scale)
+    assert fa.last_device_status() == 0
+    rdq, rdk, rdv, ro, rl = oracle.attn_bwd_varlen(f64(q), f64(k), f64(v), f64(do), cq, cq, scale, causal=False)
+    assert_o_close(o.cpu().double().numpy(), ro)
+    assert_lse_close(lse.cpu().numpy(), rl)
+    assert_grad_close(dq.cpu().double().numpy(), rdq, "dQ")
+    assert_grad_close(dk.cpu().double().numpy(), rdk, "dK")
+    assert_grad_close(dv.cpu().double().numpy(), rdv, "dV")
+
+
+def test_dense_many_empty_units_per_cta():
+    """The dense layout's counterpart: key length 0 for all but one sequence, many units per persistent CTA."""
+    B, H, N, d = 40, 16, 512, 64
+    q, k, v, do = [inputs.gaussian((B, H, N, d), 70 + t, "bf16") for t in range(4)]
+    kl = np.array([0] * (B - 1) + [N], dtype=np.int32)
+    kld = torch.as_tensor(kl).cuda()
+    o, lse = fa.attention_fwd(q.cuda(), k.cuda(), v.cuda(), key_lens=kld)
+    assert fa.last_device_status() == 0
+    ro, rl = oracle.attn_fwd(f64(q[-1:]), f64(k[-1:]), f64(v[-1:]), 0.125)
+    assert_o_close(o[-1:].cpu().double().numpy(), ro)
+    assert torch.all(o[:-1] == 0) and torch.all(torch.isneginf(lse[:-1]))
