@@ -339,6 +339,41 @@ def measure_varlen(stream, flush, peak):
     return out
 
 
+def measure_decode(stream, flush, hbm_gbs):
+    """Split-K/V decode (inference with a full K/V cache): B8 H16, one new query per sequence against 16384 cached
+    keys, d128 bf16, causal (aligned with the end of the keys).  Bound by reading the cache: algorithmic bytes are
+    K and V (2*B*H*Nk*d*2) plus Q and O; reported as GB/s and as a fraction of the measured HBM copy bandwidth."""
+    import torch
+    from exact_io_aware_48_b200 import _lib, inputs
+    B, H, Nq, Nk, d = 8, 16, 1, 16384, 128
+    q = inputs.gaussian((B, H, Nq, d), 500, "bf16").cuda()
+    k = inputs.gaussian((B, H, Nk, d), 501, "bf16").cuda()
+    v = inputs.gaussian((B, H, Nk, d), 502, "bf16").cuda()
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, Nq), device="cuda", dtype=torch.float32)
+    ws_bytes = _lib.fa_fwd_splitkv_workspace_size(B, H, Nq, Nk, d, 0)
+    ws = torch.empty(ws_bytes, device="cuda", dtype=torch.uint8)
+    scale = 1.0 / math.sqrt(d)
+
+    def step(st):
+        rc = _lib.fa_fwd_splitkv(q, k, v, o, lse, B, H, Nq, Nk, d, scale, True, None, 0, ws, ws_bytes, _lib.FA_BF16,
+                                 st)
+        if rc:
+            raise RuntimeError(f"fa_fwd_splitkv: {_lib.fa_status_string(rc)}")
+
+    for _ in range(3):
+        step(stream)
+    ms, _ = time_loop(step, 20, stream, flush)
+    status = _lib.fa_last_device_status(stream)
+    if status:
+        raise RuntimeError(f"split-K/V forward reported {_lib.fa_status_string(status)}")
+    t = statistics.median(ms)
+    nbytes = 2 * B * H * Nk * d * 2 + 2 * B * H * Nq * d * 2
+    gbs = nbytes / t / 1e6
+    return {"workload": f"decode B{B} H{H} Nq{Nq} Nk{Nk} d{d} bf16 causal, split-K/V", "ms": round(t, 4),
+            "bytes": nbytes, "gbs": round(gbs, 1), "hbm_frac": round(gbs / hbm_gbs, 4) if hbm_gbs else None}
+
+
 def run_ours(args):
     import numpy as np
     import torch
@@ -402,6 +437,7 @@ def run_ours(args):
 
     targets = measure_targets(stream, flush, peak) if (args.targets and rank == 0) else None
     varlen = measure_varlen(stream, flush, peak) if (args.targets and rank == 0) else None
+    decode = measure_decode(stream, flush, hbm) if (args.targets and rank == 0) else None
     cpu = cpu_baseline(p.w) if rank == 0 and world == 1 and args.cpu_baseline else None
 
     if rank == 0:
@@ -423,6 +459,7 @@ def run_ours(args):
             "clocks": clk.summary(),
             "targets": targets,
             "varlen": varlen,
+            "decode": decode,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)

@@ -13,8 +13,8 @@ from . import _lib
 from ._lib import (FA_BF16, FA_FP16, FA_OK, FA_ERR_CUDA, FA_ERR_INVALID_ARG, FA_ERR_TIMEOUT, FA_ERR_UNSUPPORTED,
                    FA_ERR_WORKSPACE)
 
-__all__ = ["attention_fwd", "attention_bwd", "attention_fwd_varlen", "attention_bwd_varlen", "blockmask_lists",
-           "FAError", "FA_BF16", "FA_FP16"]
+__all__ = ["attention_fwd", "attention_bwd", "attention_fwd_varlen", "attention_bwd_varlen",
+           "attention_fwd_splitkv", "blockmask_lists", "FAError", "FA_BF16", "FA_FP16"]
 
 
 class FAError(RuntimeError):
@@ -137,4 +137,22 @@ def attention_bwd_varlen(q, k, v, o, dout, lse, cu_seqlens_q, cu_seqlens_k, max_
                               max_seqlen_k, total_q, total_k, d, scale, causal, ws, ws_bytes, _dtype_code(q), stream),
            "fa_bwd_varlen")
     return dq, dk, dv
+
+
+def attention_fwd_splitkv(q, k, v, causal=False, softmax_scale=None, key_lens=None, num_splits=0, stream=None):
+    """O, LSE for decoding: q [B, H, Nq, d] are the last Nq positions of sequences whose keys/values k, v are
+    [B, H, Nk, d] (key_lens: optional int32 [B], valid cache entries).  Causal aligns the queries with the end of
+    the keys.  The keys are split into num_splits ranges (0 = automatic) processed in parallel."""
+    import torch
+    _require_cuda(q, k, v, key_lens)
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    scale = softmax_scale if softmax_scale is not None else 1.0 / math.sqrt(d)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, Nq), device=q.device, dtype=torch.float32)
+    ws_bytes = _lib.fa_fwd_splitkv_workspace_size(B, H, Nq, Nk, d, num_splits)
+    ws = torch.empty(max(ws_bytes, 1), device=q.device, dtype=torch.uint8)
+    _check(_lib.fa_fwd_splitkv(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, key_lens, num_splits, ws, ws_bytes,
+                               _dtype_code(q), stream), "fa_fwd_splitkv")
+    return o, lse
 

@@ -37,6 +37,8 @@ SIGNATURES = {
     "fa_bwd_noalloc": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P, _P, _I, _P], _I),
     "fa_fwd_varlen": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P], _I),
     "fa_bwd_varlen_workspace_size": ([_I, _I, _I, _I], _SZ),
+    "fa_fwd_splitkv_workspace_size": ([_I, _I, _I, _I, _I, _I], _SZ),
+    "fa_fwd_splitkv": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P, _I, _P, _SZ, _I, _P], _I),
     "fa_bwd_varlen": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P, _SZ, _I,
                        _P], _I),
 }
@@ -180,3 +182,14 @@ def fa_bwd_varlen(q, k, v, o, dout, lse, dq, dk, dv, cu_q, cu_k, B, H, max_q, ma
     return load().fa_bwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
                                 _ptr(dv), _ptr(cu_q), _ptr(cu_k), B, H, max_q, max_k, total_q, total_k, d,
                                 softmax_scale, int(causal), _ptr(workspace), workspace_bytes, dtype, _stream(stream))
+
+
+def fa_fwd_splitkv_workspace_size(B, H, Nq, Nk, d, num_splits) -> int:
+    return load().fa_fwd_splitkv_workspace_size(B, H, Nq, Nk, d, num_splits)
+
+
+def fa_fwd_splitkv(q, k, v, o, lse, B, H, Nq, Nk, d, softmax_scale, causal, key_lens, num_splits, workspace,
+                   workspace_bytes, dtype, stream=None) -> int:
+    return load().fa_fwd_splitkv(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nq, Nk, d, softmax_scale,
+                                 int(causal), _ptr(key_lens), num_splits, _ptr(workspace), workspace_bytes, dtype,
+                                 _stream(stream))

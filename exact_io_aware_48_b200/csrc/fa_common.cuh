@@ -54,6 +54,18 @@ __device__ __forceinline__ int kv_tile_end(int i, int kv_lim, bool causal) {
   return end;
 }
 
+// The same when query row r sees keys c <= r + off (off = len_k - N_q aligns the queries with the end of the keys,
+// as when a few new queries attend to a cache; off = 0 is kv_tile_end).
+__device__ __forceinline__ int kv_tile_end_off(int i, int kv_lim, bool causal, int off) {
+  int end = (kv_lim + kTile - 1) / kTile;
+  if (causal) {
+    const int last = i * kTile + kTile - 1 + off;  // last key the tile's last row may see
+    const int e = last < 0 ? 0 : last / kTile + 1;
+    if (end > e) end = e;
+  }
+  return end;
+}
+
 // Iterates, in ascending order, the K/V tiles visible to either of the two Q tiles a forward CTA owns.  Every
 // role (loader, MMA issuer, softmax warps) walks the same sequence, so their pipelines stay in step.
 //   dense : tile t sees [0, end_t)
@@ -65,11 +77,11 @@ struct PairTileIter {
   bool sparse;
   int next_dense;
 
-  __device__ __forceinline__ void init_dense(int end0, int end1) {
+  __device__ __forceinline__ void init_dense(int end0, int end1, int begin = 0) {
     sparse = false;
     len[0] = end0; len[1] = end1;
     pos[0] = pos[1] = 0;
-    next_dense = 0;
+    next_dense = begin;  // tiles [begin, end_t)
     list[0] = list[1] = nullptr;
   }
 
@@ -109,6 +121,7 @@ struct PairTileIter {
     return true;
   }
 
+  // tiles tile t visits in a dense walk from 0 (sparse: its list length)
   __device__ __forceinline__ int count(int t) const { return len[t]; }
 };
 

@@ -60,6 +60,11 @@ struct FwdArgs {
   int total_q, total_k;  // packed: token counts; O is [total_q, H, d], LSE [H, total_q]
   int H, N, nT, npairs, BH;  // packed: N = the longest query sequence, Nk the longest key sequence
   int Nk;
+  // split-K/V decode: the N queries of (b, h) are the last N positions of its sequence, so query r sees key c iff
+  // c < len_k and (causal) c <= r + len_k - N; unit s of a Q tile covers K/V tiles [s*kv_split_tiles, ...+ that)
+  int nsplit, kv_split_tiles;
+  float* o_part;    // [nsplit][BH][128*nT][d] fp32: O of each split, normalised by its own l
+  float* lse_part;  // [nsplit][BH][128*nT] fp32: natural-log LSE of each split, -inf if it saw no key
   int causal;
   float scale_log2;  // softmax_scale * log2(e)
   uint64_t budget_ns;
@@ -69,24 +74,45 @@ struct FwdArgs {
 // tiles first under the causal mask); the kernel is persistent and walks them with UnitSeq.
 struct FwdUnit {
   int qt0, bh, h, kv_lim, end0, end1;
+  int split, begin, off;  // split-K/V: split index, first K/V tile, causal offset (0 otherwise)
   SeqGeom g;
   bool has1;
 };
 
-template <bool kPacked>
+constexpr int kModeDense = 0, kModePacked = 1, kModeSplit = 2;
+
+template <int kMode>
 __device__ __forceinline__ FwdUnit fwd_unit(int L, const FwdArgs& a, int tiles) {
   FwdUnit u;
+  u.split = 0;
+  if constexpr (kMode == kModeSplit) {  // units split-major: every split of every Q tile
+    const int per = a.npairs * a.BH;
+    u.split = L / per;
+    L -= u.split * per;
+  }
   const int pair = a.npairs - 1 - L / a.BH;
   u.bh = L % a.BH;
   u.h = u.bh % a.H;
   u.qt0 = tiles * pair;
-  u.g = seq_geom(kPacked ? a.cu_q : nullptr, a.cu_k, a.key_lens, u.bh / a.H, a.N, a.Nk, a.total_q, a.total_k);
+  u.g = seq_geom(kMode == kModePacked ? a.cu_q : nullptr, a.cu_k, a.key_lens, u.bh / a.H, a.N, a.Nk, a.total_q,
+                 a.total_k);
+  if constexpr (kMode == kModeSplit) u.g.lk = key_limit(a.key_lens, u.bh / a.H, a.Nk);
   const int nTq = (u.g.lq + kTile - 1) / kTile;  // Q tiles of this sequence
   u.has1 = tiles == 2 && u.qt0 + 1 < nTq;
   u.kv_lim = u.g.lk;
   const bool causal = a.causal != 0;
-  u.end0 = u.qt0 < nTq ? kv_tile_end(u.qt0, u.kv_lim, causal) : 0;  // a tile past the sequence sees nothing
-  u.end1 = u.has1 ? kv_tile_end(u.qt0 + 1, u.kv_lim, causal) : 0;
+  if constexpr (kMode == kModeSplit) {
+    u.off = causal ? u.kv_lim - a.N : 0;
+    u.begin = u.split * a.kv_split_tiles;
+    const int stop = u.begin + a.kv_split_tiles;
+    u.end0 = u.qt0 < nTq ? min(kv_tile_end_off(u.qt0, u.kv_lim, causal, u.off), stop) : 0;
+    u.end1 = u.has1 ? min(kv_tile_end_off(u.qt0 + 1, u.kv_lim, causal, u.off), stop) : 0;
+  } else {
+    u.off = 0;
+    u.begin = 0;
+    u.end0 = u.qt0 < nTq ? kv_tile_end(u.qt0, u.kv_lim, causal) : 0;  // a tile past the sequence sees nothing
+    u.end1 = u.has1 ? kv_tile_end(u.qt0 + 1, u.kv_lim, causal) : 0;
+  }
   return u;
 }
 
@@ -94,12 +120,13 @@ __device__ __forceinline__ void fwd_tiles(PairTileIter& it, const FwdUnit& u, co
   if (a.row_ptr != nullptr)
     it.init_sparse(a.row_ptr, a.col_idx, u.qt0, a.nT, u.end0, u.end1);
   else
-    it.init_dense(u.end0, u.end1);
+    it.init_dense(u.end0, u.end1, u.begin);
 }
 
-// kPacked: packed variable-length batch (FwdArgs::cu_q set); a separate instantiation so the dense kernels carry
-// none of its state.
-template <int D, bool kBF16, int kTiles, bool kPacked>
+// kMode: kModeDense, kModePacked (packed variable-length batch, FwdArgs::cu_q set) or kModeSplit (split-K/V
+// decode, partial results to o_part / lse_part); separate instantiations, so the dense kernels carry none of the
+// other modes' state.
+template <int D, bool kBF16, int kTiles, int kMode>
 __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
     fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                const __grid_constant__ CUtensorMap map_v, const FwdArgs args) {
@@ -118,8 +145,9 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const bool causal = args.causal != 0;
-  constexpr bool packed = kPacked;
-  const int total_units = args.npairs * args.BH;
+  constexpr bool packed = kMode == kModePacked;
+  constexpr bool split = kMode == kModeSplit;
+  const int total_units = args.npairs * args.BH * (split ? args.nsplit : 1);
 
   if (threadIdx.x == 0) {
     ptx::mbar_init(ptx::smem_addr(&bar_q), 1);
@@ -163,7 +191,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
       int n = 0, ku = 0, j, fl;
       bool ok = true;
       while (ok && us.next(L)) {
-        const FwdUnit u = fwd_unit<kPacked>(L, args, kTiles);
+        const FwdUnit u = fwd_unit<kMode>(L, args, kTiles);
         PairTileIter it;
         fwd_tiles(it, u, args);
         // the Q buffer is free once every S MMA of the previous unit has completed
@@ -250,7 +278,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
       };
 
       while (ok && us.next(L)) {
-        const FwdUnit u = fwd_unit<kPacked>(L, args, kTiles);
+        const FwdUnit u = fwd_unit<kMode>(L, args, kTiles);
         PairTileIter it;
         fwd_tiles(it, u, args);
         if (!(ok = wait_or_abort(ptx::smem_addr(&bar_q), ku & 1, args.budget_ns, abortp))) break;
@@ -323,12 +351,16 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
     int ku = 0;
     bool ok = true;
     while (ok && us.next(L)) {
-      FwdUnit u = fwd_unit<kPacked>(L, args, kTiles);
+      FwdUnit u = fwd_unit<kMode>(L, args, kTiles);
       PairTileIter it;
       fwd_tiles(it, u, args);
+      const int u_bh = u.bh;
+      const bool u_has1 = u.has1;
       const int qt = u.qt0 + t;
       const int grow = qt * kTile + row;  // row within the sequence
       const int kv_lim = u.kv_lim;
+      int coff = 0;  // split-K/V causal: keys c <= grow + coff
+      if constexpr (split) coff = u.off;
       float m_ref = -INFINITY;
       ptx::f32x2 lacc[2] = {{0.f, 0.f}, {0.f, 0.f}};  // running denominator l, as four partial sums
       int kidx = 0;
@@ -348,12 +380,22 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
         ptx::tmem_ld_wait();
         float* s = reinterpret_cast<float*>(sr);
         // element masks only on tiles that straddle the diagonal or the key limit
-        if ((causal && j >= qt) || (j + 1) * kTile > kv_lim) {
-          const int c0 = j * kTile;
-          const int lim = causal ? min(kv_lim, grow + 1) : kv_lim;  // keys c < lim are visible
+        if constexpr (split) {
+          if ((causal && (j + 1) * kTile - 1 > qt * kTile + coff) || (j + 1) * kTile > kv_lim) {
+            const int c0 = j * kTile;
+            const int lim = causal ? min(kv_lim, grow + 1 + coff) : kv_lim;  // keys c < lim are visible
 #pragma unroll
-          for (int i = 0; i < 128; ++i)
-            if (c0 + i >= lim) s[i] = -INFINITY;
+            for (int i = 0; i < 128; ++i)
+              if (c0 + i >= lim) s[i] = -INFINITY;
+          }
+        } else {
+          if ((causal && j >= qt) || (j + 1) * kTile > kv_lim) {
+            const int c0 = j * kTile;
+            const int lim = causal ? min(kv_lim, grow + 1) : kv_lim;  // keys c < lim are visible
+#pragma unroll
+            for (int i = 0; i < 128; ++i)
+              if (c0 + i >= lim) s[i] = -INFINITY;
+          }
         }
         // row max: 8 independent partial maxima with 3-input max (two new elements per instruction), then a tree
         float pm[8];
@@ -418,11 +460,20 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
       ptx::tc_fence_after();
       // packed: the unit is worked out again rather than kept in registers through the K/V loop (the softmax
       // warps are at their register limit and the packed unit carries more state)
-      if constexpr (kPacked) u = fwd_unit<kPacked>(L, args, kTiles);
+      if constexpr (packed || split) {
+        u = fwd_unit<kMode>(L, args, kTiles);
+      } else {
+        u.bh = u_bh;  // dense: only these two are needed below
+        u.has1 = u_has1;
+        u.g.lq = args.N;
+      }
       const bool row_ok = grow < u.g.lq && (t == 0 || u.has1);
       const float l_sum = (lacc[0].x + lacc[0].y) + (lacc[1].x + lacc[1].y);
       const bool nonempty = l_sum > 0.f;
       const float inv = nonempty ? 1.0f / l_sum : 0.0f;
+      // split-K/V: this split's normalised O (fp32) and LSE go to the partial buffers for the combine kernel
+      size_t prow = 0;
+      if constexpr (split) prow = ((size_t)u.split * args.BH + u.bh) * (size_t)(args.nT * kTile) + grow;
       const size_t orow_idx = packed ? (size_t)(u.g.q0 + grow) * args.H + u.h : (size_t)u.bh * args.N + grow;
       uint8_t* orow = reinterpret_cast<uint8_t*>(args.o) + orow_idx * D * 2;
 #pragma unroll 1
@@ -434,22 +485,40 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
           ptx::tc_fence_before();
           ptx::mbar_arrive(ptx::smem_addr(&bar_o_free[t]));
         }
-        uint32_t pk[16];
+        if constexpr (split) {
+          if (row_ok) {
+            float4* dst = reinterpret_cast<float4*>(args.o_part + prow * D + c * 32);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float a = nonempty ? __uint_as_float(orr[2 * i]) * inv : 0.0f;
-          const float bb = nonempty ? __uint_as_float(orr[2 * i + 1]) * inv : 0.0f;
-          pk[i] = ptx::pack2<kBF16>(a, bb);
-        }
-        if (row_ok) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 64);
+            for (int v = 0; v < 8; ++v) {
+              const float4 x = make_float4(__uint_as_float(orr[4 * v]), __uint_as_float(orr[4 * v + 1]),
+                                           __uint_as_float(orr[4 * v + 2]), __uint_as_float(orr[4 * v + 3]));
+              dst[v] = nonempty ? make_float4(x.x * inv, x.y * inv, x.z * inv, x.w * inv)
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+          }
+        } else {
+          uint32_t pk[16];
 #pragma unroll
-          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          for (int i = 0; i < 16; ++i) {
+            const float a = nonempty ? __uint_as_float(orr[2 * i]) * inv : 0.0f;
+            const float bb = nonempty ? __uint_as_float(orr[2 * i + 1]) * inv : 0.0f;
+            pk[i] = ptx::pack2<kBF16>(a, bb);
+          }
+          if (row_ok) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 64);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          }
         }
       }
       if (row_ok) {
-        const size_t li = packed ? (size_t)u.h * args.total_q + u.g.q0 + grow : (size_t)u.bh * args.N + grow;
-        args.lse[li] = nonempty ? (m_ref + __log2f(l_sum)) * 0.69314718055994530942f : -INFINITY;
+        const float lse_v = nonempty ? (m_ref + __log2f(l_sum)) * 0.69314718055994530942f : -INFINITY;
+        if constexpr (split) {
+          args.lse_part[prow] = lse_v;
+        } else {
+          const size_t li = packed ? (size_t)u.h * args.total_q + u.g.q0 + grow : (size_t)u.bh * args.N + grow;
+          args.lse[li] = lse_v;
+        }
       }
       ++ku;
     }
@@ -460,6 +529,61 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
   if (warp == C::kWarpMma) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------------------------------------ split combine
+// Merges the splits of a split-K/V forward (the online-softmax merge of the explainer page applied to whole
+// partial results): with m = max_s LSE_s and w_s = exp(LSE_s - m),  O = sum_s w_s O_s / sum_s w_s,
+// LSE = m + log sum_s w_s; all splits empty -> O = 0, LSE = -inf.  One warp per (b, h, query row); lane s holds
+// split s's LSE (nsplit <= 32), each lane D/32 output columns.  Memory-bound and small.
+template <int D, bool kBF16>
+__global__ void __launch_bounds__(256) splitkv_combine_kernel(const float* __restrict__ o_part,
+                                                              const float* __restrict__ lse_part,
+                                                              void* __restrict__ o, float* __restrict__ lse,
+                                                              int nsplit, int BH, int N, int Npad) {
+  const int lane = threadIdx.x % 32;
+  const long long rows = (long long)BH * N;
+  const long long nwarps = ((long long)gridDim.x * blockDim.x) / 32;
+  for (long long r = ((long long)blockIdx.x * blockDim.x + threadIdx.x) / 32; r < rows; r += nwarps) {
+    const long long bh = r / N;
+    const int q = (int)(r % N);
+    const size_t prow0 = (size_t)bh * Npad + q;  // row of split 0
+    const size_t split_stride = (size_t)BH * Npad;
+    const float ls = lane < nsplit ? lse_part[lane * split_stride + prow0] : -INFINITY;
+    float m = ls;
+#pragma unroll
+    for (int k = 16; k > 0; k >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, k));
+    const float w = (m == -INFINITY || ls == -INFINITY) ? 0.f : __expf(ls - m);
+    float wsum = w;
+#pragma unroll
+    for (int k = 16; k > 0; k >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, k);
+    constexpr int kCols = D / 32;  // columns per lane: lane * kCols .. + kCols - 1
+    float acc[kCols];
+#pragma unroll
+    for (int c = 0; c < kCols; ++c) acc[c] = 0.f;
+    for (int s = 0; s < nsplit; ++s) {
+      const float ws = __shfl_sync(0xffffffffu, w, s);
+      if (ws == 0.f) continue;
+      const float* src = o_part + (s * split_stride + prow0) * D + lane * kCols;
+#pragma unroll
+      for (int c = 0; c < kCols; c += 2) {
+        const float2 x = *reinterpret_cast<const float2*>(src + c);
+        acc[c] = fmaf(ws, x.x, acc[c]);
+        acc[c + 1] = fmaf(ws, x.y, acc[c + 1]);
+      }
+    }
+    const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+    uint32_t pk[kCols / 2];
+#pragma unroll
+    for (int c = 0; c < kCols; c += 2) pk[c / 2] = ptx::pack2<kBF16>(acc[c] * inv, acc[c + 1] * inv);
+    uint16_t* dst = reinterpret_cast<uint16_t*>(o) + ((size_t)bh * N + q) * D + lane * kCols;
+    if constexpr (kCols == 4) {
+      *reinterpret_cast<uint2*>(dst) = make_uint2(pk[0], pk[1]);
+    } else {
+      *reinterpret_cast<uint32_t*>(dst) = pk[0];
+    }
+    if (lane == 0) lse[(size_t)bh * N + q] = wsum > 0.f ? m + __logf(wsum) : -INFINITY;
   }
 }
 

@@ -15,7 +15,7 @@
 
 namespace {
 
-constexpr int kVersion = 10100;  // 1.1.0: packed variable-length batches
+constexpr int kVersion = 10200;  // 1.2.0: split-K/V decode forward
 constexpr int kMaxN = 1 << 20;
 constexpr long long kMaxElems = 1LL << 34;
 
@@ -146,7 +146,7 @@ cudaError_t ensure_smem(Kernel kernel, int bytes, std::atomic<uint64_t>& done_ma
   return e;
 }
 
-template <int D, bool BF, int T, bool P>
+template <int D, bool BF, int T, int P>
 cudaError_t launch_fwd_k(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, fa::FwdArgs a,
                          cudaStream_t st) {
   using C = fa::FwdCfg<D, T>;
@@ -158,7 +158,7 @@ cudaError_t launch_fwd_k(const CUtensorMap& mq, const CUtensorMap& mk, const CUt
   int dev = 0, sms = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = fa::device_sm_count(dev, &sms)) != cudaSuccess) return e;
-  const long long units = (long long)a.BH * a.npairs;
+  const long long units = (long long)a.BH * a.npairs * (P == fa::kModeSplit ? a.nsplit : 1);
   const unsigned grid = (unsigned)std::min<long long>(units, (long long)sms * (3 - T));
   if ((e = mark(FA_KERNEL_FWD, 0, st)) != cudaSuccess) return e;
   fa::fwd_kernel<D, BF, T, P><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mk, mv, a);
@@ -169,7 +169,8 @@ cudaError_t launch_fwd_k(const CUtensorMap& mq, const CUtensorMap& mk, const CUt
 template <int D, bool BF, int T>
 cudaError_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const fa::FwdArgs& a,
                        cudaStream_t st) {
-  return a.cu_q ? launch_fwd_k<D, BF, T, true>(mq, mk, mv, a, st) : launch_fwd_k<D, BF, T, false>(mq, mk, mv, a, st);
+  return a.cu_q ? launch_fwd_k<D, BF, T, fa::kModePacked>(mq, mk, mv, a, st)
+                : launch_fwd_k<D, BF, T, fa::kModeDense>(mq, mk, mv, a, st);
 }
 
 // Q tiles per forward CTA for this call (see FwdCfg).  Measured on B200 (bf16, causal): d = 64 prefers one-tile
@@ -213,6 +214,10 @@ int run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, in
   a.total_q = pk.total_q;
   a.total_k = pk.total_k;
   a.Nk = pk.cu_q ? pk.Nk : N;
+  a.nsplit = 1;
+  a.kv_split_tiles = 0;
+  a.o_part = nullptr;
+  a.lse_part = nullptr;
   a.H = H;
   a.N = N;
   a.nT = (N + fa::kTile - 1) / fa::kTile;
@@ -268,6 +273,58 @@ int launch_lists(const uint8_t* mask, int nT, const Lists& l, cudaStream_t st) {
 }
 
 }  // namespace
+
+// ------------------------------------------------------------------------------------------ split-K/V decode
+constexpr int kMaxSplits = 32;
+
+// Splits for a split-K/V forward: enough units to fill the SMs twice (two one-tile CTAs fit on an SM), at most
+// one K/V tile per split and kMaxSplits.
+int splitkv_splits(int B, int H, int Nq, int Nk, int requested) {
+  const int tiles_k = (Nk + fa::kTile - 1) / fa::kTile;
+  if (requested > 0) return std::min(std::min(requested, kMaxSplits), tiles_k);
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess || fa::device_sm_count(dev, &sms) != cudaSuccess) sms = 148;
+  const long long base = (long long)B * H * ((Nq + fa::kTile - 1) / fa::kTile);
+  long long s = (2LL * sms + base - 1) / base;
+  if (s > kMaxSplits) s = kMaxSplits;
+  if (s > tiles_k) s = tiles_k;
+  return (int)std::max(1LL, s);
+}
+
+size_t splitkv_bytes(int B, int H, int Nq, int d, int nsplit) {
+  const size_t rows = (size_t)nsplit * B * H * ((Nq + fa::kTile - 1) / fa::kTile) * fa::kTile;
+  return align_up(rows * d * 4, 256) + align_up(rows * 4, 256);
+}
+
+template <int D, bool BF>
+cudaError_t launch_splitkv(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, fa::FwdArgs a,
+                           void* o, float* lse, cudaStream_t st) {
+  cudaError_t e = launch_fwd_k<D, BF, 1, fa::kModeSplit>(mq, mk, mv, a, st);
+  if (e != cudaSuccess) return e;
+  const long long rows = (long long)a.BH * a.N;
+  const unsigned blocks = (unsigned)std::min<long long>((rows + 7) / 8, 148LL * 16);
+  fa::splitkv_combine_kernel<D, BF><<<blocks, 256, 0, st>>>(a.o_part, a.lse_part, o, lse, a.nsplit, a.BH, a.N,
+                                                            a.nT * fa::kTile);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------------------------------ packed batches
+int check_packed(const void* q, const void* k, const void* v, const int32_t* cu_q, const int32_t* cu_k, int B, int H,
+                 int max_q, int max_k, int total_q, int total_k, int d, float scale, int dtype) {
+  if (!q || !k || !v || !cu_q || !cu_k) return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(cu_q, 4) || !aligned(cu_k, 4))
+    return FA_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || max_q < 1 || max_k < 1 || max_q > kMaxN || max_k > kMaxN) return FA_ERR_INVALID_ARG;
+  if (total_q < 1 || total_k < 1) return FA_ERR_INVALID_ARG;
+  if (dtype != FA_BF16 && dtype != FA_FP16) return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.0f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  const long long npad = (long long)(max_q + fa::kTile - 1) / fa::kTile * fa::kTile;
+  if ((long long)total_q * H * d > kMaxElems || (long long)total_k * H * d > kMaxElems ||
+      (long long)B * H * npad * d > kMaxElems)
+    return FA_ERR_INVALID_ARG;
+  return FA_OK;
+}
 
 extern "C" {
 
@@ -366,24 +423,6 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
   return e == cudaSuccess ? FA_OK : cuda_fail(e);
 }
 
-// ------------------------------------------------------------------------------------------ packed batches
-int check_packed(const void* q, const void* k, const void* v, const int32_t* cu_q, const int32_t* cu_k, int B, int H,
-                 int max_q, int max_k, int total_q, int total_k, int d, float scale, int dtype) {
-  if (!q || !k || !v || !cu_q || !cu_k) return FA_ERR_INVALID_ARG;
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(cu_q, 4) || !aligned(cu_k, 4))
-    return FA_ERR_INVALID_ARG;
-  if (B < 1 || H < 1 || max_q < 1 || max_k < 1 || max_q > kMaxN || max_k > kMaxN) return FA_ERR_INVALID_ARG;
-  if (total_q < 1 || total_k < 1) return FA_ERR_INVALID_ARG;
-  if (dtype != FA_BF16 && dtype != FA_FP16) return FA_ERR_INVALID_ARG;
-  if (!(scale > 0.0f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
-  const long long npad = (long long)(max_q + fa::kTile - 1) / fa::kTile * fa::kTile;
-  if ((long long)total_q * H * d > kMaxElems || (long long)total_k * H * d > kMaxElems ||
-      (long long)B * H * npad * d > kMaxElems)
-    return FA_ERR_INVALID_ARG;
-  return FA_OK;
-}
-
 int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int32_t* cu_seqlens_q,
                   const int32_t* cu_seqlens_k, int B, int H, int max_seqlen_q, int max_seqlen_k, int total_q,
                   int total_k, int d, float softmax_scale, int causal, int dtype, void* stream) {
@@ -431,6 +470,64 @@ int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, co
                               static_cast<cudaStream_t>(stream), t_events[FA_KERNEL_BWD_MAIN][0],
                               t_events[FA_KERNEL_BWD_MAIN][1], cu_seqlens_q, cu_seqlens_k, total_q, total_k,
                               max_seqlen_k);
+  return e == cudaSuccess ? FA_OK : cuda_fail(e);
+}
+
+size_t fa_fwd_splitkv_workspace_size(int B, int H, int Nq, int Nk, int d, int num_splits) {
+  if (B < 1 || H < 1 || Nq < 1 || Nk < 1 || Nq > kMaxN || Nk > kMaxN || (d != 64 && d != 128)) return 0;
+  if (num_splits < 0 || num_splits > kMaxSplits) return 0;
+  return splitkv_bytes(B, H, Nq, d, splitkv_splits(B, H, Nq, Nk, num_splits));
+}
+
+int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq, int Nk,
+                   int d, float softmax_scale, int causal, const int32_t* key_lens, int num_splits, void* workspace,
+                   size_t workspace_bytes, int dtype, void* stream) {
+  int rc = check_common(q, k, v, B, H, Nk, d, softmax_scale, dtype);
+  if (rc != FA_OK) return rc;
+  if (Nq < 1 || Nq > kMaxN || (long long)B * H * Nq * d > kMaxElems) return FA_ERR_INVALID_ARG;
+  if (num_splits < 0 || num_splits > kMaxSplits) return FA_ERR_INVALID_ARG;
+  if (!o || !lse || !aligned(o, 16) || !aligned(lse, 4) || (key_lens && !aligned(key_lens, 4)))
+    return FA_ERR_INVALID_ARG;
+  const int nsplit = splitkv_splits(B, H, Nq, Nk, num_splits);
+  const size_t need = splitkv_bytes(B, H, Nq, d, nsplit);
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < need) return FA_ERR_WORKSPACE;
+  CUtensorMap mq, mk, mv;
+  if ((rc = make_map(&mq, q, B * H, Nq, d, dtype)) != FA_OK) return rc;
+  if ((rc = make_map(&mk, k, B * H, Nk, d, dtype)) != FA_OK) return rc;
+  if ((rc = make_map(&mv, v, B * H, Nk, d, dtype)) != FA_OK) return rc;
+  fa::FwdArgs a;
+  a.o = o;
+  a.lse = lse;
+  a.key_lens = key_lens;
+  a.row_ptr = nullptr;
+  a.col_idx = nullptr;
+  a.cu_q = nullptr;
+  a.cu_k = nullptr;
+  a.total_q = 0;
+  a.total_k = 0;
+  a.H = H;
+  a.N = Nq;
+  a.Nk = Nk;
+  a.nT = (Nq + fa::kTile - 1) / fa::kTile;
+  a.npairs = a.nT;  // one Q tile per CTA
+  a.BH = B * H;
+  a.causal = causal ? 1 : 0;
+  a.scale_log2 = softmax_scale * 1.4426950408889634f;
+  a.budget_ns = g_budget_ns.load();
+  const int tiles_k = (Nk + fa::kTile - 1) / fa::kTile;
+  a.nsplit = nsplit;
+  a.kv_split_tiles = (tiles_k + nsplit - 1) / nsplit;
+  const size_t rows = (size_t)nsplit * a.BH * a.nT * fa::kTile;
+  a.o_part = static_cast<float*>(workspace);
+  a.lse_part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + align_up(rows * d * 4, 256));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool bf = dtype == FA_BF16;
+  cudaError_t e;
+  if (d == 64)
+    e = bf ? launch_splitkv<64, true>(mq, mk, mv, a, o, lse, st) : launch_splitkv<64, false>(mq, mk, mv, a, o, lse, st);
+  else
+    e = bf ? launch_splitkv<128, true>(mq, mk, mv, a, o, lse, st)
+           : launch_splitkv<128, false>(mq, mk, mv, a, o, lse, st);
   return e == cudaSuccess ? FA_OK : cuda_fail(e);
 }
 

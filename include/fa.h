@@ -128,6 +128,28 @@ int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* l
                   const int32_t* cu_seqlens_k, int B, int H, int max_seqlen_q, int max_seqlen_k, int total_q,
                   int total_k, int d, float softmax_scale, int causal, int dtype, void* stream);
 
+/*
+ * Split-K/V forward for decoding: a few new queries per (b, h) against a long key/value cache.  The pages give no
+ * interface for this (they note the kernel's central role in inference and keeping K/V resident, review page,
+ * "Impact"); it reuses the tiled forward with the keys cut into ranges processed in parallel, each range's
+ * normalised O and LSE kept in fp32, and a merge of the ranges by their LSE (the online-softmax rescaling of the
+ * explainer page applied to whole partial results).
+ *   Layout      q, o: [B, H, Nq, d]; k, v: [B, H, Nk, d] (16-bit, d innermost); lse: [B, H, Nq] fp32 natural log.
+ *               key_lens: optional [B] int32, the number of valid cache entries of sequence b (<= Nk).
+ *   Visibility  The Nq queries are the last Nq positions of their sequence: with len = key_lens[b] (or Nk), key c
+ *               is visible from query r iff c < len && (causal == 0 || c <= r + len - Nq).  (This differs from
+ *               fa_fwd's causal, which aligns query and key 0.)  A query with no visible key gets O = 0, LSE = -inf.
+ *   Splits      num_splits in [0, 32]; 0 picks enough ranges to fill the GPU.  The result does not depend on the
+ *               number of splits beyond fp32 rounding.
+ *   Workspace   fa_fwd_splitkv_workspace_size(B, H, Nq, Nk, d, num_splits) bytes (256-byte aligned device memory).
+ *   Shapes      1 <= Nq, Nk <= 2^20, B*H*Nq*d and B*H*Nk*d <= 2^34, d in {64, 128}.  Everything else as fa_fwd.
+ */
+size_t fa_fwd_splitkv_workspace_size(int B, int H, int Nq, int Nk, int d, int num_splits);
+
+int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq, int Nk,
+                   int d, float softmax_scale, int causal, const int32_t* key_lens, int num_splits, void* workspace,
+                   size_t workspace_bytes, int dtype, void* stream);
+
 /* Bytes of workspace fa_bwd_varlen needs (fp32 dQ accumulator and per-row LSE/D over B*H padded sequences). */
 size_t fa_bwd_varlen_workspace_size(int B, int H, int max_seqlen_q, int d);
 

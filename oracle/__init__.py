@@ -239,6 +239,36 @@ def attn_bwd_varlen(q, k, v, do, cu_q, cu_k, scale, causal=False):
     return dq, dk, dv, o, lse
 
 
+def attn_fwd_decode(q, k, v, scale, causal=False, key_lens=None):
+    """Attention of Nq new queries per (b, h) against Nk cached keys/values (q [B,H,Nq,d], k, v [B,H,Nk,d]): the
+    queries are the last Nq positions of their sequence, so with len = key_lens[b] (else Nk) key c is visible from
+    query r iff c < len and (causal) c <= r + len - Nq.  Softmax of scale * q k^T over the visible keys, written
+    out directly in numpy (fp64).  Returns (O [B,H,Nq,d], LSE [B,H,Nq]); a row with no visible key has O = 0 and
+    LSE = -inf."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    o = np.zeros((B, H, Nq, d))
+    lse = np.full((B, H, Nq), -np.inf)
+    r = np.arange(Nq)[:, None]
+    c = np.arange(Nk)[None, :]
+    for b in range(B):
+        n = Nk if key_lens is None else int(min(max(int(key_lens[b]), 0), Nk))
+        vis = c < n
+        if causal:
+            vis = vis & (c <= r + n - Nq)
+        for h in range(H):
+            s = scale * (q[b, h] @ k[b, h].T)
+            s = np.where(vis, s, -np.inf)
+            m = s.max(axis=1, keepdims=True)
+            ok = np.isfinite(m[:, 0])
+            e = np.where(vis, np.exp(s - np.where(np.isfinite(m), m, 0.0)), 0.0)
+            l = e.sum(axis=1)
+            o[b, h, ok] = (e[ok] @ v[b, h]) / l[ok, None]
+            lse[b, h, ok] = m[ok, 0] + np.log(l[ok])
+    return o, lse
+
+
 def blockmask_csr(mask):
     """CSR of a square 0/1 tile mask: (row_ptr [nT+1] int32, col_idx [nnz] int32), ascending columns."""
     m = np.ascontiguousarray(mask, dtype=np.uint8)

@@ -411,3 +411,44 @@ def test_varlen_gradient_invariants_per_sequence():
         np.testing.assert_allclose(dk[ks].sum(axis=0), 0.0, atol=1e-11)
         nonempty = np.isfinite(lse[:, qs]).T[..., None]
         np.testing.assert_allclose(dv[ks].sum(axis=0), (do[qs] * nonempty).sum(axis=0), atol=1e-11)
+
+
+# ----------------------------------------------------------------------------------------------- decode
+# The decode oracle (numpy statement, queries aligned with the end of the keys) is pinned against the C oracle:
+# with as many queries as keys it is the ordinary attention; with fewer, its rows are the last rows of an ordinary
+# causal attention over the full sequence; key lengths truncate the cache; queries with no visible key are empty.
+@pytest.mark.parametrize("causal", [False, True])
+def test_decode_full_length_is_ordinary_attention(causal):
+    q, k, v = qkv(2, 2, 23, 8, 210)
+    o, lse = oracle.attn_fwd(q, k, v, 0.3, causal=causal)
+    od, ld = oracle.attn_fwd_decode(q, k, v, 0.3, causal=causal)
+    np.testing.assert_allclose(od, o, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(ld, lse, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("nq", [1, 4, 19])
+def test_decode_rows_are_last_rows_of_causal_attention(nq):
+    B, H, N, d = 2, 2, 37, 8
+    qf, k, v = qkv(B, H, N, d, 220)
+    o, lse = oracle.attn_fwd(qf, k, v, 0.4, causal=True)
+    od, ld = oracle.attn_fwd_decode(qf[:, :, N - nq:], k, v, 0.4, causal=True)
+    np.testing.assert_allclose(od, o[:, :, N - nq:], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(ld, lse[:, :, N - nq:], rtol=0, atol=1e-12)
+    if nq == 1:  # the last query sees every key either way
+        on, ln = oracle.attn_fwd_decode(qf[:, :, N - 1:], k, v, 0.4, causal=False)
+        np.testing.assert_allclose(on, od, rtol=0, atol=1e-14)
+
+
+def test_decode_key_lengths_truncate_the_cache_and_empty_queries():
+    B, H, Nq, Nk, d = 2, 1, 5, 30, 4
+    q, k, v = rnd((B, H, Nq, d), 230), rnd((B, H, Nk, d), 231), rnd((B, H, Nk, d), 232)
+    kl = np.array([17, 3], np.int32)
+    o, lse = oracle.attn_fwd_decode(q, k, v, 0.5, causal=True, key_lens=kl)
+    for b in range(B):
+        n = int(kl[b])
+        ob, lb = oracle.attn_fwd_decode(q[b:b + 1], k[b:b + 1, :, :n], v[b:b + 1, :, :n], 0.5, causal=True)
+        np.testing.assert_allclose(o[b:b + 1], ob, rtol=0, atol=1e-14)
+        np.testing.assert_allclose(lse[b:b + 1], lb, rtol=0, atol=1e-14)
+    # sequence 1 has 3 keys for 5 queries: queries 0 and 1 see nothing (c <= r + 3 - 5 < 0), query 2 sees key 0
+    assert np.all(o[1, :, :2] == 0) and np.all(np.isneginf(lse[1, :, :2]))
+    np.testing.assert_allclose(o[1, :, 2], v[1, :, 0], rtol=0, atol=1e-15)
