@@ -86,6 +86,7 @@ struct BwdArgs {
   int total_q, total_k;  // packed: token counts; dK, dV are [total_k, H, d]
   int H, N, nT, BH;  // nT = Q tiles of the padded row space (packed: of the longest query sequence)
   int Nk, nTk;       // key rows and K/V tiles per head (packed: of the longest key sequence)
+  int dl;            // head dim of the tensors (32 / 96 run on the 64 / 128 kernels; dq_acc rows are dl wide)
   int causal;
   float scale;       // softmax scale
   float scale_log2;  // softmax scale * log2(e)
@@ -142,7 +143,7 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const void* __restrict__ o
                                                       const float* __restrict__ lse, float* __restrict__ dq_acc,
                                                       float* __restrict__ lse2, float* __restrict__ Dv, int N,
                                                       int Npad, long long rows, float scale,
-                                                      const int32_t* __restrict__ cu_q, int total_q, int H) {
+                                                      const int32_t* __restrict__ cu_q, int total_q, int H, int dl) {
   constexpr int kLanesPerRow = D / 8;          // 8 or 16
   constexpr int kRowsPerWarp = 32 / kLanesPerRow;  // 4 or 2
   const int lane = threadIdx.x % 32;
@@ -158,8 +159,9 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const void* __restrict__ o
     const bool valid = r < g.lq;
     const size_t prow = cu_q ? (size_t)(g.q0 + r) * H + (size_t)(bh % H) : (size_t)bh * N + r;  // row of O, dO
     float dsum = 0.f;
-    if (in && valid) {
-      const size_t off = prow * D + (size_t)l * 8;
+    const bool col_ok = l * 8 < dl;  // lanes past the head dim (32 / 96 on the 64 / 128 kernels) hold nothing
+    if (in && valid && col_ok) {
+      const size_t off = prow * dl + (size_t)l * 8;
       const uint4 a = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(o) + off);
       const uint4 c = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(dout) + off);
       const uint32_t va[4] = {a.x, a.y, a.z, a.w}, vc[4] = {c.x, c.y, c.z, c.w};
@@ -173,9 +175,11 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const void* __restrict__ o
 #pragma unroll
     for (int m = kLanesPerRow / 2; m > 0; m >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, m);
     if (in) {
-      float4* acc = reinterpret_cast<float4*>(dq_acc + row * D);
-      acc[2 * l] = make_float4(0.f, 0.f, 0.f, 0.f);
-      acc[2 * l + 1] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (col_ok) {
+        float4* acc = reinterpret_cast<float4*>(dq_acc + row * dl);
+        acc[2 * l] = make_float4(0.f, 0.f, 0.f, 0.f);
+        acc[2 * l + 1] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
       if (l == 0) {
         float nl2 = -INFINITY;  // padded row or no visible key: recomputed P = exp2(x - inf) = 0
         if (valid) {
@@ -195,21 +199,21 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const void* __restrict__ o
 template <int D, bool kBF16>
 __global__ void __launch_bounds__(256) bwd_dq_kernel(const float* __restrict__ dq_acc, void* __restrict__ dq, int N,
                                                      int Npad, long long total_vec8, const int32_t* __restrict__ cu_q,
-                                                     int total_q, int H) {
+                                                     int total_q, int H, int dl) {
   for (long long v = (long long)blockIdx.x * blockDim.x + threadIdx.x; v < total_vec8;
        v += (long long)gridDim.x * blockDim.x) {
     const long long e = v * 8;
-    const long long row = e / D;  // dense: bh * N + r; packed: bh * Npad + r
-    const int c = (int)(e % D);
+    const long long row = e / dl;  // dense: bh * N + r; packed: bh * Npad + r
+    const int c = (int)(e % dl);
     const long long bh = row / (cu_q ? Npad : N);
     const int r = (int)(row % (cu_q ? Npad : N));
     size_t out_e = (size_t)e;
     if (cu_q) {
       const SeqGeom g = seq_geom(cu_q, cu_q, nullptr, (int)(bh / H), N, N, total_q, total_q);
       if (r >= g.lq) continue;
-      out_e = ((size_t)(g.q0 + r) * H + (size_t)(bh % H)) * D + c;
+      out_e = ((size_t)(g.q0 + r) * H + (size_t)(bh % H)) * dl + c;
     }
-    const float4* src = reinterpret_cast<const float4*>(dq_acc + ((size_t)bh * Npad + r) * D + c);
+    const float4* src = reinterpret_cast<const float4*>(dq_acc + ((size_t)bh * Npad + r) * dl + c);
     const float4 a = src[0], b = src[1];
     uint4 out;
     out.x = ptx::pack2<kBF16>(a.x, a.y);
@@ -678,11 +682,12 @@ __global__ void __launch_bounds__(512, 1)
         ptx::tmem_ld32(tmem + lane_base + C::kColDQ, ra);
         ptx::tmem_ld32(tmem + lane_base + C::kColDQ + 32, rb);
         ptx::tmem_ld_wait();
+        // boxes past the head dim (32 / 96 on the 64 / 128 kernels) hold only zeros and are not reduced
         if constexpr (D == 64) {
           ptx::tc_fence_before();
           ptx::mbar_arrive(ptx::smem_addr(&bar_dq_free));  // TMEM columns may now be overwritten
           reduce_box(ra, 0);
-          reduce_box(rb, 32);
+          if (32 < args.dl) reduce_box(rb, 32);
         } else {
           // d = 128: the columns are the next dP^T's, so all four chunks leave TMEM before any wait on the
           // staging buffer (registers hold up to three chunks)
@@ -695,7 +700,7 @@ __global__ void __launch_bounds__(512, 1)
           ptx::mbar_arrive(ptx::smem_addr(&bar_dq_free));
           reduce_box(rb, 32);
           reduce_box(rc, 64);
-          reduce_box(rd, 96);
+          if (96 < args.dl) reduce_box(rd, 96);
         }
         ++gi;
       }
@@ -705,8 +710,8 @@ __global__ void __launch_bounds__(512, 1)
       // dense: every row of the head (keys past a key length get zero); packed: the sequence's own keys only
       const bool row_ok = packed ? gc < u.g.lk : gc < args.N;
       const size_t krow = packed ? (size_t)(u.g.k0 + gc) * args.H + u.h : (size_t)u.bh * args.N + gc;
-      uint8_t* dv_row = reinterpret_cast<uint8_t*>(args.dv) + krow * D * 2;
-      uint8_t* dk_row = reinterpret_cast<uint8_t*>(args.dk) + krow * D * 2;
+      uint8_t* dv_row = reinterpret_cast<uint8_t*>(args.dv) + krow * args.dl * 2;
+      uint8_t* dk_row = reinterpret_cast<uint8_t*>(args.dk) + krow * args.dl * 2;
       if (n_iters > 0) {
         ok = __all_sync(0xffffffffu, wait_or_abort(ptx::smem_addr(&bar_done), ku & 1, args.budget_ns, abortp));
         if (!ok) break;
@@ -731,7 +736,7 @@ __global__ void __launch_bounds__(512, 1)
         uint32_t pkd[16];
 #pragma unroll
         for (int v = 0; v < 16; ++v) pkd[v] = ptx::pack2<kBF16>(__uint_as_float(r[2 * v]), __uint_as_float(r[2 * v + 1]));
-        if (row_ok) {
+        if (row_ok && cc * 32 < args.dl) {
           uint4* dst = reinterpret_cast<uint4*>((is_dk ? dk_row : dv_row) + cc * 64);
 #pragma unroll
           for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pkd[4 * v], pkd[4 * v + 1], pkd[4 * v + 2], pkd[4 * v + 3]);
@@ -764,7 +769,7 @@ cudaError_t launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   const unsigned pre_blocks = (unsigned)std::min<long long>((pre_warps + 7) / 8, 148LL * 16);
   bwd_pre_kernel<D, BF><<<pre_blocks, 256, 0, st>>>(o, dout, lse, a.dq_acc, const_cast<float*>(a.lse2),
                                                      const_cast<float*>(a.Dv), a.N, Npad, rows, a.scale, a.cu_q,
-                                                     a.total_q, a.H);
+                                                     a.total_q, a.H, a.dl);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   static std::atomic<uint64_t> smem_set{0};
@@ -784,9 +789,9 @@ cudaError_t launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   bwd_kernel<D, BF><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mk, mv, mdo, mdq, a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (ev_stop && (e = cudaEventRecord(ev_stop, st)) != cudaSuccess) return e;
-  const long long total_vec8 = (long long)a.BH * (a.cu_q ? Npad : a.N) * D / 8;
+  const long long total_vec8 = (long long)a.BH * (a.cu_q ? Npad : a.N) * a.dl / 8;
   const unsigned blocks = (unsigned)std::min<long long>((total_vec8 + 255) / 256, 148LL * 16);
-  bwd_dq_kernel<D, BF><<<blocks, 256, 0, st>>>(a.dq_acc, dq, a.N, Npad, total_vec8, a.cu_q, a.total_q, a.H);
+  bwd_dq_kernel<D, BF><<<blocks, 256, 0, st>>>(a.dq_acc, dq, a.N, Npad, total_vec8, a.cu_q, a.total_q, a.H, a.dl);
   return cudaGetLastError();
 }
 
@@ -810,6 +815,7 @@ inline cudaError_t run_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const C
   a.dq_acc = reinterpret_cast<float*>(ws);
   a.lse2 = reinterpret_cast<const float*>(ws + al((size_t)BH * npad * d * 4));
   a.Dv = reinterpret_cast<const float*>(ws + al((size_t)BH * npad * d * 4) + al((size_t)BH * npad * 4));
+  a.dl = d;
   a.key_lens = key_lens;
   a.col_ptr = col_ptr;
   a.row_idx = row_idx;
@@ -827,7 +833,7 @@ inline cudaError_t run_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const C
   a.scale = scale;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.budget_ns = budget_ns;
-  if (d == 64)
+  if (d <= 64)  // 32 runs on the 64 kernel
     return bf16 ? launch_bwd<64, true>(mq, mk, mv, mdo, mdq, o, dout, lse, dq, a, st, ev_start, ev_stop)
                 : launch_bwd<64, false>(mq, mk, mv, mdo, mdq, o, dout, lse, dq, a, st, ev_start, ev_stop);
   return bf16 ? launch_bwd<128, true>(mq, mk, mv, mdo, mdq, o, dout, lse, dq, a, st, ev_start, ev_stop)

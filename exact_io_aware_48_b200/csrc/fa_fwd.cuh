@@ -60,6 +60,7 @@ struct FwdArgs {
   int total_q, total_k;  // packed: token counts; O is [total_q, H, d], LSE [H, total_q]
   int H, N, nT, npairs, BH;  // packed: N = the longest query sequence, Nk the longest key sequence
   int Nk;
+  int dl;  // head dim of the tensors: D, or 32 / 96 run on the 64 / 128 kernels (TMA zero-fills the columns past dl)
   // split-K/V decode: the N queries of (b, h) are the last N positions of its sequence, so query r sees key c iff
   // c < len_k and (causal) c <= r + len_k - N; unit s of a Q tile covers K/V tiles [s*kv_split_tiles, ...+ that)
   int nsplit, kv_split_tiles;
@@ -475,7 +476,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
       size_t prow = 0;
       if constexpr (split) prow = ((size_t)u.split * args.BH + u.bh) * (size_t)(args.nT * kTile) + grow;
       const size_t orow_idx = packed ? (size_t)(u.g.q0 + grow) * args.H + u.h : (size_t)u.bh * args.N + grow;
-      uint8_t* orow = reinterpret_cast<uint8_t*>(args.o) + orow_idx * D * 2;
+      uint8_t* orow = reinterpret_cast<uint8_t*>(args.o) + orow_idx * args.dl * 2;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t orr[32];
@@ -504,7 +505,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
             const float bb = nonempty ? __uint_as_float(orr[2 * i + 1]) * inv : 0.0f;
             pk[i] = ptx::pack2<kBF16>(a, bb);
           }
-          if (row_ok) {
+          if (row_ok && c * 32 < args.dl) {
             uint4* dst = reinterpret_cast<uint4*>(orow + c * 64);
 #pragma unroll
             for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
@@ -541,7 +542,7 @@ template <int D, bool kBF16>
 __global__ void __launch_bounds__(256) splitkv_combine_kernel(const float* __restrict__ o_part,
                                                               const float* __restrict__ lse_part,
                                                               void* __restrict__ o, float* __restrict__ lse,
-                                                              int nsplit, int BH, int N, int Npad) {
+                                                              int nsplit, int BH, int N, int Npad, int dl) {
   const int lane = threadIdx.x % 32;
   const long long rows = (long long)BH * N;
   const long long nwarps = ((long long)gridDim.x * blockDim.x) / 32;
@@ -577,11 +578,13 @@ __global__ void __launch_bounds__(256) splitkv_combine_kernel(const float* __res
     uint32_t pk[kCols / 2];
 #pragma unroll
     for (int c = 0; c < kCols; c += 2) pk[c / 2] = ptx::pack2<kBF16>(acc[c] * inv, acc[c + 1] * inv);
-    uint16_t* dst = reinterpret_cast<uint16_t*>(o) + ((size_t)bh * N + q) * D + lane * kCols;
-    if constexpr (kCols == 4) {
-      *reinterpret_cast<uint2*>(dst) = make_uint2(pk[0], pk[1]);
-    } else {
-      *reinterpret_cast<uint32_t*>(dst) = pk[0];
+    uint16_t* dst = reinterpret_cast<uint16_t*>(o) + ((size_t)bh * N + q) * dl + lane * kCols;
+    if (lane * kCols < dl) {  // columns past the head dim are the zero padding
+      if constexpr (kCols == 4) {
+        *reinterpret_cast<uint2*>(dst) = make_uint2(pk[0], pk[1]);
+      } else {
+        *reinterpret_cast<uint32_t*>(dst) = pk[0];
+      }
     }
     if (lane == 0) lse[(size_t)bh * N + q] = wsum > 0.f ? m + __logf(wsum) : -INFINITY;
   }

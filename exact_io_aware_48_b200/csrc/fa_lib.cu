@@ -47,6 +47,10 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// Head dims: 64 and 128 natively; 32 and 96 run on the 64 / 128 kernels, whose TMA boxes are 64 columns wide and
+// zero-fill the columns past the tensor's own, so the extra columns add nothing to any product.
+bool head_dim_ok(int d) { return d == 32 || d == 64 || d == 96 || d == 128; }
+
 int cuda_fail(cudaError_t e) {
   t_last_error = cudaGetErrorString(e);
   return FA_ERR_CUDA;
@@ -61,7 +65,7 @@ int check_common(const void* q, const void* k, const void* v, int B, int H, int 
   if (B < 1 || H < 1 || N < 1 || N > kMaxN) return FA_ERR_INVALID_ARG;
   if (dtype != FA_BF16 && dtype != FA_FP16) return FA_ERR_INVALID_ARG;
   if (!(scale > 0.0f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (!head_dim_ok(d)) return FA_ERR_UNSUPPORTED;
   if ((long long)B * H * N * d > kMaxElems) return FA_ERR_INVALID_ARG;
   return FA_OK;
 }
@@ -179,7 +183,7 @@ cudaError_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
 int fwd_tiles_for(int d) {
   const int forced = g_fwd_tiles.load();
   if (forced == 1 || forced == 2) return forced;
-  return d == 64 ? 1 : 2;
+  return d <= 64 ? 1 : 2;
 }
 
 // Packed variable-length batch description (all null / zero for the dense [B, H, N, d] layout).
@@ -214,6 +218,7 @@ int run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, in
   a.total_q = pk.total_q;
   a.total_k = pk.total_k;
   a.Nk = pk.cu_q ? pk.Nk : N;
+  a.dl = d;
   a.nsplit = 1;
   a.kv_split_tiles = 0;
   a.o_part = nullptr;
@@ -229,12 +234,12 @@ int run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, in
   cudaError_t e;
   const bool bf = dtype == FA_BF16;
   if (fwd_tiles_for(d) == 2) {
-    if (d == 64)
+    if (d <= 64)
       e = bf ? launch_fwd<64, true, 2>(mq, mk, mv, a, st) : launch_fwd<64, false, 2>(mq, mk, mv, a, st);
     else
       e = bf ? launch_fwd<128, true, 2>(mq, mk, mv, a, st) : launch_fwd<128, false, 2>(mq, mk, mv, a, st);
   } else {
-    if (d == 64)
+    if (d <= 64)
       e = bf ? launch_fwd<64, true, 1>(mq, mk, mv, a, st) : launch_fwd<64, false, 1>(mq, mk, mv, a, st);
     else
       e = bf ? launch_fwd<128, true, 1>(mq, mk, mv, a, st) : launch_fwd<128, false, 1>(mq, mk, mv, a, st);
@@ -301,9 +306,12 @@ int splitkv_splits(int B, int H, int Nq, int Nk, int requested) {
   return best;
 }
 
+// Partial results of a split-K/V forward: O rows as wide as the kernel's head dim (64 or 128), then LSE.
+int kernel_dim(int d) { return d <= 64 ? 64 : 128; }
+
 size_t splitkv_bytes(int B, int H, int Nq, int d, int nsplit) {
   const size_t rows = (size_t)nsplit * B * H * ((Nq + fa::kTile - 1) / fa::kTile) * fa::kTile;
-  return align_up(rows * d * 4, 256) + align_up(rows * 4, 256);
+  return align_up(rows * kernel_dim(d) * 4, 256) + align_up(rows * 4, 256);
 }
 
 template <int D, bool BF>
@@ -314,7 +322,7 @@ cudaError_t launch_splitkv(const CUtensorMap& mq, const CUtensorMap& mk, const C
   const long long rows = (long long)a.BH * a.N;
   const unsigned blocks = (unsigned)std::min<long long>((rows + 7) / 8, 148LL * 16);
   fa::splitkv_combine_kernel<D, BF><<<blocks, 256, 0, st>>>(a.o_part, a.lse_part, o, lse, a.nsplit, a.BH, a.N,
-                                                            a.nT * fa::kTile);
+                                                            a.nT * fa::kTile, a.dl);
   return cudaGetLastError();
 }
 
@@ -328,7 +336,7 @@ int check_packed(const void* q, const void* k, const void* v, const int32_t* cu_
   if (total_q < 1 || total_k < 1) return FA_ERR_INVALID_ARG;
   if (dtype != FA_BF16 && dtype != FA_FP16) return FA_ERR_INVALID_ARG;
   if (!(scale > 0.0f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (!head_dim_ok(d)) return FA_ERR_UNSUPPORTED;
   const long long npad = (long long)(max_q + fa::kTile - 1) / fa::kTile * fa::kTile;
   if ((long long)total_q * H * d > kMaxElems || (long long)total_k * H * d > kMaxElems ||
       (long long)B * H * npad * d > kMaxElems)
@@ -394,7 +402,7 @@ int fa_blockmask_lists(const uint8_t* mask, int nT, int32_t* row_ptr, int32_t* c
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d, int has_block_mask) {
-  if (B < 1 || H < 1 || N < 1 || N > kMaxN || (d != 64 && d != 128)) return 0;
+  if (B < 1 || H < 1 || N < 1 || N > kMaxN || !head_dim_ok(d)) return 0;
   const int nT = (N + fa::kTile - 1) / fa::kTile;
   return fa::bwd_workspace_bytes(B * H, nT, d) + (has_block_mask ? lists_bytes(nT) : 0);
 }
@@ -451,7 +459,7 @@ int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* l
 }
 
 size_t fa_bwd_varlen_workspace_size(int B, int H, int max_seqlen_q, int d) {
-  if (B < 1 || H < 1 || max_seqlen_q < 1 || max_seqlen_q > kMaxN || (d != 64 && d != 128)) return 0;
+  if (B < 1 || H < 1 || max_seqlen_q < 1 || max_seqlen_q > kMaxN || !head_dim_ok(d)) return 0;
   return fa::bwd_workspace_bytes(B * H, (max_seqlen_q + fa::kTile - 1) / fa::kTile, d);
 }
 
@@ -484,7 +492,7 @@ int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, co
 }
 
 size_t fa_fwd_splitkv_workspace_size(int B, int H, int Nq, int Nk, int d, int num_splits) {
-  if (B < 1 || H < 1 || Nq < 1 || Nk < 1 || Nq > kMaxN || Nk > kMaxN || (d != 64 && d != 128)) return 0;
+  if (B < 1 || H < 1 || Nq < 1 || Nk < 1 || Nq > kMaxN || Nk > kMaxN || !head_dim_ok(d)) return 0;
   if (num_splits < 0 || num_splits > kMaxSplits) return 0;
   return splitkv_bytes(B, H, Nq, d, splitkv_splits(B, H, Nq, Nk, num_splits));
 }
@@ -518,6 +526,7 @@ int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* 
   a.H = H;
   a.N = Nq;
   a.Nk = Nk;
+  a.dl = d;
   a.nT = (Nq + fa::kTile - 1) / fa::kTile;
   a.npairs = a.nT;  // one Q tile per CTA
   a.BH = B * H;
@@ -529,11 +538,11 @@ int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* 
   a.kv_split_tiles = (tiles_k + nsplit - 1) / nsplit;
   const size_t rows = (size_t)nsplit * a.BH * a.nT * fa::kTile;
   a.o_part = static_cast<float*>(workspace);
-  a.lse_part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + align_up(rows * d * 4, 256));
+  a.lse_part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + align_up(rows * kernel_dim(d) * 4, 256));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const bool bf = dtype == FA_BF16;
   cudaError_t e;
-  if (d == 64)
+  if (d <= 64)
     e = bf ? launch_splitkv<64, true>(mq, mk, mv, a, o, lse, st) : launch_splitkv<64, false>(mq, mk, mv, a, o, lse, st);
   else
     e = bf ? launch_splitkv<128, true>(mq, mk, mv, a, o, lse, st)

@@ -51,7 +51,7 @@ extern "C" int fa_bwd_noalloc(const void* q, const void* k, const void* v, const
                               float softmax_scale, int causal, const int32_t* key_lens, const uint8_t* block_mask,
                               int dtype, void* stream) {
   const size_t need = fa_bwd_workspace_size(B, H, N, d, block_mask != nullptr);
-  if (need == 0) return (d != 64 && d != 128 && B >= 1 && H >= 1 && N >= 1) ? FA_ERR_UNSUPPORTED
+  if (need == 0) return (d != 32 && d != 64 && d != 96 && d != 128 && B >= 1 && H >= 1 && N >= 1) ? FA_ERR_UNSUPPORTED
                                                                              : FA_ERR_INVALID_ARG;
   if (need > (size_t)FA_NOALLOC_SCRATCH_BYTES) return FA_ERR_WORKSPACE;  // problem too large for the fixed array
   void* scratch = nullptr;

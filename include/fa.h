@@ -19,7 +19,8 @@
  *   Pointers    Device pointers, 16-byte aligned, caller-owned; the library never allocates, frees or keeps them.
  *               Scratch that a call needs is passed in as `workspace` (device memory, 256-byte aligned) of at
  *               least the size returned by the matching *_workspace_size query.
- *   Shapes      B >= 1, H >= 1, 1 <= N <= 1048576 (2^20), d in {64, 128}, B*H*N*d <= 2^34, softmax_scale finite
+ *   Shapes      B >= 1, H >= 1, 1 <= N <= 1048576 (2^20), d in {32, 64, 96, 128} (32 and 96 run on the 64 and 128
+ *               kernels with the extra columns zero, at their cost), B*H*N*d <= 2^34, softmax_scale finite
  *               and > 0.
  *   Execution   Asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).  Inputs must stay valid
  *               until the stream reaches the work.
@@ -42,7 +43,7 @@ extern "C" {
 typedef enum {
   FA_OK = 0,
   FA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad shape, scale <= 0, bad dtype */
-  FA_ERR_UNSUPPORTED = 2, /* head dimension other than 64 or 128 */
+  FA_ERR_UNSUPPORTED = 2, /* head dimension other than 32, 64, 96 or 128 */
   FA_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed (message: fa_last_error_string) */
   FA_ERR_TIMEOUT = 4,     /* a kernel wait ran out of its time budget (device-detected) */
   FA_ERR_WORKSPACE = 5    /* workspace missing, misaligned or smaller than the query says */
@@ -121,7 +122,7 @@ int fa_blockmask_lists(const uint8_t* mask, int nT, int32_t* row_ptr, int32_t* c
  *               device (no access leaves the tensors) but the results for such sequences are unspecified.
  *   Visibility  Key c of sequence b is visible from its query r (positions within the sequence) iff
  *               c < len_k(b) && (causal == 0 || c <= r).  For len_q == len_k this is ordinary causal self-attention.
- *   Shapes      total_q, total_k >= 1; total*H*d and B*H*ceil(max_seqlen_q/128)*128*d <= 2^34; d in {64, 128}.
+ *   Shapes      total_q, total_k >= 1; total*H*d and B*H*ceil(max_seqlen_q/128)*128*d <= 2^34; d as for fa_fwd.
  * Everything else (pointers, execution, errors) is as for fa_fwd / fa_bwd.  No block mask, no key_lens.
  */
 int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int32_t* cu_seqlens_q,
@@ -142,7 +143,7 @@ int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* l
  *   Splits      num_splits in [0, 32]; 0 picks enough ranges to fill the GPU.  The result does not depend on the
  *               number of splits beyond fp32 rounding.
  *   Workspace   fa_fwd_splitkv_workspace_size(B, H, Nq, Nk, d, num_splits) bytes (256-byte aligned device memory).
- *   Shapes      1 <= Nq, Nk <= 2^20, B*H*Nq*d and B*H*Nk*d <= 2^34, d in {64, 128}.  Everything else as fa_fwd.
+ *   Shapes      1 <= Nq, Nk <= 2^20, B*H*Nq*d and B*H*Nk*d <= 2^34, d as for fa_fwd.  Everything else as fa_fwd.
  */
 size_t fa_fwd_splitkv_workspace_size(int B, int H, int Nq, int Nk, int d, int num_splits);
 
