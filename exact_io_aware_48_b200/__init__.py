@@ -47,7 +47,8 @@ def _require_cuda(*ts):
 def attention_fwd(q, k, v, causal=False, softmax_scale=None, key_lens=None, block_mask=None, stream=None):
     """O, LSE = exact attention of [B, H, N, d] CUDA tensors (bf16 or fp16).
 
-    key_lens: optional int32 CUDA tensor [B]; block_mask: optional uint8 CUDA tensor [nT, nT] (128x128 tiles).
+    key_lens: optional int32 CUDA tensor [B]; block_mask: optional uint8 CUDA tensor [nT, nT] (128x128 tiles,
+    shared by all heads) or [H, nT, nT] (one mask per head).
     Returns O (same dtype) and LSE (fp32, natural log) [B, H, N].
     """
     import torch
@@ -59,6 +60,11 @@ def attention_fwd(q, k, v, causal=False, softmax_scale=None, key_lens=None, bloc
     dt = _dtype_code(q)
     if block_mask is None:
         _check(_lib.fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, key_lens, dt, stream), "fa_fwd")
+    elif block_mask.dim() == 3:  # one mask per head
+        ws_bytes = _lib.fa_blocksparse_heads_workspace_size(H, N)
+        ws = torch.empty(ws_bytes, device=q.device, dtype=torch.uint8)
+        _check(_lib.fa_fwd_blocksparse_heads(q, k, v, o, lse, B, H, N, d, scale, causal, key_lens, block_mask, ws,
+                                             ws_bytes, dt, stream), "fa_fwd_blocksparse_heads")
     else:
         ws_bytes = _lib.fa_blocksparse_workspace_size(N)
         ws = torch.empty(ws_bytes, device=q.device, dtype=torch.uint8)
@@ -75,6 +81,13 @@ def attention_bwd(q, k, v, o, dout, lse, causal=False, softmax_scale=None, key_l
     B, H, N, d = q.shape
     scale = softmax_scale if softmax_scale is not None else 1.0 / math.sqrt(d)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    if block_mask is not None and block_mask.dim() == 3:  # one mask per head
+        ws_bytes = _lib.fa_bwd_blocksparse_heads_workspace_size(B, H, N, d)
+        ws = torch.empty(ws_bytes, device=q.device, dtype=torch.uint8)
+        _check(_lib.fa_bwd_blocksparse_heads(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, causal, key_lens,
+                                             block_mask, ws, ws_bytes, _dtype_code(q), stream),
+               "fa_bwd_blocksparse_heads")
+        return dq, dk, dv
     ws_bytes = _lib.fa_bwd_workspace_size(B, H, N, d, block_mask is not None)
     ws = torch.empty(ws_bytes, device=q.device, dtype=torch.uint8)
     _check(_lib.fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, causal, key_lens, block_mask, ws,

@@ -38,6 +38,11 @@ SIGNATURES = {
     "fa_fwd_varlen": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P], _I),
     "fa_bwd_varlen_workspace_size": ([_I, _I, _I, _I], _SZ),
     "fa_fwd_splitkv_workspace_size": ([_I, _I, _I, _I, _I, _I], _SZ),
+    "fa_blocksparse_heads_workspace_size": ([_I, _I], _SZ),
+    "fa_fwd_blocksparse_heads": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P, _P, _P, _SZ, _I, _P], _I),
+    "fa_bwd_blocksparse_heads_workspace_size": ([_I, _I, _I, _I], _SZ),
+    "fa_bwd_blocksparse_heads": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P, _P, _P, _SZ, _I,
+                                  _P], _I),
     "fa_fwd_splitkv": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P, _I, _P, _SZ, _I, _P], _I),
     "fa_bwd_varlen": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P, _SZ, _I,
                        _P], _I),
@@ -193,3 +198,26 @@ def fa_fwd_splitkv(q, k, v, o, lse, B, H, Nq, Nk, d, softmax_scale, causal, key_
     return load().fa_fwd_splitkv(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nq, Nk, d, softmax_scale,
                                  int(causal), _ptr(key_lens), num_splits, _ptr(workspace), workspace_bytes, dtype,
                                  _stream(stream))
+
+
+def fa_blocksparse_heads_workspace_size(H, N) -> int:
+    return load().fa_blocksparse_heads_workspace_size(H, N)
+
+
+def fa_fwd_blocksparse_heads(q, k, v, o, lse, B, H, N, d, softmax_scale, causal, key_lens, block_masks, workspace,
+                             workspace_bytes, dtype, stream=None) -> int:
+    return load().fa_fwd_blocksparse_heads(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, softmax_scale,
+                                           int(causal), _ptr(key_lens), _ptr(block_masks), _ptr(workspace),
+                                           workspace_bytes, dtype, _stream(stream))
+
+
+def fa_bwd_blocksparse_heads_workspace_size(B, H, N, d) -> int:
+    return load().fa_bwd_blocksparse_heads_workspace_size(B, H, N, d)
+
+
+def fa_bwd_blocksparse_heads(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, softmax_scale, causal, key_lens,
+                             block_masks, workspace, workspace_bytes, dtype, stream=None) -> int:
+    return load().fa_bwd_blocksparse_heads(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq),
+                                           _ptr(dk), _ptr(dv), B, H, N, d, softmax_scale, int(causal), _ptr(key_lens),
+                                           _ptr(block_masks), _ptr(workspace), workspace_bytes, dtype,
+                                           _stream(stream))

@@ -81,6 +81,7 @@ struct BwdArgs {
   const int32_t* key_lens;
   const int32_t* col_ptr;  // CSC of the block mask (nullptr: dense)
   const int32_t* row_idx;
+  long long list_head_stride;  // per-head masks: int32 distance between heads' lists (0: one mask for all heads)
   const int32_t* cu_q;  // packed variable-length batch: cumulative sequence lengths (nullptr: dense [B,H,N,d])
   const int32_t* cu_k;
   int total_q, total_k;  // packed: token counts; dK, dV are [total_k, H, d]
@@ -327,7 +328,8 @@ __global__ void __launch_bounds__(512, 1)
       while (ok && us.next(L)) {
         const BwdUnit u = bwd_unit(L, args);
         ColTileIter it;
-        it.init(args.col_ptr, args.row_idx, u.j, u.nTq, causal ? u.j : 0, u.visible);
+        it.init(args.col_ptr ? args.col_ptr + u.h * args.list_head_stride : nullptr,
+                args.row_idx + u.h * args.list_head_stride, u.j, u.nTq, causal ? u.j : 0, u.visible);
         if (it.count() == 0) continue;
         const int kb = ku % KB;
         // the buffer's previous K/V tiles must have been read by every MMA of their unit
@@ -443,7 +445,8 @@ __global__ void __launch_bounds__(512, 1)
       while (ok && us.next(L)) {
         const BwdUnit u = bwd_unit(L, args);
         ColTileIter it;
-        it.init(args.col_ptr, args.row_idx, u.j, u.nTq, causal ? u.j : 0, u.visible);
+        it.init(args.col_ptr ? args.col_ptr + u.h * args.list_head_stride : nullptr,
+                args.row_idx + u.h * args.list_head_stride, u.j, u.nTq, causal ? u.j : 0, u.visible);
         if (it.count() == 0) continue;
         const int kb = ku % KB;
         dk_k = ptx::sw128_desc(ptx::smem_addr(sK(kb)), 16, 1024);
@@ -541,7 +544,8 @@ __global__ void __launch_bounds__(512, 1)
     while (ok && us.next(L)) {
       const BwdUnit u = bwd_unit(L, args);
       ColTileIter it;
-      it.init(args.col_ptr, args.row_idx, u.j, u.nTq, causal ? u.j : 0, u.visible);
+      it.init(args.col_ptr ? args.col_ptr + u.h * args.list_head_stride : nullptr,
+                args.row_idx + u.h * args.list_head_stride, u.j, u.nTq, causal ? u.j : 0, u.visible);
       const int j = u.j, kv_lim = u.kv_lim;
       const int gc = j * kTile + c;  // key index in the sequence
       int i;
@@ -655,7 +659,8 @@ __global__ void __launch_bounds__(512, 1)
     while (ok && us.next(L)) {
       const BwdUnit u = bwd_unit(L, args);
       ColTileIter it;
-      it.init(args.col_ptr, args.row_idx, u.j, u.nTq, causal ? u.j : 0, u.visible);
+      it.init(args.col_ptr ? args.col_ptr + u.h * args.list_head_stride : nullptr,
+                args.row_idx + u.h * args.list_head_stride, u.j, u.nTq, causal ? u.j : 0, u.visible);
       const int n_iters = it.count();
       int i;
       while (it.next(i)) {
@@ -801,7 +806,7 @@ inline cudaError_t run_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const C
                            const int32_t* key_lens, const int32_t* col_ptr, const int32_t* row_idx, void* workspace,
                            bool bf16, uint64_t budget_ns, cudaStream_t st, cudaEvent_t ev_start,
                            cudaEvent_t ev_stop, const int32_t* cu_q = nullptr, const int32_t* cu_k = nullptr,
-                           int total_q = 0, int total_k = 0, int Nk = 0) {
+                           int total_q = 0, int total_k = 0, int Nk = 0, long long list_head_stride = 0) {
   // packed variable-length batches: N / Nk are the longest query / key sequences; dense: Nk = N
   if (Nk <= 0) Nk = N;
   const int nT = (N + kTile - 1) / kTile;
@@ -819,6 +824,7 @@ inline cudaError_t run_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const C
   a.key_lens = key_lens;
   a.col_ptr = col_ptr;
   a.row_idx = row_idx;
+  a.list_head_stride = list_head_stride;
   a.cu_q = cu_q;
   a.cu_k = cu_k;
   a.total_q = total_q;

@@ -55,6 +55,7 @@ struct FwdArgs {
   const int32_t* key_lens;
   const int32_t* row_ptr;  // CSR of the block mask (nullptr: dense)
   const int32_t* col_idx;
+  long long list_head_stride;  // per-head masks: int32 distance between heads' lists (0: one mask for all heads)
   const int32_t* cu_q;  // packed variable-length batch: cumulative sequence lengths (nullptr: dense [B,H,N,d])
   const int32_t* cu_k;
   int total_q, total_k;  // packed: token counts; O is [total_q, H, d], LSE [H, total_q]
@@ -119,7 +120,8 @@ __device__ __forceinline__ FwdUnit fwd_unit(int L, const FwdArgs& a, int tiles) 
 
 __device__ __forceinline__ void fwd_tiles(PairTileIter& it, const FwdUnit& u, const FwdArgs& a) {
   if (a.row_ptr != nullptr)
-    it.init_sparse(a.row_ptr, a.col_idx, u.qt0, a.nT, u.end0, u.end1);
+    it.init_sparse(a.row_ptr + u.h * a.list_head_stride, a.col_idx + u.h * a.list_head_stride, u.qt0, a.nT, u.end0,
+                   u.end1);
   else
     it.init_dense(u.end0, u.end1, u.begin);
 }

@@ -15,7 +15,7 @@
 
 namespace {
 
-constexpr int kVersion = 10200;  // 1.2.0: split-K/V decode forward
+constexpr int kVersion = 10300;  // 1.3.0: head dims 32 and 96, per-head block masks
 constexpr int kMaxN = 1 << 20;
 constexpr long long kMaxElems = 1LL << 34;
 
@@ -195,7 +195,7 @@ struct Packed {
 
 int run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
             float scale, int causal, const int32_t* key_lens, const int32_t* row_ptr, const int32_t* col_idx,
-            int dtype, cudaStream_t st, const Packed& pk = Packed()) {
+            int dtype, cudaStream_t st, const Packed& pk = Packed(), long long list_head_stride = 0) {
   CUtensorMap mq, mk, mv;
   int rc;
   if (pk.cu_q) {
@@ -213,6 +213,7 @@ int run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, in
   a.key_lens = key_lens;
   a.row_ptr = row_ptr;
   a.col_idx = col_idx;
+  a.list_head_stride = list_head_stride;
   a.cu_q = pk.cu_q;
   a.cu_k = pk.cu_k;
   a.total_q = pk.total_q;
@@ -271,8 +272,11 @@ Lists carve_lists(void* ws, int nT) {
   return l;
 }
 
-int launch_lists(const uint8_t* mask, int nT, const Lists& l, cudaStream_t st) {
-  fa::blockmask_lists_kernel<<<1, fa::kMaskThreads, 0, st>>>(mask, nT, l.row_ptr, l.col_idx, l.col_ptr, l.row_idx);
+// Tile lists of `heads` masks ([heads][nT][nT]); head h's lists are lists_bytes(nT) bytes after head 0's.
+int launch_lists(const uint8_t* mask, int nT, const Lists& l, cudaStream_t st, int heads = 1) {
+  const long long stride = heads > 1 ? (long long)(lists_bytes(nT) / 4) : 0;
+  fa::blockmask_lists_kernel<<<heads, fa::kMaskThreads, 0, st>>>(mask, nT, l.row_ptr, l.col_idx, l.col_ptr,
+                                                                 l.row_idx, stride);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? FA_OK : cuda_fail(e);
 }
@@ -519,6 +523,7 @@ int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* 
   a.key_lens = key_lens;
   a.row_ptr = nullptr;
   a.col_idx = nullptr;
+  a.list_head_stride = 0;
   a.cu_q = nullptr;
   a.cu_k = nullptr;
   a.total_q = 0;
@@ -547,6 +552,66 @@ int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* 
   else
     e = bf ? launch_splitkv<128, true>(mq, mk, mv, a, o, lse, st)
            : launch_splitkv<128, false>(mq, mk, mv, a, o, lse, st);
+  return e == cudaSuccess ? FA_OK : cuda_fail(e);
+}
+
+size_t fa_blocksparse_heads_workspace_size(int H, int N) {
+  if (H < 1 || N < 1 || N > kMaxN) return 0;
+  return (size_t)H * lists_bytes((N + fa::kTile - 1) / fa::kTile);
+}
+
+int fa_fwd_blocksparse_heads(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
+                             int d, float softmax_scale, int causal, const int32_t* key_lens,
+                             const uint8_t* block_masks, void* workspace, size_t workspace_bytes, int dtype,
+                             void* stream) {
+  int rc = check_common(q, k, v, B, H, N, d, softmax_scale, dtype);
+  if (rc != FA_OK) return rc;
+  if (!o || !lse || !block_masks || !aligned(o, 16) || !aligned(lse, 4) || (key_lens && !aligned(key_lens, 4)))
+    return FA_ERR_INVALID_ARG;
+  const int nT = (N + fa::kTile - 1) / fa::kTile;
+  if (nT > fa::kMaxMaskTiles) return FA_ERR_INVALID_ARG;
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < fa_blocksparse_heads_workspace_size(H, N))
+    return FA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Lists l = carve_lists(workspace, nT);
+  if ((rc = launch_lists(block_masks, nT, l, st, H)) != FA_OK) return rc;
+  return run_fwd(q, k, v, o, lse, B, H, N, d, softmax_scale, causal, key_lens, l.row_ptr, l.col_idx, dtype, st,
+                 Packed(), H > 1 ? (long long)(lists_bytes(nT) / 4) : 0);
+}
+
+size_t fa_bwd_blocksparse_heads_workspace_size(int B, int H, int N, int d) {
+  if (B < 1 || H < 1 || N < 1 || N > kMaxN || !head_dim_ok(d)) return 0;
+  const int nT = (N + fa::kTile - 1) / fa::kTile;
+  return fa::bwd_workspace_bytes(B * H, nT, d) + (size_t)H * lists_bytes(nT);
+}
+
+int fa_bwd_blocksparse_heads(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                             const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                             float softmax_scale, int causal, const int32_t* key_lens, const uint8_t* block_masks,
+                             void* workspace, size_t workspace_bytes, int dtype, void* stream) {
+  int rc = check_common(q, k, v, B, H, N, d, softmax_scale, dtype);
+  if (rc != FA_OK) return rc;
+  if (!o || !dout || !lse || !dq || !dk || !dv || !block_masks) return FA_ERR_INVALID_ARG;
+  if (!aligned(o, 16) || !aligned(dout, 16) || !aligned(lse, 4) || !aligned(dq, 16) || !aligned(dk, 16) ||
+      !aligned(dv, 16) || (key_lens && !aligned(key_lens, 4)))
+    return FA_ERR_INVALID_ARG;
+  const int nT = (N + fa::kTile - 1) / fa::kTile;
+  if (nT > fa::kMaxMaskTiles) return FA_ERR_INVALID_ARG;
+  const size_t need = fa_bwd_blocksparse_heads_workspace_size(B, H, N, d);
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < need) return FA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Lists l = carve_lists(static_cast<uint8_t*>(workspace) + fa::bwd_workspace_bytes(B * H, nT, d), nT);
+  if ((rc = launch_lists(block_masks, nT, l, st, H)) != FA_OK) return rc;
+  CUtensorMap mq, mk, mv, mdo, mdq;
+  if ((rc = make_map(&mq, q, B * H, N, d, dtype)) != FA_OK) return rc;
+  if ((rc = make_map(&mk, k, B * H, N, d, dtype)) != FA_OK) return rc;
+  if ((rc = make_map(&mv, v, B * H, N, d, dtype)) != FA_OK) return rc;
+  if ((rc = make_map(&mdo, dout, B * H, N, d, dtype)) != FA_OK) return rc;
+  if ((rc = make_map_f32(&mdq, workspace, (long long)B * H * nT * fa::kTile, d)) != FA_OK) return rc;
+  cudaError_t e = fa::run_bwd(mq, mk, mv, mdo, mdq, o, dout, lse, dq, dk, dv, B, H, N, d, softmax_scale, causal != 0,
+                              key_lens, l.col_ptr, l.row_idx, workspace, dtype == FA_BF16, g_budget_ns.load(), st,
+                              t_events[FA_KERNEL_BWD_MAIN][0], t_events[FA_KERNEL_BWD_MAIN][1], nullptr, nullptr, 0, 0,
+                              0, H > 1 ? (long long)(lists_bytes(nT) / 4) : 0);
   return e == cudaSuccess ? FA_OK : cuda_fail(e);
 }
 

@@ -11,10 +11,17 @@ constexpr int kMaxMaskTiles = 8192;
 // One CTA of 1024 threads.  Phase 1 counts kept tiles per row and per column, phase 2 turns the counts into
 // exclusive prefix sums (row_ptr, col_ptr), phase 3 writes each row's columns and each column's rows in
 // ascending order.  Integer only; the result is unique, so it must equal any correct CPU construction exactly.
+// Per-head masks: CTA h reads mask + h*nT*nT and writes lists `head_stride` int32 further on (grid = number of
+// masks; one mask shared by all heads: grid 1, stride 0).
 __global__ void __launch_bounds__(kMaskThreads, 1)
     blockmask_lists_kernel(const uint8_t* __restrict__ mask, int nT, int32_t* __restrict__ row_ptr,
                            int32_t* __restrict__ col_idx, int32_t* __restrict__ col_ptr,
-                           int32_t* __restrict__ row_idx) {
+                           int32_t* __restrict__ row_idx, long long head_stride) {
+  mask += (size_t)blockIdx.x * nT * nT;
+  row_ptr += blockIdx.x * head_stride;
+  col_idx += blockIdx.x * head_stride;
+  col_ptr += blockIdx.x * head_stride;
+  row_idx += blockIdx.x * head_stride;
   __shared__ int32_t part_r[kMaskThreads], part_c[kMaskThreads];
   const int tid = threadIdx.x;
   for (int i = tid; i < nT; i += kMaskThreads) {

@@ -111,6 +111,27 @@ int fa_blockmask_lists(const uint8_t* mask, int nT, int32_t* row_ptr, int32_t* c
                        int32_t* row_idx, void* stream);
 
 /*
+ * Per-head block masks: as fa_fwd_blocksparse / fa_bwd, but block_masks is [H, nT, nT] uint8 (head h's mask at
+ * block_masks + h*nT*nT, shared by all b).  The pages describe one tile mask; a separate mask per head is the same
+ * tile skipping with one CSR/CSC list set per head (explainer page, block-sparse section).  Workspace:
+ * fa_blocksparse_heads_workspace_size(H, N) for the forward, fa_bwd_blocksparse_heads_workspace_size(B, H, N, d)
+ * for the backward.
+ */
+size_t fa_blocksparse_heads_workspace_size(int H, int N);
+
+int fa_fwd_blocksparse_heads(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
+                             int d, float softmax_scale, int causal, const int32_t* key_lens,
+                             const uint8_t* block_masks, void* workspace, size_t workspace_bytes, int dtype,
+                             void* stream);
+
+size_t fa_bwd_blocksparse_heads_workspace_size(int B, int H, int N, int d);
+
+int fa_bwd_blocksparse_heads(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                             const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                             float softmax_scale, int causal, const int32_t* key_lens, const uint8_t* block_masks,
+                             void* workspace, size_t workspace_bytes, int dtype, void* stream);
+
+/*
  * Packed variable-length batches.  The pages give no interface for this (it generalises the key-length masking
  * they describe for padded BERT batches, explainer page, block-sparse and masking section): B sequences of
  * different lengths are stored back to back without padding.

@@ -269,6 +269,16 @@ def attn_fwd_decode(q, k, v, scale, causal=False, key_lens=None):
     return o, lse
 
 
+def attn_bwd_head_masks(q, k, v, do, scale, masks, causal=False, key_lens=None, tile=128):
+    """Per-head block masks (masks [H, nT, nT]): head h is attn_bwd of that head's slice with mask masks[h].
+    Returns (dQ, dK, dV, O, LSE) like attn_bwd."""
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    outs = [attn_bwd(q[:, h:h + 1], k[:, h:h + 1], v[:, h:h + 1], do[:, h:h + 1], scale, causal=causal,
+                     key_lens=key_lens, block_mask=np.asarray(masks[h], dtype=np.uint8), tile=tile)
+            for h in range(q.shape[1])]
+    return tuple(np.concatenate([o[i] for o in outs], axis=1) for i in range(5))
+
+
 def blockmask_csr(mask):
     """CSR of a square 0/1 tile mask: (row_ptr [nT+1] int32, col_idx [nnz] int32), ascending columns."""
     m = np.ascontiguousarray(mask, dtype=np.uint8)

@@ -31,7 +31,7 @@ def test_header_and_binding_agree(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.fa_version() == 10200
+    assert lib.fa_version() == 10300
     assert _lib.fa_status_string(0) == "FA_OK"
     assert _lib.fa_status_string(4) == "FA_ERR_TIMEOUT"
     assert _lib.fa_status_string(99) == "FA_UNKNOWN_STATUS"

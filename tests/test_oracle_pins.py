@@ -452,3 +452,28 @@ def test_decode_key_lengths_truncate_the_cache_and_empty_queries():
     # sequence 1 has 3 keys for 5 queries: queries 0 and 1 see nothing (c <= r + 3 - 5 < 0), query 2 sees key 0
     assert np.all(o[1, :, :2] == 0) and np.all(np.isneginf(lse[1, :, :2]))
     np.testing.assert_allclose(o[1, :, 2], v[1, :, 0], rtol=0, atol=1e-15)
+
+
+# ----------------------------------------------------------------------------------------------- per-head masks
+def test_head_masks_all_equal_give_the_shared_mask_result():
+    B, H, N, d = 2, 3, 16, 4
+    q, k, v = qkv(B, H, N, d, 240)
+    do = rnd((B, H, N, d), 241)
+    m = np.array([[1, 0, 1, 1], [1, 1, 0, 0], [0, 1, 1, 0], [1, 1, 1, 1]], np.uint8)
+    shared = oracle.attn_bwd(q, k, v, do, 0.5, block_mask=m, tile=4)
+    per = oracle.attn_bwd_head_masks(q, k, v, do, 0.5, np.stack([m] * H), tile=4)
+    for a, b in zip(per, shared):
+        np.testing.assert_allclose(a, b, rtol=0, atol=1e-14)
+
+
+def test_head_masks_differ_per_head():
+    B, H, N, d = 1, 2, 16, 4
+    q, k, v = qkv(B, H, N, d, 250)
+    do = rnd((B, H, N, d), 251)
+    ones = np.ones((4, 4), np.uint8)
+    band = np.eye(4, dtype=np.uint8)
+    dq, dk, dv, o, lse = oracle.attn_bwd_head_masks(q, k, v, do, 0.5, np.stack([ones, band]), tile=4)
+    od, _ = oracle.attn_fwd(q[:, :1], k[:, :1], v[:, :1], 0.5)  # head 0: all tiles kept = dense
+    np.testing.assert_allclose(o[:, :1], od, rtol=0, atol=1e-14)
+    ob, _ = oracle.attn_fwd(q[:, 1:], k[:, 1:], v[:, 1:], 0.5, block_mask=band, tile=4)
+    np.testing.assert_allclose(o[:, 1:], ob, rtol=0, atol=1e-14)
