@@ -582,7 +582,9 @@ __global__ void __launch_bounds__(256) splitkv_combine_kernel(const float* __res
     for (int c = 0; c < kCols; c += 2) pk[c / 2] = ptx::pack2<kBF16>(acc[c] * inv, acc[c + 1] * inv);
     uint16_t* dst = reinterpret_cast<uint16_t*>(o) + ((size_t)bh * N + q) * dl + lane * kCols;
     if (lane * kCols < dl) {  // columns past the head dim are the zero padding
-      if constexpr (kCols == 4) {
+      if constexpr (kCols == 8) {
+        *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      } else if constexpr (kCols == 4) {
         *reinterpret_cast<uint2*>(dst) = make_uint2(pk[0], pk[1]);
       } else {
         *reinterpret_cast<uint32_t*>(dst) = pk[0];

@@ -10,6 +10,7 @@
 #include "fa.h"
 #include "fa_common.cuh"
 #include "fa_fwd.cuh"
+#include "fa_fwd256.cuh"
 #include "fa_bwd.cuh"
 #include "fa_mask.cuh"
 
@@ -50,6 +51,8 @@ EncodeTiledFn encode_fn() {
 // Head dims: 64 and 128 natively; 32 and 96 run on the 64 / 128 kernels, whose TMA boxes are 64 columns wide and
 // zero-fill the columns past the tensor's own, so the extra columns add nothing to any product.
 bool head_dim_ok(int d) { return d == 32 || d == 64 || d == 96 || d == 128; }
+// The forward also runs d = 256 (its own kernel, fa_fwd256.cuh); the backward does not.
+bool fwd_head_dim_ok(int d) { return head_dim_ok(d) || d == 256; }
 
 int cuda_fail(cudaError_t e) {
   t_last_error = cudaGetErrorString(e);
@@ -59,20 +62,22 @@ int cuda_fail(cudaError_t e) {
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 // Shape/pointer checks shared by every attention entry point.
-int check_common(const void* q, const void* k, const void* v, int B, int H, int N, int d, float scale, int dtype) {
+int check_common(const void* q, const void* k, const void* v, int B, int H, int N, int d, float scale, int dtype,
+                 bool fwd = false) {
   if (!q || !k || !v) return FA_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16)) return FA_ERR_INVALID_ARG;
   if (B < 1 || H < 1 || N < 1 || N > kMaxN) return FA_ERR_INVALID_ARG;
   if (dtype != FA_BF16 && dtype != FA_FP16) return FA_ERR_INVALID_ARG;
   if (!(scale > 0.0f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
-  if (!head_dim_ok(d)) return FA_ERR_UNSUPPORTED;
+  if (!(fwd ? fwd_head_dim_ok(d) : head_dim_ok(d))) return FA_ERR_UNSUPPORTED;
   if ((long long)B * H * N * d > kMaxElems) return FA_ERR_INVALID_ARG;
   return FA_OK;
 }
 
 // [B*H, N, d] view of a [B, H, N, d] tensor: rows past N of a head are out of bounds (zero-filled by TMA),
-// so a ragged last tile never reads the next head.  Box: 128 rows x 64 columns (128 bytes), 128-byte swizzle.
-int make_map(CUtensorMap* m, const void* ptr, int BH, int N, int d, int dtype) {
+// so a ragged last tile never reads the next head.  Box: `box_rows` rows (128, or 32 for the d = 256 V chunks) x
+// 64 columns (128 bytes), 128-byte swizzle.
+int make_map(CUtensorMap* m, const void* ptr, int BH, int N, int d, int dtype, int box_rows = 128) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) {
     t_last_error = "cuTensorMapEncodeTiled unavailable";
@@ -80,7 +85,7 @@ int make_map(CUtensorMap* m, const void* ptr, int BH, int N, int d, int dtype) {
   }
   cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
   cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)N * d * 2};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
   cuuint32_t es[3] = {1, 1, 1};
   CUresult r = enc(m, dtype == FA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
                    const_cast<void*>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -95,7 +100,7 @@ int make_map(CUtensorMap* m, const void* ptr, int BH, int N, int d, int dtype) {
 // {d, H, total} view of a packed [total, H, d] tensor with a {64, 1, 128} box: 128 consecutive tokens of one head,
 // 64 columns (128 bytes), 128-byte swizzle -- the same shared-memory image as the dense box.  Tokens past `total`
 // read as zero.
-int make_map_packed(CUtensorMap* m, const void* ptr, int total, int H, int d, int dtype) {
+int make_map_packed(CUtensorMap* m, const void* ptr, int total, int H, int d, int dtype, int box_rows = 128) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) {
     t_last_error = "cuTensorMapEncodeTiled unavailable";
@@ -103,7 +108,7 @@ int make_map_packed(CUtensorMap* m, const void* ptr, int total, int H, int d, in
   }
   cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)total};
   cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2};
-  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
   cuuint32_t es[3] = {1, 1, 1};
   CUresult r = enc(m, dtype == FA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
                    const_cast<void*>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -177,6 +182,26 @@ cudaError_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
                 : launch_fwd_k<D, BF, T, fa::kModeDense>(mq, mk, mv, a, st);
 }
 
+// d = 256: one CTA per SM, persistent over single Q tiles (see Fwd256Cfg).
+template <bool BF, int P>
+cudaError_t launch_fwd256(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, fa::FwdArgs a,
+                          cudaStream_t st) {
+  using C = fa::Fwd256Cfg;
+  static std::atomic<uint64_t> smem_set{0};
+  cudaError_t e = ensure_smem(fa::fwd256_kernel<BF, P>, C::kSmemBytes, smem_set);
+  if (e != cudaSuccess) return e;
+  a.npairs = a.nT;
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = fa::device_sm_count(dev, &sms)) != cudaSuccess) return e;
+  const long long units = (long long)a.BH * a.npairs * (P == fa::kModeSplit ? a.nsplit : 1);
+  const unsigned grid = (unsigned)std::min<long long>(units, (long long)sms);
+  if ((e = mark(FA_KERNEL_FWD, 0, st)) != cudaSuccess) return e;
+  fa::fwd256_kernel<BF, P><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mk, mv, a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  return mark(FA_KERNEL_FWD, 1, st);
+}
+
 // Q tiles per forward CTA for this call (see FwdCfg).  Measured on B200 (bf16, causal): d = 64 prefers one-tile
 // CTAs (GPT-2 shape 273 vs 242 TFLOP/s, BERT shape 203 vs 188), d = 128 two-tile CTAs (N = 4096/8192/16384:
 // 763/973/1094 vs 671/930/1034).
@@ -198,14 +223,15 @@ int run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, in
             int dtype, cudaStream_t st, const Packed& pk = Packed(), long long list_head_stride = 0) {
   CUtensorMap mq, mk, mv;
   int rc;
+  const int v_rows = d == 256 ? 32 : 128;  // d = 256 streams V in chunks of 32 keys
   if (pk.cu_q) {
     if ((rc = make_map_packed(&mq, q, pk.total_q, H, d, dtype)) != FA_OK) return rc;
     if ((rc = make_map_packed(&mk, k, pk.total_k, H, d, dtype)) != FA_OK) return rc;
-    if ((rc = make_map_packed(&mv, v, pk.total_k, H, d, dtype)) != FA_OK) return rc;
+    if ((rc = make_map_packed(&mv, v, pk.total_k, H, d, dtype, v_rows)) != FA_OK) return rc;
   } else {
     if ((rc = make_map(&mq, q, B * H, N, d, dtype)) != FA_OK) return rc;
     if ((rc = make_map(&mk, k, B * H, N, d, dtype)) != FA_OK) return rc;
-    if ((rc = make_map(&mv, v, B * H, N, d, dtype)) != FA_OK) return rc;
+    if ((rc = make_map(&mv, v, B * H, N, d, dtype, v_rows)) != FA_OK) return rc;
   }
   fa::FwdArgs a;
   a.o = o;
@@ -234,7 +260,14 @@ int run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, in
   a.budget_ns = g_budget_ns.load();
   cudaError_t e;
   const bool bf = dtype == FA_BF16;
-  if (fwd_tiles_for(d) == 2) {
+  if (d == 256) {
+    if (pk.cu_q)
+      e = bf ? launch_fwd256<true, fa::kModePacked>(mq, mk, mv, a, st)
+             : launch_fwd256<false, fa::kModePacked>(mq, mk, mv, a, st);
+    else
+      e = bf ? launch_fwd256<true, fa::kModeDense>(mq, mk, mv, a, st)
+             : launch_fwd256<false, fa::kModeDense>(mq, mk, mv, a, st);
+  } else if (fwd_tiles_for(d) == 2) {
     if (d <= 64)
       e = bf ? launch_fwd<64, true, 2>(mq, mk, mv, a, st) : launch_fwd<64, false, 2>(mq, mk, mv, a, st);
     else
@@ -310,8 +343,8 @@ int splitkv_splits(int B, int H, int Nq, int Nk, int requested) {
   return best;
 }
 
-// Partial results of a split-K/V forward: O rows as wide as the kernel's head dim (64 or 128), then LSE.
-int kernel_dim(int d) { return d <= 64 ? 64 : 128; }
+// Partial results of a split-K/V forward: O rows as wide as the kernel's head dim (64, 128 or 256), then LSE.
+int kernel_dim(int d) { return d <= 64 ? 64 : d <= 128 ? 128 : 256; }
 
 size_t splitkv_bytes(int B, int H, int Nq, int d, int nsplit) {
   const size_t rows = (size_t)nsplit * B * H * ((Nq + fa::kTile - 1) / fa::kTile) * fa::kTile;
@@ -321,7 +354,11 @@ size_t splitkv_bytes(int B, int H, int Nq, int d, int nsplit) {
 template <int D, bool BF>
 cudaError_t launch_splitkv(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, fa::FwdArgs a,
                            void* o, float* lse, cudaStream_t st) {
-  cudaError_t e = launch_fwd_k<D, BF, 1, fa::kModeSplit>(mq, mk, mv, a, st);
+  cudaError_t e;
+  if constexpr (D == 256)
+    e = launch_fwd256<BF, fa::kModeSplit>(mq, mk, mv, a, st);
+  else
+    e = launch_fwd_k<D, BF, 1, fa::kModeSplit>(mq, mk, mv, a, st);
   if (e != cudaSuccess) return e;
   const long long rows = (long long)a.BH * a.N;
   const unsigned blocks = (unsigned)std::min<long long>((rows + 7) / 8, 148LL * 16);
@@ -332,7 +369,7 @@ cudaError_t launch_splitkv(const CUtensorMap& mq, const CUtensorMap& mk, const C
 
 // ------------------------------------------------------------------------------------------ packed batches
 int check_packed(const void* q, const void* k, const void* v, const int32_t* cu_q, const int32_t* cu_k, int B, int H,
-                 int max_q, int max_k, int total_q, int total_k, int d, float scale, int dtype) {
+                 int max_q, int max_k, int total_q, int total_k, int d, float scale, int dtype, bool fwd = false) {
   if (!q || !k || !v || !cu_q || !cu_k) return FA_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(cu_q, 4) || !aligned(cu_k, 4))
     return FA_ERR_INVALID_ARG;
@@ -340,7 +377,7 @@ int check_packed(const void* q, const void* k, const void* v, const int32_t* cu_
   if (total_q < 1 || total_k < 1) return FA_ERR_INVALID_ARG;
   if (dtype != FA_BF16 && dtype != FA_FP16) return FA_ERR_INVALID_ARG;
   if (!(scale > 0.0f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
-  if (!head_dim_ok(d)) return FA_ERR_UNSUPPORTED;
+  if (!(fwd ? fwd_head_dim_ok(d) : head_dim_ok(d))) return FA_ERR_UNSUPPORTED;
   const long long npad = (long long)(max_q + fa::kTile - 1) / fa::kTile * fa::kTile;
   if ((long long)total_q * H * d > kMaxElems || (long long)total_k * H * d > kMaxElems ||
       (long long)B * H * npad * d > kMaxElems)
@@ -368,7 +405,7 @@ const char* fa_last_error_string(void) { return t_last_error.c_str(); }
 
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
            float softmax_scale, int causal, const int32_t* key_lens, int dtype, void* stream) {
-  int rc = check_common(q, k, v, B, H, N, d, softmax_scale, dtype);
+  int rc = check_common(q, k, v, B, H, N, d, softmax_scale, dtype, true);
   if (rc != FA_OK) return rc;
   if (!o || !lse || !aligned(o, 16) || !aligned(lse, 4) || (key_lens && !aligned(key_lens, 4)))
     return FA_ERR_INVALID_ARG;
@@ -384,7 +421,7 @@ size_t fa_blocksparse_workspace_size(int N) {
 int fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
                        float softmax_scale, int causal, const int32_t* key_lens, const uint8_t* block_mask,
                        void* workspace, size_t workspace_bytes, int dtype, void* stream) {
-  int rc = check_common(q, k, v, B, H, N, d, softmax_scale, dtype);
+  int rc = check_common(q, k, v, B, H, N, d, softmax_scale, dtype, true);
   if (rc != FA_OK) return rc;
   if (!o || !lse || !block_mask || !aligned(o, 16) || !aligned(lse, 4) || (key_lens && !aligned(key_lens, 4)))
     return FA_ERR_INVALID_ARG;
@@ -449,7 +486,7 @@ int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* l
                   const int32_t* cu_seqlens_k, int B, int H, int max_seqlen_q, int max_seqlen_k, int total_q,
                   int total_k, int d, float softmax_scale, int causal, int dtype, void* stream) {
   int rc = check_packed(q, k, v, cu_seqlens_q, cu_seqlens_k, B, H, max_seqlen_q, max_seqlen_k, total_q, total_k, d,
-                        softmax_scale, dtype);
+                        softmax_scale, dtype, true);
   if (rc != FA_OK) return rc;
   if (!o || !lse || !aligned(o, 16) || !aligned(lse, 4)) return FA_ERR_INVALID_ARG;
   Packed pk;
@@ -496,7 +533,7 @@ int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, co
 }
 
 size_t fa_fwd_splitkv_workspace_size(int B, int H, int Nq, int Nk, int d, int num_splits) {
-  if (B < 1 || H < 1 || Nq < 1 || Nk < 1 || Nq > kMaxN || Nk > kMaxN || !head_dim_ok(d)) return 0;
+  if (B < 1 || H < 1 || Nq < 1 || Nk < 1 || Nq > kMaxN || Nk > kMaxN || !fwd_head_dim_ok(d)) return 0;
   if (num_splits < 0 || num_splits > kMaxSplits) return 0;
   return splitkv_bytes(B, H, Nq, d, splitkv_splits(B, H, Nq, Nk, num_splits));
 }
@@ -504,7 +541,7 @@ size_t fa_fwd_splitkv_workspace_size(int B, int H, int Nq, int Nk, int d, int nu
 int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq, int Nk,
                    int d, float softmax_scale, int causal, const int32_t* key_lens, int num_splits, void* workspace,
                    size_t workspace_bytes, int dtype, void* stream) {
-  int rc = check_common(q, k, v, B, H, Nk, d, softmax_scale, dtype);
+  int rc = check_common(q, k, v, B, H, Nk, d, softmax_scale, dtype, true);
   if (rc != FA_OK) return rc;
   if (Nq < 1 || Nq > kMaxN || (long long)B * H * Nq * d > kMaxElems) return FA_ERR_INVALID_ARG;
   if (num_splits < 0 || num_splits > kMaxSplits) return FA_ERR_INVALID_ARG;
@@ -516,7 +553,7 @@ int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* 
   CUtensorMap mq, mk, mv;
   if ((rc = make_map(&mq, q, B * H, Nq, d, dtype)) != FA_OK) return rc;
   if ((rc = make_map(&mk, k, B * H, Nk, d, dtype)) != FA_OK) return rc;
-  if ((rc = make_map(&mv, v, B * H, Nk, d, dtype)) != FA_OK) return rc;
+  if ((rc = make_map(&mv, v, B * H, Nk, d, dtype, d == 256 ? 32 : 128)) != FA_OK) return rc;
   fa::FwdArgs a;
   a.o = o;
   a.lse = lse;
@@ -549,9 +586,12 @@ int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* 
   cudaError_t e;
   if (d <= 64)
     e = bf ? launch_splitkv<64, true>(mq, mk, mv, a, o, lse, st) : launch_splitkv<64, false>(mq, mk, mv, a, o, lse, st);
-  else
+  else if (d <= 128)
     e = bf ? launch_splitkv<128, true>(mq, mk, mv, a, o, lse, st)
            : launch_splitkv<128, false>(mq, mk, mv, a, o, lse, st);
+  else
+    e = bf ? launch_splitkv<256, true>(mq, mk, mv, a, o, lse, st)
+           : launch_splitkv<256, false>(mq, mk, mv, a, o, lse, st);
   return e == cudaSuccess ? FA_OK : cuda_fail(e);
 }
 
@@ -564,7 +604,7 @@ int fa_fwd_blocksparse_heads(const void* q, const void* k, const void* v, void* 
                              int d, float softmax_scale, int causal, const int32_t* key_lens,
                              const uint8_t* block_masks, void* workspace, size_t workspace_bytes, int dtype,
                              void* stream) {
-  int rc = check_common(q, k, v, B, H, N, d, softmax_scale, dtype);
+  int rc = check_common(q, k, v, B, H, N, d, softmax_scale, dtype, true);
   if (rc != FA_OK) return rc;
   if (!o || !lse || !block_masks || !aligned(o, 16) || !aligned(lse, 4) || (key_lens && !aligned(key_lens, 4)))
     return FA_ERR_INVALID_ARG;

@@ -55,7 +55,8 @@ A = 1 << 12  # an aligned fake address: only used for calls that must fail valid
     (dict(q=None), _lib.FA_ERR_INVALID_ARG),
     (dict(q=A + 2), _lib.FA_ERR_INVALID_ARG),
     (dict(d=48), _lib.FA_ERR_UNSUPPORTED),
-    (dict(d=256), _lib.FA_ERR_UNSUPPORTED),
+    (dict(d=192), _lib.FA_ERR_UNSUPPORTED),
+    (dict(d=512), _lib.FA_ERR_UNSUPPORTED),
     (dict(N=0), _lib.FA_ERR_INVALID_ARG),
     (dict(N=(1 << 20) + 1), _lib.FA_ERR_INVALID_ARG),
     (dict(B=0), _lib.FA_ERR_INVALID_ARG),
@@ -87,6 +88,15 @@ def test_bwd_and_blocksparse_argument_errors(lib):
     assert rc == _lib.FA_ERR_WORKSPACE
     assert _lib.fa_blockmask_lists(A, 0, A, A, A, A, 0) == _lib.FA_ERR_INVALID_ARG
     assert _lib.fa_blockmask_lists(A, 8193, A, A, A, A, 0) == _lib.FA_ERR_INVALID_ARG
+
+
+def test_head_dim_256_is_forward_only(lib):
+    # d = 256 has a forward kernel; the backward entry points refuse it before any CUDA call
+    rc = _lib.fa_bwd(A, A, A, A, A, A, A, A, A, 1, 1, 128, 256, 0.0625, 0, None, None, A, 1 << 30, 0, 0)
+    assert rc == _lib.FA_ERR_UNSUPPORTED
+    assert _lib.fa_bwd_workspace_size(1, 2, 1024, 256, False) == 0
+    assert _lib.fa_bwd_varlen_workspace_size(1, 2, 1024, 256) == 0
+    assert _lib.fa_fwd_splitkv_workspace_size(1, 2, 1, 4096, 256, 0) > 0
 
 
 def test_budget_and_selftest_argument_errors(lib):

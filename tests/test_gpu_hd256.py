@@ -1,0 +1,102 @@
+"""Head dim 256 on the GPU (forward only: fwd256_kernel, one Q tile per CTA with two score buffers) vs the fp64
+oracle: dense forward with causal masks, key lengths (0 included), ragged tiles, more units than SMs, shared and
+per-head block masks, a packed variable-length batch and the split-K/V decode path.  Tolerance as for the other
+head dims: O and LSE max-abs <= 1e-2.  The backward refuses d = 256 (FA_ERR_UNSUPPORTED)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import exact_io_aware_48_b200 as fa
+from exact_io_aware_48_b200 import _lib, inputs
+from parity import assert_lse_close, assert_o_close, f64, gpu_fwd, log_errors
+
+pytestmark = pytest.mark.gpu
+
+D = 256
+
+DENSE = [
+    # B, H, N, dtype, causal, key_lens
+    (1, 2, 300, "bf16", True, None),
+    (2, 2, 640, "fp16", False, [640, 200]),
+    (1, 3, 1000, "bf16", True, None),
+    (3, 1, 129, "bf16", False, [1, 129, 0]),
+    (2, 16, 1200, "bf16", True, None),        # 320 units: several per CTA
+    (2, 64, 256, "fp16", False, [0, 256]),    # runs of units with no visible key
+]
+
+
+@pytest.mark.parametrize("B,H,N,dtype,causal,kl", DENSE)
+def test_d256_dense_fwd(B, H, N, dtype, causal, kl):
+    q, k, v = [inputs.gaussian((B, H, N, D), 700 + N + t, dtype) for t in range(3)]
+    scale = 1.0 / np.sqrt(D)
+    o, lse = gpu_fwd(q, k, v, causal, scale, key_lens=kl)
+    kla = None if kl is None else np.array(kl, np.int32)
+    ro, rl = oracle.attn_fwd(f64(q), f64(k), f64(v), scale, causal=causal, key_lens=kla)
+    eo = assert_o_close(o.double().numpy(), ro)
+    el = assert_lse_close(lse.numpy(), rl)
+    log_errors(f"d256 B{B} H{H} N{N} {dtype} causal={causal} kl={kl}", O=eo, LSE=el)
+
+
+def test_d256_repeatable():
+    q, k, v = [inputs.gaussian((1, 4, 900, D), 760 + t, "bf16") for t in range(3)]
+    a = gpu_fwd(q, k, v, True, 0.0625)
+    b = gpu_fwd(q, k, v, True, 0.0625)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_d256_block_masks():
+    B, H, N = 1, 2, 640
+    q, k, v = [inputs.gaussian((B, H, N, D), 770 + t, "bf16") for t in range(3)]
+    nT = 5
+    shared = np.tril(np.ones((nT, nT), np.uint8))
+    shared[3, 1] = 0
+    shared[4, 4] = 0
+    o, lse = gpu_fwd(q, k, v, False, 0.07, block_mask=shared)
+    ro, rl = oracle.attn_fwd(f64(q), f64(k), f64(v), 0.07, block_mask=shared)
+    assert_o_close(o.double().numpy(), ro)
+    assert_lse_close(lse.numpy(), rl)
+    heads = np.stack([shared, (np.arange(nT)[:, None] + np.arange(nT)[None, :]) % 2 == 0]).astype(np.uint8)
+    o, lse = gpu_fwd(q, k, v, True, 0.07, block_mask=heads)
+    for h in range(H):
+        ro, rl = oracle.attn_fwd(f64(q[:, h:h + 1]), f64(k[:, h:h + 1]), f64(v[:, h:h + 1]), 0.07, causal=True,
+                                 block_mask=heads[h])
+        assert_o_close(o[:, h:h + 1].double().numpy(), ro)
+        assert_lse_close(lse[:, h:h + 1].numpy(), rl)
+
+
+def test_d256_packed_varlen():
+    lens = [200, 1, 129, 384]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    H = 2
+    q, k, v = [inputs.gaussian((int(cu[-1]), H, D), 780 + t, "bf16") for t in range(3)]
+    cud = torch.as_tensor(cu).cuda()
+    o, lse = fa.attention_fwd_varlen(q.cuda(), k.cuda(), v.cuda(), cud, cud, 384, 384, causal=True)
+    assert fa.last_device_status() == 0
+    ro, rl = oracle.attn_fwd_varlen(f64(q), f64(k), f64(v), cu, cu, 1.0 / np.sqrt(D), causal=True)
+    eo = assert_o_close(o.cpu().double().numpy(), ro)
+    el = assert_lse_close(lse.cpu().numpy(), rl)
+    log_errors("d256 varlen", O=eo, LSE=el)
+
+
+@pytest.mark.parametrize("splits", [0, 3])
+def test_d256_decode(splits):
+    B, H, Nq, Nk = 2, 2, 3, 5000
+    q = inputs.gaussian((B, H, Nq, D), 790, "fp16")
+    k = inputs.gaussian((B, H, Nk, D), 791, "fp16")
+    v = inputs.gaussian((B, H, Nk, D), 792, "fp16")
+    kl = np.array([5000, 777], np.int32)
+    o, lse = fa.attention_fwd_splitkv(q.cuda(), k.cuda(), v.cuda(), causal=True,
+                                      key_lens=torch.as_tensor(kl).cuda(), num_splits=splits)
+    assert fa.last_device_status() == 0
+    ro, rl = oracle.attn_fwd_decode(f64(q), f64(k), f64(v), 1.0 / np.sqrt(D), causal=True, key_lens=kl)
+    eo = assert_o_close(o.cpu().double().numpy(), ro)
+    el = assert_lse_close(lse.cpu().numpy(), rl)
+    log_errors(f"d256 decode splits={splits}", O=eo, LSE=el)
+
+
+def test_d256_backward_is_refused():
+    q, k, v, do = [inputs.gaussian((1, 1, 128, D), 795 + t, "bf16").cuda() for t in range(4)]
+    o, lse = fa.attention_fwd(q, k, v)
+    with pytest.raises(RuntimeError, match="FA_ERR_UNSUPPORTED"):
+        fa.attention_bwd(q, k, v, o, do, lse)
