@@ -9,9 +9,8 @@
 //     (At d <= 128 two Q tiles ping-pong instead; here two O accumulators would not fit.)
 //   * Shared memory holds Q (64 KB) and a ring of ten 16 KB chunks: a K tile arrives as four chunks of 64 head
 //     dims (128 keys each, the K-dimension of Q K^T), a V tile as four chunks of 32 keys (all 256 dims, the
-//     K-dimension of P V, read as an N = 256 operand).  The TMA warp fetches K one tile ahead of V (K_0, K_1,
-//     V_0, K_2, V_1, ...), the order in which the MMA thread consumes them, so K_{j+2} is resident when P_j V_j
-//     has been issued.
+//     K-dimension of P V, read as an N = 256 operand).  The TMA warp fetches K two tiles ahead of V (K_0, K_1,
+//     V_0, K_2, V_1, ...), the order in which the MMA thread consumes them (see the issue order below).
 //
 // Roles (192 threads, one CTA per SM, persistent over 128-row Q tiles ordered longest first):
 //   warps 0-3  softmax and epilogue: thread = query row = TMEM lane, whole rows, no shuffles;
@@ -66,6 +65,38 @@ struct StepWalker {
     }
   }
 };
+
+// The same stream one step ahead: the caller can see whether the next step opens a unit (ok_nx, fresh_nx) and
+// whether the step it takes closes one (`last`).  u is the unit of the step last returned.
+template <int kMode>
+struct LookaheadWalker {
+  StepWalker<kMode> w;
+  FwdUnit u, u_nx;
+  bool ok_nx, fresh_nx;
+  int j_nx;
+  __device__ __forceinline__ void init(int total_units, const FwdArgs& a) {
+    w.init(total_units);
+    ok_nx = w.next(a, j_nx, fresh_nx);
+    u_nx = w.u;
+  }
+  __device__ __forceinline__ bool next(const FwdArgs& a, int& j, bool& fresh, bool& last) {
+    if (!ok_nx) return false;
+    j = j_nx;
+    fresh = fresh_nx;
+    u = u_nx;
+    ok_nx = w.next(a, j_nx, fresh_nx);
+    u_nx = w.u;
+    last = !ok_nx || fresh_nx;
+    return true;
+  }
+};
+
+// Issue order shared by the TMA and MMA roles (ring chunks are consumed in the order they are produced):
+//   S (or K) runs two steps ahead of P V (or V): after P_j V_j comes S_{j+2};
+//   except that a unit's first S waits until every P V of the previous unit has been issued -- it waits for the
+//   new Q, and the previous unit's last P V (and so its epilogue) must not wait behind that.
+// So across a unit boundary the order is ..., P V_{n-2}, P V_{n-1}, S_n, S_{n+1}, P V_n, S_{n+2}, ...
+// The Q buffer is released right after a unit's last S, one step before the next unit's first S is due.
 
 template <bool kBF16, int kMode>
 __global__ void __launch_bounds__(Fwd256Cfg::kThreads, 1)
@@ -125,11 +156,13 @@ __global__ void __launch_bounds__(Fwd256Cfg::kThreads, 1)
       ptx::prefetch_tensormap(&map_k);
       ptx::prefetch_tensormap(&map_v);
       const uint32_t bq = ptx::smem_addr(&bar_q);
-      StepWalker<kMode> kw, vw;
-      kw.init(total_units);
+      LookaheadWalker<kMode> kw;
+      StepWalker<kMode> vw;
+      kw.init(total_units, args);
       vw.init(total_units);
       int n = 0, nq = 0;  // ring chunks issued, Q tiles issued
-      bool ok = true, kdone = false;
+      int kc = 0, vc = 0;  // K tiles and V tiles issued
+      bool ok = true;
       // next free ring slot (waits for its previous chunk to be consumed); arms its full barrier
       auto slot = [&](uint32_t& dst, uint32_t& bf) -> bool {
         const int s = n % NS;
@@ -144,11 +177,9 @@ __global__ void __launch_bounds__(Fwd256Cfg::kThreads, 1)
       // K of the next step (and that unit's Q first when the step opens a unit)
       auto load_k = [&]() -> bool {
         int j;
-        bool fresh;
-        if (!kw.next(args, j, fresh)) {
-          kdone = true;
-          return true;
-        }
+        bool fresh, last;
+        if (!kw.next(args, j, fresh, last)) return true;
+        ++kc;
         const FwdUnit& u = kw.u;
         if (fresh) {
           // the Q buffer is free once every S MMA of the previous unit has completed
@@ -166,19 +197,28 @@ __global__ void __launch_bounds__(Fwd256Cfg::kThreads, 1)
         }
         return true;
       };
-      ok = load_k();
+      // K tiles up to two steps ahead of V; a unit's first K only once every V before it is issued
+      auto top_up = [&]() -> bool {
+        while (kc < vc + 2 && kw.ok_nx) {
+          if (kw.fresh_nx && kc != vc) break;
+          if (!load_k()) return false;
+        }
+        return true;
+      };
+      ok = top_up();
       while (ok) {
-        if (!kdone && !(ok = load_k())) break;
         int j;
         bool fresh;
         if (!vw.next(args, j, fresh)) break;
         const FwdUnit& u = vw.u;
-        for (int kc = 0; kc < C::kChunks && ok; ++kc) {  // chunk kc: keys [32kc, 32kc+32), four 64-dim boxes
+        for (int c = 0; c < C::kChunks && ok; ++c) {  // chunk c: keys [32c, 32c+32), four 64-dim boxes
           uint32_t dst, bf;
           if (!(ok = slot(dst, bf))) break;
           for (int cb = 0; cb < D / 64; ++cb)
-            tma_rows(dst + cb * 4096, &map_v, cb, j * kTile + 32 * kc, u.g.k0, u.bh, u.h, packed, bf);
+            tma_rows(dst + cb * 4096, &map_v, cb, j * kTile + 32 * c, u.g.k0, u.bh, u.h, packed, bf);
         }
+        ++vc;
+        if (ok) ok = top_up();
       }
       // Let every copy this thread issued land before the CTA can exit (immediate in the normal path).
       if (nq > 0) ptx::mbar_wait(bq, (nq - 1) & 1, args.budget_ns);
@@ -204,15 +244,14 @@ __global__ void __launch_bounds__(Fwd256Cfg::kThreads, 1)
         ptx::tc_fence_after();
         return true;
       };
-      StepWalker<kMode> sw;
-      sw.init(total_units);
+      LookaheadWalker<kMode> sw;
+      sw.init(total_units, args);
       // S_b = Q K_j^T for the next step of the stream (b = its parity); nothing when the stream is over
       auto issue_next_s = [&]() -> bool {
         int j;
-        bool fresh;
-        if (!sw.next(args, j, fresh)) return true;
+        bool fresh, last;
+        if (!sw.next(args, j, fresh, last)) return true;
         if (fresh) {
-          if (nq > 0) ptx::mma_commit(ptx::smem_addr(&bar_q_free));  // every S of the previous unit issued
           if (!wait_or_abort(ptx::smem_addr(&bar_q), nq & 1, args.budget_ns, abortp)) return false;
           ptx::tc_fence_after();
           ++nq;
@@ -230,11 +269,20 @@ __global__ void __launch_bounds__(Fwd256Cfg::kThreads, 1)
           ptx::mma_commit(ptx::smem_addr(&bar_empty[s]));
         }
         ptx::mma_commit(ptx::smem_addr(&bar_s[gs & 1]));
+        if (last) ptx::mma_commit(ptx::smem_addr(&bar_q_free));  // every S of this unit issued
         ++gs;
         return true;
       };
-      ok = issue_next_s() && issue_next_s();
       int gp = 0, ku = 0;  // P V steps issued, units finished
+      // S up to two steps ahead of P V; a unit's first S only at a unit end (allow_fresh) with every P V issued
+      auto top_up = [&](bool allow_fresh) -> bool {
+        while (gs < gp + 2 && sw.ok_nx) {
+          if (sw.fresh_nx && !(allow_fresh && gs == gp)) break;
+          if (!issue_next_s()) return false;
+        }
+        return true;
+      };
+      ok = top_up(true);
       UnitSeq us;
       us.init(total_units);
       int L;
@@ -265,7 +313,7 @@ __global__ void __launch_bounds__(Fwd256Cfg::kThreads, 1)
           ptx::mma_commit(ptx::smem_addr(&bar_pv));
           ++gp;
           ++li;
-          ok = issue_next_s();  // two steps ahead of this P V; its buffer's P was read by the P V just issued
+          ok = top_up(false);  // S two steps ahead; its buffer's P was read by the P V just issued
         }
         if (!ok) break;
         // a unit with no P V waits for the previous epilogue here, so bar_o never runs two phases ahead
@@ -274,6 +322,7 @@ __global__ void __launch_bounds__(Fwd256Cfg::kThreads, 1)
           break;
         ptx::mma_commit(ptx::smem_addr(&bar_o));
         ++ku;
+        ok = top_up(true);  // the next unit's first S (and the one after)
       }
       // No MMA may still be running when the tensor memory is released.
       ptx::mma_commit(ptx::smem_addr(&bar_drain));
