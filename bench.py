@@ -374,6 +374,34 @@ def measure_decode(stream, flush, hbm_gbs):
             "bytes": nbytes, "gbs": round(gbs, 1), "hbm_frac": round(gbs / hbm_gbs, 4) if hbm_gbs else None}
 
 
+def measure_d256(stream, flush, peak):
+    """Head dim 256 forward (its own kernel; no backward at d = 256): B1 H16 N8192 bf16 causal, the long-context
+    shape at twice the head dim.  TFLOP/s by the algorithmic convention (4*d per visible pair)."""
+    import torch
+    from exact_io_aware_48_b200 import _lib, inputs
+    B, H, N, d = 1, 16, 8192, 256
+    q, k, v = [inputs.gaussian((B, H, N, d), 510 + t, "bf16").cuda() for t in range(3)]
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), device="cuda", dtype=torch.float32)
+    scale = 1.0 / math.sqrt(d)
+
+    def step(st):
+        rc = _lib.fa_fwd(q, k, v, o, lse, B, H, N, d, scale, True, None, _lib.FA_BF16, st)
+        if rc:
+            raise RuntimeError(f"fa_fwd: {_lib.fa_status_string(rc)}")
+
+    for _ in range(3):
+        step(stream)
+    ms, _ = time_loop(step, 10, stream, flush)
+    status = _lib.fa_last_device_status(stream)
+    if status:
+        raise RuntimeError(f"d = 256 forward reported {_lib.fa_status_string(status)}")
+    t = statistics.median(ms)
+    tf = 4 * d * B * H * (N * (N + 1) // 2) / t / 1e9
+    return {"workload": f"fwd B{B} H{H} N{N} d{d} bf16 causal", "ms": round(t, 4), "tflops": round(tf, 1),
+            "frac": round(tf / peak, 4) if peak else None}
+
+
 def run_ours(args):
     import numpy as np
     import torch
@@ -438,6 +466,7 @@ def run_ours(args):
     targets = measure_targets(stream, flush, peak) if (args.targets and rank == 0) else None
     varlen = measure_varlen(stream, flush, peak) if (args.targets and rank == 0) else None
     decode = measure_decode(stream, flush, hbm) if (args.targets and rank == 0) else None
+    d256 = measure_d256(stream, flush, peak) if (args.targets and rank == 0) else None
     cpu = cpu_baseline(p.w) if rank == 0 and world == 1 and args.cpu_baseline else None
 
     if rank == 0:
@@ -460,6 +489,7 @@ def run_ours(args):
             "targets": targets,
             "varlen": varlen,
             "decode": decode,
+            "d256": d256,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)

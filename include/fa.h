@@ -20,8 +20,9 @@
  *               Scratch that a call needs is passed in as `workspace` (device memory, 256-byte aligned) of at
  *               least the size returned by the matching *_workspace_size query.
  *   Shapes      B >= 1, H >= 1, 1 <= N <= 1048576 (2^20), d in {32, 64, 96, 128} (32 and 96 run on the 64 and 128
- *               kernels with the extra columns zero, at their cost), B*H*N*d <= 2^34, softmax_scale finite
- *               and > 0.
+ *               kernels with the extra columns zero, at their cost); the forward calls (fa_fwd, fa_fwd_blocksparse,
+ *               fa_fwd_blocksparse_heads, fa_fwd_varlen, fa_fwd_splitkv) also take d = 256, the backward calls do
+ *               not (FA_ERR_UNSUPPORTED).  B*H*N*d <= 2^34, softmax_scale finite and > 0.
  *   Execution   Asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).  Inputs must stay valid
  *               until the stream reaches the work.
  *   Errors      Argument errors are detected on the host before anything is launched and returned as an
@@ -43,7 +44,7 @@ extern "C" {
 typedef enum {
   FA_OK = 0,
   FA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad shape, scale <= 0, bad dtype */
-  FA_ERR_UNSUPPORTED = 2, /* head dimension other than 32, 64, 96 or 128 */
+  FA_ERR_UNSUPPORTED = 2, /* head dimension other than 32, 64, 96, 128 (or 256 for the forward calls) */
   FA_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed (message: fa_last_error_string) */
   FA_ERR_TIMEOUT = 4,     /* a kernel wait ran out of its time budget (device-detected) */
   FA_ERR_WORKSPACE = 5    /* workspace missing, misaligned or smaller than the query says */
