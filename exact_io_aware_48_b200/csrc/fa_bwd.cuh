@@ -263,7 +263,8 @@ __global__ void __launch_bounds__(512, 1)
   auto sV = [&](int kb) { return sKV + kb * 2 * C::kTileBytes + C::kTileBytes; };
 
   __shared__ __align__(8) uint64_t bar_kv[KB], bar_kv_free[KB], bar_full[NS], bar_empty[NS], bar_s, bar_dp, bar_p,
-      bar_ds, bar_dq_full, bar_dq_free, bar_ds_free, bar_pt_free, bar_done, bar_acc_free, bar_drain;
+      bar_ds, bar_dq_full, bar_dq_free, bar_ds_free, bar_pt_free, bar_dv_done, bar_done, bar_dv_free, bar_dk_free,
+      bar_drain;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
   volatile int* abortp = &abort_flag;
@@ -294,8 +295,10 @@ __global__ void __launch_bounds__(512, 1)
     ptx::mbar_init(ptx::smem_addr(&bar_dq_free), 128);
     ptx::mbar_init(ptx::smem_addr(&bar_ds_free), 1);
     ptx::mbar_init(ptx::smem_addr(&bar_pt_free), 1);
+    ptx::mbar_init(ptx::smem_addr(&bar_dv_done), 1);
     ptx::mbar_init(ptx::smem_addr(&bar_done), 1);
-    ptx::mbar_init(ptx::smem_addr(&bar_acc_free), 128);
+    ptx::mbar_init(ptx::smem_addr(&bar_dv_free), 128);
+    ptx::mbar_init(ptx::smem_addr(&bar_dk_free), 128);
     ptx::mbar_init(ptx::smem_addr(&bar_drain), 1);
     abort_flag = 0;
     ptx::fence_barrier_init();
@@ -452,10 +455,11 @@ __global__ void __launch_bounds__(512, 1)
         dk_k = ptx::sw128_desc(ptx::smem_addr(sK(kb)), 16, 1024);
         dk_mn = ptx::sw128_desc(ptx::smem_addr(sK(kb)), 16384, 1024);
         dv_k = ptx::sw128_desc(ptx::smem_addr(sV(kb)), 16, 1024);
-        // dV and dK start over in TMEM: the epilogue must have read the previous unit's
-        auto acc_ready = [&]() -> bool {
+        // dV and dK start over in TMEM: the epilogue must have read the previous unit's (dV and dK are released
+        // separately: dV as soon as the previous unit's last dV MMA is done, so this unit's first dV rarely waits)
+        auto acc_ready = [&](uint64_t& bar_free) -> bool {
           if (ku == 0) return true;
-          if (!wait_or_abort(ptx::smem_addr(&bar_acc_free), (ku - 1) & 1, args.budget_ns, abortp)) return false;
+          if (!wait_or_abort(ptx::smem_addr(&bar_free), (ku - 1) & 1, args.budget_ns, abortp)) return false;
           ptx::tc_fence_after();
           return true;
         };
@@ -477,12 +481,14 @@ __global__ void __launch_bounds__(512, 1)
             int inext;
             const bool have_next = it.next(inext);
             if (have_next && !(ok = issue_s(kq + 2))) break;
-            if (li == 0 && !(ok = acc_ready())) break;
+            if (li == 0 && !(ok = acc_ready(bar_dv_free))) break;
             issue_dv(ko, li == 0);
             ptx::mma_commit(ptx::smem_addr(&bar_pt_free));
+            if (!have_next) ptx::mma_commit(ptx::smem_addr(&bar_dv_done));  // this unit's dV is final
             if (!(ok = wait_or_abort(ptx::smem_addr(&bar_ds), ph, args.budget_ns, abortp))) break;
             ptx::tc_fence_after();
             if (have_next && !(ok = issue_dp(ko + 2))) break;
+            if (li == 0 && !(ok = acc_ready(bar_dk_free))) break;
             issue_dk(kq, li == 0);
             if (gi > 0 && !(ok = wait_or_abort(ptx::smem_addr(&bar_dq_free), ph_prev, args.budget_ns, abortp)))
               break;
@@ -508,14 +514,16 @@ __global__ void __launch_bounds__(512, 1)
             if (!(ok = issue_dp(ko))) break;
             if (!(ok = wait_or_abort(ptx::smem_addr(&bar_p), ph, args.budget_ns, abortp))) break;
             ptx::tc_fence_after();
-            if (li == 0 && !(ok = acc_ready())) break;
+            if (li == 0 && !(ok = acc_ready(bar_dv_free))) break;
             issue_dv(ko, li == 0);
             int inext;
             const bool have_next = it.next(inext);
+            if (!have_next) ptx::mma_commit(ptx::smem_addr(&bar_dv_done));  // this unit's dV is final
             if (have_next && !(ok = issue_s(kq + 2))) break;
             if (!(ok = wait_or_abort(ptx::smem_addr(&bar_ds), ph, args.budget_ns, abortp))) break;
             ptx::tc_fence_after();
             issue_dq();
+            if (li == 0 && !(ok = acc_ready(bar_dk_free))) break;
             issue_dk(kq, li == 0);
             ptx::mma_commit(ptx::smem_addr(&bar_ds_free));
             ++gi;
@@ -525,7 +533,7 @@ __global__ void __launch_bounds__(512, 1)
           }
         }
         if (!ok) break;
-        ptx::mma_commit(ptx::smem_addr(&bar_done));        // dK, dV of this unit are final
+        ptx::mma_commit(ptx::smem_addr(&bar_done));        // dK of this unit is final (and every MMA before it)
         ptx::mma_commit(ptx::smem_addr(&bar_kv_free[kb]));  // K_j, V_j no longer read
         ++ku;
       }
@@ -648,8 +656,9 @@ __global__ void __launch_bounds__(512, 1)
     // its staging buffer in the 128-byte-swizzled layout of the dq_acc tensor map (16-byte chunk k of row r lands at
     // k ^ (r % 8): conflict-free), then one lane issues a TMA reduce-add of that box into dq_acc.  The TMEM region
     // is released as soon as the last columns are in registers.
-    // dK, dV epilogue: after a unit's last MMA each warp reads its 32 key rows of dV and dK (dK already carries
-    // the softmax scale through dS), releases the accumulators to the next unit, and stores them 16-bit.
+    // dK, dV epilogue: each warp reads its 32 key rows of dV as soon as the unit's last dV MMA is done (before the
+    // last dQ drain) and of dK after the unit's last MMA (dK already carries the softmax scale through dS), releases
+    // each accumulator to the next unit as soon as it is read, and stores them 16-bit.
     const int wq = warp - kWarpDrain;
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
     uint8_t* stage = sStage + wq * 4096;
@@ -662,8 +671,49 @@ __global__ void __launch_bounds__(512, 1)
       it.init(args.col_ptr ? args.col_ptr + u.h * args.list_head_stride : nullptr,
                 args.row_idx + u.h * args.list_head_stride, u.j, u.nTq, causal ? u.j : 0, u.visible);
       const int n_iters = it.count();
-      int i;
+      const int gc = u.j * kTile + wq * 32 + lane;  // key row of this lane in the dK, dV epilogue
+      // dense: every row of the head (keys past a key length get zero); packed: the sequence's own keys only
+      const bool row_ok = packed ? gc < u.g.lk : gc < args.N;
+      const size_t krow = packed ? (size_t)(u.g.k0 + gc) * args.H + u.h : (size_t)u.bh * args.N + gc;
+      // dV (is_dk false) or dK of this unit: read out of TMEM chunk by chunk, release the columns to the next unit
+      // after the last read, store 16-bit; a unit with no visible query writes zeros
+      auto epilogue = [&](bool is_dk) {
+        uint8_t* row = reinterpret_cast<uint8_t*>(is_dk ? args.dk : args.dv) + krow * args.dl * 2;
+#pragma unroll 1
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t r[32];
+          if (n_iters > 0) {
+            ptx::tmem_ld32(tmem + lane_base + (is_dk ? C::kColDK : C::kColDV) + cc * 32, r);
+            ptx::tmem_ld_wait();
+            if (cc == D / 32 - 1) {
+              ptx::tc_fence_before();
+              ptx::mbar_arrive(ptx::smem_addr(is_dk ? &bar_dk_free : &bar_dv_free));
+            }
+          } else {
+#pragma unroll
+            for (int v = 0; v < 32; ++v) r[v] = 0u;  // no visible query: zero gradient
+          }
+          uint32_t pkd[16];
+#pragma unroll
+          for (int v = 0; v < 16; ++v)
+            pkd[v] = ptx::pack2<kBF16>(__uint_as_float(r[2 * v]), __uint_as_float(r[2 * v + 1]));
+          if (row_ok && cc * 32 < args.dl) {
+            uint4* dst = reinterpret_cast<uint4*>(row + cc * 64);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              dst[v] = make_uint4(pkd[4 * v], pkd[4 * v + 1], pkd[4 * v + 2], pkd[4 * v + 3]);
+          }
+        }
+      };
+      int i, it_idx = 0;
       while (it.next(i)) {
+        if (it_idx++ == n_iters - 1) {
+          // the unit's last dV MMA precedes its last dQ: take dV out first, so the next unit's dV can start
+          ok = __all_sync(0xffffffffu, wait_or_abort(ptx::smem_addr(&bar_dv_done), ku & 1, args.budget_ns, abortp));
+          if (!ok) break;
+          ptx::tc_fence_after();
+          epilogue(false);
+        }
         ok = __all_sync(0xffffffffu, wait_or_abort(ptx::smem_addr(&bar_dq_full), gi & 1, args.budget_ns, abortp));
         if (!ok) break;
         ptx::tc_fence_after();
@@ -710,43 +760,15 @@ __global__ void __launch_bounds__(512, 1)
         ++gi;
       }
       if (!ok) break;
-      // ---- dK, dV epilogue of this unit
-      const int gc = u.j * kTile + wq * 32 + lane;  // key row
-      // dense: every row of the head (keys past a key length get zero); packed: the sequence's own keys only
-      const bool row_ok = packed ? gc < u.g.lk : gc < args.N;
-      const size_t krow = packed ? (size_t)(u.g.k0 + gc) * args.H + u.h : (size_t)u.bh * args.N + gc;
-      uint8_t* dv_row = reinterpret_cast<uint8_t*>(args.dv) + krow * args.dl * 2;
-      uint8_t* dk_row = reinterpret_cast<uint8_t*>(args.dk) + krow * args.dl * 2;
+      // ---- dK of this unit (dV went out before the last dQ), or zeros for both when no query sees the keys
       if (n_iters > 0) {
         ok = __all_sync(0xffffffffu, wait_or_abort(ptx::smem_addr(&bar_done), ku & 1, args.budget_ns, abortp));
         if (!ok) break;
         ptx::tc_fence_after();
+      } else {
+        epilogue(false);
       }
-#pragma unroll 1
-      for (int ch = 0; ch < 2 * (D / 32); ++ch) {  // chunks of 32 columns: dV then dK
-        const bool is_dk = ch >= D / 32;
-        const int cc = is_dk ? ch - D / 32 : ch;
-        uint32_t r[32];
-        if (n_iters > 0) {
-          ptx::tmem_ld32(tmem + lane_base + (is_dk ? C::kColDK : C::kColDV) + cc * 32, r);
-          ptx::tmem_ld_wait();
-          if (ch == 2 * (D / 32) - 1) {
-            ptx::tc_fence_before();
-            ptx::mbar_arrive(ptx::smem_addr(&bar_acc_free));  // the next unit may overwrite dK, dV
-          }
-        } else {
-#pragma unroll
-          for (int v = 0; v < 32; ++v) r[v] = 0u;  // no visible query: zero gradient
-        }
-        uint32_t pkd[16];
-#pragma unroll
-        for (int v = 0; v < 16; ++v) pkd[v] = ptx::pack2<kBF16>(__uint_as_float(r[2 * v]), __uint_as_float(r[2 * v + 1]));
-        if (row_ok && cc * 32 < args.dl) {
-          uint4* dst = reinterpret_cast<uint4*>((is_dk ? dk_row : dv_row) + cc * 64);
-#pragma unroll
-          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pkd[4 * v], pkd[4 * v + 1], pkd[4 * v + 2], pkd[4 * v + 3]);
-        }
-      }
+      epilogue(true);
       if (n_iters > 0) ++ku;
     }
     if (lane == 0) ptx::bulk_wait_group<0>();  // all reductions performed before the CTA retires
