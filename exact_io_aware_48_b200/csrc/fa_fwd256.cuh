@@ -4,9 +4,9 @@
 // stream past a resident 128-row Q tile, the running max and denominator stay on chip, O and the per-row
 // logsumexp are the only outputs.  What changes at d = 256 is the fit on the SM:
 //   * TMEM (512 columns) holds one Q tile's O (256 columns) and TWO score buffers S_0, S_1 (128 columns each),
-//     so the score MMA of K/V tile j+2 is issued as soon as P_j V_j is, while the softmax warps work on tile j+1:
-//     the tensor core never waits for a softmax, and the softmax warps find every S finished when they get to it.
-//     (At d <= 128 two Q tiles ping-pong instead; here two O accumulators would not fit.)
+//     so the score MMA of K/V tile j+2 is issued as soon as P_j V_j is and runs while the softmax warps work on
+//     tile j+1: within one Q tile the softmax and the tensor core overlap, and S is normally complete before the
+//     softmax warps get to it.  (At d <= 128 two Q tiles ping-pong instead; here two O accumulators would not fit.)
 //   * Shared memory holds Q (64 KB) and a ring of ten 16 KB chunks: a K tile arrives as four chunks of 64 head
 //     dims (128 keys each, the K-dimension of Q K^T), a V tile as four chunks of 32 keys (all 256 dims, the
 //     K-dimension of P V, read as an N = 256 operand).  The TMA warp fetches K two tiles ahead of V (K_0, K_1,
