@@ -8,6 +8,7 @@
 #include <string>
 
 #include "fa.h"
+#include "fa_abi_checks.h"
 #include "fa_common.cuh"
 #include "fa_fwd.cuh"
 #include "fa_fwd256.cuh"
@@ -385,6 +386,20 @@ int check_packed(const void* q, const void* k, const void* v, const int32_t* cu_
   return FA_OK;
 }
 
+int fa_abi::bwd_check_args(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                           const float* lse, const void* dq, const void* dk, const void* dv, int B, int H, int N, int d,
+                           float softmax_scale, const int32_t* key_lens, const uint8_t* block_mask, int dtype) {
+  int rc = check_common(q, k, v, B, H, N, d, softmax_scale, dtype);
+  if (rc != FA_OK) return rc;
+  if (!o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  if (!aligned(o, 16) || !aligned(dout, 16) || !aligned(lse, 4) || !aligned(dq, 16) || !aligned(dk, 16) ||
+      !aligned(dv, 16) || (key_lens && !aligned(key_lens, 4)))
+    return FA_ERR_INVALID_ARG;
+  const int nT = (N + fa::kTile - 1) / fa::kTile;
+  if (block_mask && nT > fa::kMaxMaskTiles) return FA_ERR_INVALID_ARG;
+  return FA_OK;
+}
+
 extern "C" {
 
 int fa_version(void) { return kVersion; }
@@ -444,6 +459,7 @@ int fa_blockmask_lists(const uint8_t* mask, int nT, int32_t* row_ptr, int32_t* c
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d, int has_block_mask) {
   if (B < 1 || H < 1 || N < 1 || N > kMaxN || !head_dim_ok(d)) return 0;
+  if ((long long)B * H * N * d > kMaxElems) return 0;  // B*H stays far below 2^31 after this check
   const int nT = (N + fa::kTile - 1) / fa::kTile;
   return fa::bwd_workspace_bytes(B * H, nT, d) + (has_block_mask ? lists_bytes(nT) : 0);
 }
@@ -451,14 +467,10 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d, int has_block_mask) {
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse, void* dq,
            void* dk, void* dv, int B, int H, int N, int d, float softmax_scale, int causal, const int32_t* key_lens,
            const uint8_t* block_mask, void* workspace, size_t workspace_bytes, int dtype, void* stream) {
-  int rc = check_common(q, k, v, B, H, N, d, softmax_scale, dtype);
+  int rc = fa_abi::bwd_check_args(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, softmax_scale, key_lens, block_mask,
+                                  dtype);
   if (rc != FA_OK) return rc;
-  if (!o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
-  if (!aligned(o, 16) || !aligned(dout, 16) || !aligned(lse, 4) || !aligned(dq, 16) || !aligned(dk, 16) ||
-      !aligned(dv, 16) || (key_lens && !aligned(key_lens, 4)))
-    return FA_ERR_INVALID_ARG;
   const int nT = (N + fa::kTile - 1) / fa::kTile;
-  if (block_mask && nT > fa::kMaxMaskTiles) return FA_ERR_INVALID_ARG;
   const size_t need = fa_bwd_workspace_size(B, H, N, d, block_mask != nullptr);
   if (!workspace || !aligned(workspace, 256) || workspace_bytes < need) return FA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -62,9 +62,11 @@ const char* fa_status_string(int status);
 const char* fa_last_error_string(void);
 
 /*
- * Forward (review page "Method"; slide deck "Executable shape"): each CTA owns two 128-row Q tiles, streams the
- * visible 128-key K/V tiles through shared memory, keeps the running max and denominator per row on chip and
- * writes only O and LSE.  Tiles that the causal mask or the key lengths hide entirely are never loaded.
+ * Forward (review page "Method"; slide deck "Executable shape"): persistent CTAs each take 128-row Q tiles (two
+ * tiles that alternate on the tensor core per CTA at d = 96 / 128, one tile per CTA and two CTAs per SM at d <= 64,
+ * one tile per CTA at d = 256), stream the visible 128-key K/V tiles through shared memory, keep the running max
+ * and denominator per row on chip and write only O and LSE.  Tiles that the causal mask or the key lengths hide
+ * entirely are never loaded.
  *   q, k, v   in   [B,H,N,d]     o   out [B,H,N,d]     lse  out [B,H,N] fp32 (natural log)
  *   causal    nonzero: key c visible from row r only if c <= r
  *   key_lens  optional [B] int32 device array (NULL: every key visible)
@@ -217,8 +219,10 @@ int fa_set_fwd_tiles_per_cta(int tiles);
  */
 int fa_selftest_exp2(const float* x, float* out_fma, float* out_mufu, int n, void* stream);
 
-/* Size of the fixed device scratch array behind fa_bwd_noalloc: 32 MiB, held by every GPU that loads the library
- * until the process exits. */
+/* Size of the fixed device scratch array behind fa_bwd_noalloc: 32 MiB of device memory on every GPU whose context
+ * loads the array's module, held until that context is destroyed (normally process exit).  With lazy module loading
+ * (the CUDA 12 default) the module is loaded by the first fa_bwd_noalloc call on a device; with eager loading
+ * (CUDA_MODULE_LOADING=EAGER) when the context is created, whether or not fa_bwd_noalloc is ever called. */
 #define FA_NOALLOC_SCRATCH_BYTES (32u << 20)
 
 /*
@@ -231,7 +235,12 @@ int fa_selftest_exp2(const float* x, float* out_fma, float* out_mufu, int n, voi
  *   Size limit  problems whose fa_bwd_workspace_size() exceeds FA_NOALLOC_SCRATCH_BYTES are rejected with
  *               FA_ERR_WORKSPACE before anything is launched (e.g. B*H = 96, N = 1024, d = 64 needs 24.75 MiB: fits).
  *   Set-up      the first call on a device looks up the array's device address (cudaGetSymbolAddress) with that
- *               device current; make that first call before any stream capture.
+ *               device current; make that first call before any stream capture.  The address is cached per device
+ *               together with the id of the context it belongs to: after cudaDeviceReset (a new context, in which
+ *               the array may have moved) the next call looks it up again, so that call, too, must not be the
+ *               first one made inside a capture.
+ *   Checks      the same argument checks as fa_bwd, in the same order and with the same status codes; only then
+ *               is the size limit applied.
  *   Sharing     every call on a device uses the same array and it keeps the last call's contents (each call
  *               rewrites what it reads, including zeroing its dQ accumulator).  Calls that overlap on the GPU (on
  *               different streams, or from different host threads without ordering) race on the array.

@@ -76,6 +76,17 @@ def assert_grad_close(got, ref, name, tol=GRAD_REL_TOL):
     return err / scale
 
 
+def sampled_keys(seed, BH, N, heads, per_head):
+    """`per_head` distinct seeded keys in each of `heads` distinct seeded heads: (head index, key index) arrays."""
+    hb, _ = inputs.sample_rows(seed, BH, 1, heads)
+    kb, kc = [], []
+    for t, h in enumerate(hb.tolist()):
+        _, c = inputs.sample_rows(seed + 1 + t, 1, N, per_head)
+        kb.append(np.full_like(c, h))
+        kc.append(c)
+    return np.concatenate(kb), np.concatenate(kc)
+
+
 def log_errors(name, **errs):
     """Append measured parity errors (for margins) to $FA_PARITY_LOG if set."""
     path = os.environ.get("FA_PARITY_LOG")

@@ -103,3 +103,29 @@ def test_budget_and_selftest_argument_errors(lib):
     assert _lib.fa_set_wait_budget_ns(10) == _lib.FA_ERR_INVALID_ARG
     assert _lib.fa_selftest_wait_timeout(10, 0) == _lib.FA_ERR_INVALID_ARG
     assert _lib.fa_selftest_wait_timeout(2_000_000_000, 0) == _lib.FA_ERR_INVALID_ARG
+
+
+def test_noalloc_reports_the_same_status_as_fa_bwd(lib):
+    # fa_bwd_noalloc runs fa_bwd's argument checks first, so a bad argument gets the same status from both; only a
+    # valid problem too large for the fixed array gets FA_ERR_WORKSPACE.  No CUDA call is reached in these cases.
+    big = dict(B=8, H=64, N=1024, d=128)  # needs ~260 MiB of scratch
+    cases = [
+        (dict(q=None, **big), _lib.FA_ERR_INVALID_ARG),
+        (dict(dq=A + 8, **big), _lib.FA_ERR_INVALID_ARG),
+        (dict(B=8, H=64, N=(1 << 20) + 1, d=48), _lib.FA_ERR_INVALID_ARG),
+        (dict(B=8, H=64, N=1024, d=48), _lib.FA_ERR_UNSUPPORTED),
+        (dict(B=1 << 20, H=1 << 12, N=1024, d=64), _lib.FA_ERR_INVALID_ARG),  # B*H*N*d far beyond 2^34
+        (dict(scale=0.0, **big), _lib.FA_ERR_INVALID_ARG),
+        (big, _lib.FA_ERR_WORKSPACE),
+    ]
+    for args, expect in cases:
+        a = dict(q=A, dq=A, B=1, H=1, N=128, d=64, scale=0.125)
+        a.update(args)
+        rc = _lib.fa_bwd_noalloc(a["q"], A, A, A, A, A, a["dq"], A, A, a["B"], a["H"], a["N"], a["d"], a["scale"], 0,
+                                 None, None, 0, 0)
+        assert rc == expect, (args, rc)
+        if expect != _lib.FA_ERR_WORKSPACE:  # fa_bwd reports the same (with a workspace far too small)
+            rc2 = _lib.fa_bwd(a["q"], A, A, A, A, A, a["dq"], A, A, a["B"], a["H"], a["N"], a["d"], a["scale"], 0,
+                              None, None, A, 16, 0, 0)
+            assert rc2 == expect, (args, rc2)
+    assert _lib.fa_bwd_workspace_size(1 << 20, 1 << 12, 1024, 64, False) == 0  # no int overflow in B*H

@@ -28,9 +28,14 @@ def test_recorded_traffic_is_gated_by_the_source_hash(monkeypatch):
 
 
 def test_peaks_come_from_the_measured_file():
-    with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
-        p = json.load(f)
+    # the driver writes MEASURED_PEAKS.json on the machines it measured; without it the recipe's fallback is used
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     burst, sustained, hbm, src = bench.peaks()
+    if not os.path.exists(path):
+        assert (burst, sustained, hbm, src) == (1590.0, 1400.0, 6650.0, "fallback")
+        return
+    with open(path) as f:
+        p = json.load(f)
     assert (burst, sustained, hbm, src) == (float(p["bf16_tflops"]), float(p["bf16_tflops_sustained"]),
                                             float(p["hbm_gbs"]), "measured")
 

@@ -1,9 +1,10 @@
 """Backward parity on the GPU: dQ, dK, dV from libfa.so through the C ABI vs the fp64 oracle.
 
 Tolerance: per tensor, max-abs error <= 5e-2 * max |gradient| (bf16/fp16 inputs, fp32 accumulation).  Small cases
-span several tiles with ragged tails; the workload shapes run at full size (full oracle where it finishes in
-seconds; long sequences: 256 sampled query rows for dQ and sampled keys of one head for dK/dV, plus invariants
-that hold at any size).
+span several tiles with ragged tails; the workload shapes run at full size: the full oracle for tiny, GPT-2, BERT
+and the 4K long-context case (every element), and at 8K / 16K sampled elements (dQ of 2048 query rows, dK and dV of
+256 keys in each of two heads) plus invariants that hold at any size.  Every tolerance scale comes from the
+oracle's own values, never from the tensor under test.
 """
 import numpy as np
 import pytest
@@ -11,7 +12,8 @@ import torch
 
 import oracle
 from exact_io_aware_48_b200 import inputs
-from parity import assert_grad_close, assert_lse_close, assert_o_close, f64, gpu_fwd_bwd, log_errors
+from parity import (assert_grad_close, assert_lse_close, assert_o_close, f64, gpu_fwd_bwd, log_errors,
+                    sampled_keys)
 
 pytestmark = pytest.mark.gpu
 
@@ -63,8 +65,9 @@ def test_bwd_workloads_full(name):
             assert torch.all(dk[b, :, kl[b]:] == 0) and torch.all(dv[b, :, kl[b]:] == 0)
 
 
-def check_invariants(dq, dk, dv, do, lse):
-    # sum_c dK_c = 0 and sum_c dV_c = sum of dO over rows with a visible key, per head (algebra of softmax)
+def check_invariants(dk, dv, do, lse):
+    # sum_c dK_c = 0 and sum_c dV_c = sum of dO over rows with a visible key, per head (algebra of softmax).  A smoke
+    # check on the whole tensors at any size; the parity evidence is the element-wise comparison with the oracle.
     dk64, dv64 = dk.double(), dv.double()
     do64 = do.double() * torch.isfinite(lse).double()[..., None]
     ref = do64.sum(dim=2)
@@ -72,31 +75,38 @@ def check_invariants(dq, dk, dv, do, lse):
     assert torch.max(torch.abs(dk64.sum(dim=2))) <= 2e-2 * (1 + dk64.abs().sum(dim=2).max())
 
 
-@pytest.mark.parametrize("name", ["lc4k", "lc8k", "lc16k"])
+def test_bwd_lc4k_full_oracle():
+    # every element of dQ, dK, dV at B1 H16 N4096 d128 causal against the full fp64 oracle backward (all heads)
+    w = inputs.workloads()["lc4k"]
+    q, k, v, do = w.tensors()
+    o, lse, dq, dk, dv = gpu_fwd_bwd(q, k, v, do, w.causal, w.scale)
+    rq, rk, rv, ro, rl = oracle.attn_bwd(f64(q), f64(k), f64(v), f64(do), w.scale, causal=w.causal)
+    eo = assert_o_close(o.double().numpy(), ro)
+    el = assert_lse_close(lse.numpy(), rl)
+    e = [assert_grad_close(g.double().numpy(), r, n) for g, r, n in ((dq, rq, "dQ"), (dk, rk, "dK"), (dv, rv, "dV"))]
+    log_errors("bwd_lc4k_full", o=eo, lse=el, dq=e[0], dk=e[1], dv=e[2])
+
+
+@pytest.mark.parametrize("name", ["lc8k", "lc16k"])
 def test_bwd_long_context_sampled(name):
+    # The full oracle backward is too slow at these sizes, so it computes sampled elements: dQ of 2048 seeded
+    # (head, query) rows over all heads, and dK, dV of 256 seeded keys in each of two seeded heads (the oracle then
+    # runs those heads' whole forward).  The tolerance scale of each tensor is the largest magnitude among the
+    # oracle's own sampled values -- never the GPU's -- which is at most the tensor's largest magnitude, so the bar
+    # is at least as strict as 5e-2 of the largest gradient.
     w = inputs.workloads()[name]
     q, k, v, do = w.tensors()
     o, lse, dq, dk, dv = gpu_fwd_bwd(q, k, v, do, w.causal, w.scale)
     qf, kf, vf, dof = f64(q), f64(k), f64(v), f64(do)
-    sb, sr = inputs.sample_rows(w.seed + 600, w.B * w.H, w.N, 256)
+    sb, sr = inputs.sample_rows(w.seed + 600, w.B * w.H, w.N, 2048)
+    ro, rl = oracle.attn_fwd_rows(qf, kf, vf, w.scale, sb, sr, causal=w.causal)
+    eo = assert_o_close(o.reshape(-1, w.N, w.d)[sb, sr].double().numpy(), ro)
+    el = assert_lse_close(lse.reshape(-1, w.N)[sb, sr].numpy(), rl)
     rq = oracle.attn_bwd_rows(qf, kf, vf, dof, w.scale, sb, sr, causal=w.causal)
-    # dK/dV: 128 sampled keys of one head (the oracle needs that head's full forward)
-    head = int(sb[0])
-    kb, kc = inputs.sample_rows(w.seed + 700, 1, w.N, 128)
-    kb = np.full_like(kc, head)
+    kb, kc = sampled_keys(w.seed + 700, w.B * w.H, w.N, heads=2, per_head=256)
     rk, rv = oracle.attn_bwd_keys(qf, kf, vf, dof, w.scale, kb, kc, causal=w.causal)
-    # the tolerance scale is the largest gradient magnitude of the whole tensor (GPU value, within tolerance)
-    e_q = _sampled_close(dq.reshape(-1, w.N, w.d)[sb, sr], rq, dq, "dQ")
-    e_k = _sampled_close(dk.reshape(-1, w.N, w.d)[kb, kc], rk, dk, "dK")
-    e_v = _sampled_close(dv.reshape(-1, w.N, w.d)[kb, kc], rv, dv, "dV")
-    log_errors(f"bwd_{name}_sampled", dq=e_q, dk=e_k, dv=e_v)
-    check_invariants(dq, dk, dv, do, lse)
-
-
-def _sampled_close(got, ref, full, name):
-    got = got.double().numpy()
-    assert np.all(np.isfinite(got)), name
-    scale = max(float(np.max(np.abs(ref))), float(full.float().abs().max()))
-    err = float(np.max(np.abs(got - ref)))
-    assert err <= 5e-2 * scale, f"{name}: {err:.3e} > 5e-2 * {scale:.3e}"
-    return err / scale
+    e_q = assert_grad_close(dq.reshape(-1, w.N, w.d)[sb, sr].double().numpy(), rq, "dQ")
+    e_k = assert_grad_close(dk.reshape(-1, w.N, w.d)[kb, kc].double().numpy(), rk, "dK")
+    e_v = assert_grad_close(dv.reshape(-1, w.N, w.d)[kb, kc].double().numpy(), rv, "dV")
+    log_errors(f"bwd_{name}_sampled", o=eo, lse=el, dq=e_q, dk=e_k, dv=e_v)
+    check_invariants(dk, dv, do, lse)
