@@ -2,12 +2,15 @@
 """Benchmark: exact attention forward + backward on B200 through libfa.so's C ABI.
 
 One step = one pass of the whole hot path over one batch: fa_fwd (tiled forward with online softmax) followed by
-fa_bwd (preprocess, recomputing backward, dQ conversion).  The workload is the GPT-2-small-shaped causal
-self-attention (B=8, H=12, N=1024, d=64, bf16); the long-context causal rows (B=1, H=16, d=128, N=4096/8192/16384)
-are measured in the same run under "targets".  FLOPs are algorithmic: forward 4*d per visible (query, key) pair,
-backward 2.5x forward (five GEMM-shaped products per visible tile pair), step 3.5x forward.
+fa_bwd (preprocess, recomputing backward, dQ conversion).  The headline workload is the long-context causal case the
+throughput target is stated on (B=1, H=16, N=16384, d=128, bf16: the largest single-GPU configuration).  Every other
+workload shape (tiny, GPT-2-small, BERT-large with key lengths, 4K / 8K long context, 64K block-sparse) is measured in
+the same run under "configs", together with the packed-batch, decode and head-dim-256 paths and the standard
+(materialising) attention baseline on the GPT-2 shape.  FLOPs are algorithmic: forward 4*d per visible (query, key)
+pair, backward 2.5x forward (five GEMM-shaped products per visible tile pair), step 3.5x forward.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--no-targets]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+                    [--no-extras] [--no-cpu-baseline] [--no-e2e]
 
 Multi-GPU (torchrun, one process per GPU): each rank runs its own independent batch of the same shape (attention
 heads are independent, so there is no data-path collective: weak scaling); value = all ranks' FLOPs / max time.
@@ -28,6 +31,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "attention fwd / fwd+bwd TFLOP/s on 1 B200 and % of dense BF16 tensor peak"
+DEFAULT_WORKLOAD = "lc16k"
 WORKLOAD_NAMES = {
     "gpt2": "gpt2-small-shaped causal self-attention fwd+bwd B8 H12 N1024 d64 bf16",
     "tiny": "tiny exact attention fwd+bwd B1 H2 N256 d64 bf16",
@@ -35,8 +39,11 @@ WORKLOAD_NAMES = {
     "lc4k": "long-context causal fwd+bwd B1 H16 N4096 d128 bf16",
     "lc8k": "long-context causal fwd+bwd B1 H16 N8192 d128 bf16",
     "lc16k": "long-context causal fwd+bwd B1 H16 N16384 d128 bf16",
+    "bs64k": "block-sparse fwd+bwd B1 H8 N65536 d64 fp16, 128x128 tile mask band4+butterfly+2% random",
 }
 L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
+# workloads reported with HBM bandwidth next to TFLOP/s (short sequences: near or below the ridge point)
+HBM_REPORTED = ("tiny", "bert")
 
 
 # ---------------------------------------------------------------------------------------------- FLOP accounting
@@ -47,8 +54,11 @@ def visible_pairs(B, H, N, causal, key_lens=None, block_mask=None, tile=128):
         return B * H * (N * (N + 1) // 2 if causal else N * N)
     if block_mask is None and not causal:
         return H * N * int(np.sum(np.minimum(np.asarray(key_lens, dtype=np.int64), N)))
-    # general: count per tile (rows x visible keys)
     nT = -(-N // tile)
+    if key_lens is None and not causal:  # kept tiles times their (possibly ragged) extents
+        ext = np.minimum(N - np.arange(nT) * tile, tile).astype(np.int64)
+        return B * H * int(ext @ np.asarray(block_mask, dtype=np.int64) @ ext)
+    # general: count per tile (rows x visible keys)
     total = 0
     lens = [N] * B if key_lens is None else [min(int(x), N) for x in key_lens]
     for b in range(B):
@@ -66,12 +76,22 @@ def visible_pairs(B, H, N, causal, key_lens=None, block_mask=None, tile=128):
     return total * H
 
 
+def row_visible_keys(w, sel_r):
+    """Visible keys of each selected query row (integer array), for the sampled-row CPU baseline."""
+    import numpy as np
+    r = np.asarray(sel_r, dtype=np.int64)
+    if w.key_lens or w.blocksparse:
+        raise ValueError("row sampling is used on the dense long-context workloads only")
+    return np.minimum(r + 1, w.N) if w.causal else np.full_like(r, w.N)
+
+
 def kernel_src_hash():
     """sha256 (first 16 hex digits) over the kernel sources and the C header, file name + contents, sorted."""
     import glob
     import hashlib
     files = sorted(glob.glob(os.path.join(ROOT, "exact_io_aware_48_b200", "csrc", "*.cu"))
-                   + glob.glob(os.path.join(ROOT, "exact_io_aware_48_b200", "csrc", "*.cuh")))
+                   + glob.glob(os.path.join(ROOT, "exact_io_aware_48_b200", "csrc", "*.cuh"))
+                   + glob.glob(os.path.join(ROOT, "exact_io_aware_48_b200", "csrc", "*.h")))
     files.append(os.path.join(ROOT, "include", "fa.h"))
     h = hashlib.sha256()
     for f in files:
@@ -95,6 +115,15 @@ def recorded_traffic(workload, kernel):
         return None
 
 
+def recorded_standard_traffic():
+    """The ncu DRAM totals of one standard (materialising) forward and one tiled forward on the GPT-2 shape."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "standard_traffic_gpt2.json")) as f:
+            return json.load(f)
+    except Exception:
+        return None
+
+
 def fwd_flops(d, pairs):
     return 4.0 * d * pairs
 
@@ -104,6 +133,15 @@ def algorithmic_bwd_bytes(w):
     (fp32) read.  The fp32 dQ partial sums are reduced in L2 and counted separately."""
     e = 2
     return 6 * w.B * w.H * w.N * w.d * e + 2 * 4 * w.B * w.H * w.nT * 128
+
+
+def algorithmic_pass_bytes(w):
+    """Minimum HBM bytes of a whole forward call (Q, K, V read, O written, LSE written) and of a whole backward call
+    (Q, K, V, O, dO read, dQ, dK, dV written, LSE read, D written and read)."""
+    e = 2
+    t = w.B * w.H * w.N * w.d * e
+    rows = w.B * w.H * w.N
+    return 4 * t + 4 * rows, 8 * t + 12 * rows
 
 
 def peaks():
@@ -173,7 +211,8 @@ class ClockSampler:
 
 # ---------------------------------------------------------------------------------------------- GPU arm
 class Problem:
-    """Device-resident inputs, outputs and workspace for one attention workload; step() = fa_fwd + fa_bwd."""
+    """Device-resident inputs, outputs and workspace for one attention workload; step() = forward + backward through
+    fa_fwd / fa_bwd (fa_fwd_blocksparse and fa_bwd with the tile mask for the block-sparse workload)."""
 
     def __init__(self, w, seed_offset=0, device="cuda"):
         import torch
@@ -188,10 +227,14 @@ class Problem:
         self.o = torch.empty_like(self.q)
         self.lse = torch.empty((w.B, w.H, w.N), device=device, dtype=torch.float32)
         self.dq, self.dk, self.dv = (torch.empty_like(self.q) for _ in range(3))
-        self.ws_bytes = _lib.fa_bwd_workspace_size(w.B, w.H, w.N, w.d, False)
+        self.mask = w.block_mask()
+        self.bm = None if self.mask is None else torch.as_tensor(self.mask, dtype=torch.uint8, device=device)
+        self.ws_bytes = _lib.fa_bwd_workspace_size(w.B, w.H, w.N, w.d, self.bm is not None)
         self.ws = torch.empty(self.ws_bytes, device=device, dtype=torch.uint8)
+        self.fws_bytes = _lib.fa_blocksparse_workspace_size(w.N) if self.bm is not None else 0
+        self.fws = torch.empty(max(self.fws_bytes, 1), device=device, dtype=torch.uint8)
         self.dt = _lib.FA_BF16 if w.dtype == "bf16" else _lib.FA_FP16
-        self.pairs = visible_pairs(w.B, w.H, w.N, w.causal, w.key_lens_array())
+        self.pairs = visible_pairs(w.B, w.H, w.N, w.causal, w.key_lens_array(), self.mask)
         self.fwd_flops = fwd_flops(w.d, self.pairs)
         self.kl = None
         if w.key_lens:
@@ -199,15 +242,19 @@ class Problem:
 
     def fwd(self, stream):
         w, L = self.w, self.lib
-        rc = L.fa_fwd(self.q, self.k, self.v, self.o, self.lse, w.B, w.H, w.N, w.d, w.scale, w.causal, self.kl,
-                      self.dt, stream)
+        if self.bm is None:
+            rc = L.fa_fwd(self.q, self.k, self.v, self.o, self.lse, w.B, w.H, w.N, w.d, w.scale, w.causal, self.kl,
+                          self.dt, stream)
+        else:
+            rc = L.fa_fwd_blocksparse(self.q, self.k, self.v, self.o, self.lse, w.B, w.H, w.N, w.d, w.scale,
+                                      w.causal, self.kl, self.bm, self.fws, self.fws_bytes, self.dt, stream)
         if rc:
-            raise RuntimeError(f"fa_fwd: {L.fa_status_string(rc)}")
+            raise RuntimeError(f"forward: {L.fa_status_string(rc)}")
 
     def bwd(self, stream):
         w, L = self.w, self.lib
         rc = L.fa_bwd(self.q, self.k, self.v, self.o, self.do, self.lse, self.dq, self.dk, self.dv, w.B, w.H, w.N,
-                      w.d, w.scale, w.causal, self.kl, None, self.ws, self.ws_bytes, self.dt, stream)
+                      w.d, w.scale, w.causal, self.kl, self.bm, self.ws, self.ws_bytes, self.dt, stream)
         if rc:
             raise RuntimeError(f"fa_bwd: {L.fa_status_string(rc)}")
 
@@ -257,24 +304,62 @@ def time_loop(fn, steps, stream, flush, kernel_events=None):
     return step_ms, k_ms
 
 
-def measure_targets(stream, flush, peak):
-    """Long-context causal rows (d=128): fwd and bwd TFLOP/s, fraction of the dense BF16 peak."""
-    from exact_io_aware_48_b200 import inputs
-    out = {}
-    for name in ("lc4k", "lc8k", "lc16k"):
-        w = inputs.workloads()[name]
+def check_status(lib, stream, where):
+    status = lib.fa_last_device_status(stream)
+    if status:
+        raise RuntimeError(f"{where}: device status {lib.fa_status_string(status)}")
+
+
+def measure_config(name, stream, flush, peak, hbm, p=None, reps=10):
+    """Forward and backward of one workload, each timed alone (median of `reps` calls, L2 flushed before each):
+    call-level ms and TFLOP/s, the main kernels' own ms (events around their launches), fractions of the dense bf16
+    peak, and HBM GB/s by algorithmic bytes for the short-sequence workloads.  Block-sparse: TFLOP/s count kept-tile
+    pairs and the mask-to-list conversion is timed on its own."""
+    import torch
+    from exact_io_aware_48_b200 import _lib, inputs
+    w = inputs.workloads()[name]
+    own = p is None
+    if own:
         p = Problem(w)
+    for _ in range(3):
+        p.step(stream)
+    f_ms, fk = time_loop(p.fwd, reps, stream, flush, (_lib.FA_KERNEL_FWD, _lib))
+    b_ms, bk = time_loop(p.bwd, reps, stream, flush, (_lib.FA_KERNEL_BWD_MAIN, _lib))
+    check_status(_lib, stream, name)
+    f, b = statistics.median(f_ms), statistics.median(b_ms)
+    fkm, bkm = statistics.median(fk), statistics.median(bk)
+    ff = p.fwd_flops
+    out = {"workload": WORKLOAD_NAMES[name], "visible_pairs": int(p.pairs),
+           "fwd_ms": round(f, 4), "bwd_ms": round(b, 4), "fwd_bwd_ms": round(f + b, 4),
+           "fwd_tflops": round(ff / f / 1e9, 1), "bwd_tflops": round(2.5 * ff / b / 1e9, 1),
+           "fwd_bwd_tflops": round(3.5 * ff / (f + b) / 1e9, 1),
+           "fwd_frac": round(ff / f / 1e9 / peak, 4), "bwd_frac": round(2.5 * ff / b / 1e9 / peak, 4),
+           "fwd_kernel_ms": round(fkm, 4), "bwd_main_kernel_ms": round(bkm, 4),
+           "fwd_kernel_tflops": round(ff / fkm / 1e9, 1), "bwd_main_kernel_tflops": round(2.5 * ff / bkm / 1e9, 1)}
+    if name in HBM_REPORTED:
+        fb, bb = algorithmic_pass_bytes(w)
+        out.update({"fwd_us": round(f * 1e3, 2), "bwd_us": round(b * 1e3, 2),
+                    "fwd_hbm_gbs": round(fb / f / 1e6, 1), "bwd_hbm_gbs": round(bb / b / 1e6, 1),
+                    "fwd_hbm_frac": round(fb / f / 1e6 / hbm, 4), "bwd_hbm_frac": round(bb / b / 1e6 / hbm, 4),
+                    "algorithmic_bytes": {"fwd": fb, "bwd": bb}})
+    if p.bm is not None:
+        nT = w.nT
+        rp, ci, cp, ri = (torch.empty(n, device="cuda", dtype=torch.int32) for n in (nT + 1, nT * nT, nT + 1, nT * nT))
+
+        def lists(st):
+            rc = _lib.fa_blockmask_lists(p.bm, nT, rp, ci, cp, ri, st)
+            if rc:
+                raise RuntimeError(f"fa_blockmask_lists: {_lib.fa_status_string(rc)}")
         for _ in range(3):
-            p.step(stream)
-        f_ms, _ = time_loop(p.fwd, 10, stream, flush)
-        b_ms, _ = time_loop(p.bwd, 10, stream, flush)
-        f, b = statistics.median(f_ms), statistics.median(b_ms)
-        ftf = p.fwd_flops / f / 1e9
-        btf = 2.5 * p.fwd_flops / b / 1e9
-        out[name] = {"fwd_ms": round(f, 4), "bwd_ms": round(b, 4), "fwd_tflops": round(ftf, 1),
-                     "bwd_tflops": round(btf, 1), "fwd_frac": round(ftf / peak, 4), "bwd_frac": round(btf / peak, 4),
-                     "fwd_bwd_tflops": round(3.5 * p.fwd_flops / (f + b) / 1e9, 1)}
+            lists(stream)
+        l_ms, _ = time_loop(lists, reps, stream, flush)
+        lm = statistics.median(l_ms)
+        out.update({"kept_tiles": int(p.mask.sum()), "tiles": nT * nT, "mask_lists_ms": round(lm, 4),
+                    "flop_convention": "kept-tile pairs (kept tiles x 128 x 128 x H); fwd_ms and bwd_ms include "
+                                       "the mask-to-list conversion, which mask_lists_ms times alone"})
+    if own:
         del p
+        torch.cuda.empty_cache()
     return out
 
 
@@ -320,9 +405,7 @@ def measure_varlen(stream, flush, peak):
     f_ms, _ = time_loop(fwd, 10, stream, flush)
     b_ms, _ = time_loop(bwd, 10, stream, flush)
     f, b = statistics.median(f_ms), statistics.median(b_ms)
-    status = _lib.fa_last_device_status(stream)
-    if status:
-        raise RuntimeError(f"packed-batch kernels reported {_lib.fa_status_string(status)}")
+    check_status(_lib, stream, "packed-batch kernels")
     padded = Problem(w)  # the same shape padded to N with key lengths
     for _ in range(3):
         padded.step(stream)
@@ -364,9 +447,7 @@ def measure_decode(stream, flush, hbm_gbs):
     for _ in range(3):
         step(stream)
     ms, _ = time_loop(step, 20, stream, flush)
-    status = _lib.fa_last_device_status(stream)
-    if status:
-        raise RuntimeError(f"split-K/V forward reported {_lib.fa_status_string(status)}")
+    check_status(_lib, stream, "split-K/V forward")
     t = statistics.median(ms)
     nbytes = 2 * B * H * Nk * d * 2 + 2 * B * H * Nq * d * 2
     gbs = nbytes / t / 1e6
@@ -375,31 +456,106 @@ def measure_decode(stream, flush, hbm_gbs):
 
 
 def measure_d256(stream, flush, peak):
-    """Head dim 256 forward (its own kernel; no backward at d = 256): B1 H16 N8192 bf16 causal, the long-context
-    shape at twice the head dim.  TFLOP/s by the algorithmic convention (4*d per visible pair)."""
+    """Head dim 256 (its own forward and backward kernels): B1 H16 N8192 bf16 causal, the long-context shape at
+    twice the head dim.  TFLOP/s by the algorithmic convention (4*d per visible pair forward, 2.5x backward)."""
     import torch
     from exact_io_aware_48_b200 import _lib, inputs
     B, H, N, d = 1, 16, 8192, 256
-    q, k, v = [inputs.gaussian((B, H, N, d), 510 + t, "bf16").cuda() for t in range(3)]
+    q, k, v, do = [inputs.gaussian((B, H, N, d), 510 + t, "bf16").cuda() for t in range(4)]
     o = torch.empty_like(q)
     lse = torch.empty((B, H, N), device="cuda", dtype=torch.float32)
     scale = 1.0 / math.sqrt(d)
 
-    def step(st):
+    def fwd(st):
         rc = _lib.fa_fwd(q, k, v, o, lse, B, H, N, d, scale, True, None, _lib.FA_BF16, st)
         if rc:
             raise RuntimeError(f"fa_fwd: {_lib.fa_status_string(rc)}")
 
     for _ in range(3):
-        step(stream)
-    ms, _ = time_loop(step, 10, stream, flush)
-    status = _lib.fa_last_device_status(stream)
-    if status:
-        raise RuntimeError(f"d = 256 forward reported {_lib.fa_status_string(status)}")
+        fwd(stream)
+    ms, _ = time_loop(fwd, 10, stream, flush)
+    check_status(_lib, stream, "d = 256 forward")
     t = statistics.median(ms)
-    tf = 4 * d * B * H * (N * (N + 1) // 2) / t / 1e9
-    return {"workload": f"fwd B{B} H{H} N{N} d{d} bf16 causal", "ms": round(t, 4), "tflops": round(tf, 1),
-            "frac": round(tf / peak, 4) if peak else None}
+    ff = 4 * d * B * H * (N * (N + 1) // 2)
+    out = {"workload": f"B{B} H{H} N{N} d{d} bf16 causal", "fwd_ms": round(t, 4), "fwd_tflops": round(ff / t / 1e9, 1),
+           "fwd_frac": round(ff / t / 1e9 / peak, 4) if peak else None}
+    ws_bytes = _lib.fa_bwd_workspace_size(B, H, N, d, False)
+    if ws_bytes:  # the backward takes d = 256
+        ws = torch.empty(ws_bytes, device="cuda", dtype=torch.uint8)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+        def bwd(st):
+            rc = _lib.fa_bwd(q, k, v, o, do, lse, dq, dk, dv, B, H, N, d, scale, True, None, None, ws, ws_bytes,
+                             _lib.FA_BF16, st)
+            if rc:
+                raise RuntimeError(f"fa_bwd: {_lib.fa_status_string(rc)}")
+
+        for _ in range(3):
+            bwd(stream)
+        bms, _ = time_loop(bwd, 10, stream, flush)
+        check_status(_lib, stream, "d = 256 backward")
+        tb = statistics.median(bms)
+        out.update({"bwd_ms": round(tb, 4), "bwd_tflops": round(2.5 * ff / tb / 1e9, 1),
+                    "bwd_frac": round(2.5 * ff / tb / 1e9 / peak, 4) if peak else None,
+                    "fwd_bwd_tflops": round(3.5 * ff / (t + tb) / 1e9, 1)})
+    return out
+
+
+def measure_standard(stream, flush, reps=5):
+    """The slide deck's suggested experiment ("Run it": a toy that materialises the attention matrix against the
+    tiled streaming version) on the GPT-2 shape: eager PyTorch standard attention -- S = scale*QK^T written to HBM,
+    masked, softmax, P V, backward through autograd (P and dS also materialised) -- timed next to fa_fwd/fa_bwd on
+    the same inputs.  Measurement only: nothing here is on the library's path.  The DRAM-byte ratio is the one an
+    ncu capture of the same comparison recorded (profiles/standard_traffic_gpt2.json)."""
+    import torch
+    from exact_io_aware_48_b200 import inputs
+    w = inputs.workloads()["gpt2"]
+    p = Problem(w)
+    q = p.q.detach().clone().requires_grad_(True)
+    k = p.k.detach().clone().requires_grad_(True)
+    v = p.v.detach().clone().requires_grad_(True)
+    mask = torch.ones(w.N, w.N, device="cuda", dtype=torch.bool).tril() if w.causal else None
+
+    def std_fwd(_s=None):
+        s = torch.matmul(q, k.transpose(-1, -2)) * w.scale
+        if mask is not None:
+            s = s.masked_fill(~mask, float("-inf"))
+        return torch.matmul(torch.softmax(s.float(), dim=-1).to(q.dtype), v)
+
+    def std_step(_s=None):
+        o = std_fwd()
+        o.backward(p.do)
+        q.grad = k.grad = v.grad = None
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            std_step()
+            p.step(stream)
+    stream.synchronize()
+    res = {}
+    for name, fn in (("standard_fwd", lambda s: std_fwd()), ("standard_fwd_bwd", std_step),
+                     ("tiled_fwd", p.fwd), ("tiled_fwd_bwd", p.step)):
+        with torch.cuda.stream(stream):
+            ms, _ = time_loop(fn, reps, stream, flush)
+        res[name] = statistics.median(ms)
+    with torch.no_grad():
+        o_std = std_fwd().detach()
+    p.fwd(stream)
+    stream.synchronize()
+    err = float((o_std.float() - p.o.float()).abs().max())
+    out = {"workload": WORKLOAD_NAMES["gpt2"], "standard": "eager PyTorch, S and P materialised in HBM",
+           "ms": {k2: round(v2, 4) for k2, v2 in res.items()}, "standard_fwd_ms": round(res["standard_fwd"], 4),
+           "speedup_fwd": round(res["standard_fwd"] / res["tiled_fwd"], 2),
+           "speedup_fwd_bwd": round(res["standard_fwd_bwd"] / res["tiled_fwd_bwd"], 2),
+           "max_abs_diff_O": err, "l2": "flushed before every timed call"}
+    tr = recorded_standard_traffic()
+    if tr:
+        out["dram_bytes_recorded"] = {"standard_fwd": tr["standard_fwd_dram_bytes"],
+                                      "tiled_fwd": tr["tiled_fwd_dram_bytes"],
+                                      "ratio": round(tr["standard_fwd_dram_bytes"] / tr["tiled_fwd_dram_bytes"], 1),
+                                      "source": "ncu dram__bytes_read.sum + dram__bytes_write.sum (recorded)"}
+    del p
+    return out
 
 
 def run_ours(args):
@@ -445,13 +601,8 @@ def run_ours(args):
     value, total_ms = aggregate(float(sum(step_ms)), step_flops, args.steps, world, "cuda")
     ms_per_step = total_ms / args.steps
 
-    # separate fwd / bwd breakdown (not part of the headline value)
-    f_ms, fk = time_loop(p.fwd, max(10, args.steps // 2), stream, flush)
-    b_ms, _ = time_loop(p.bwd, max(10, args.steps // 2), stream, flush)
-    fwd_tf = p.fwd_flops / statistics.median(f_ms) / 1e9
-    bwd_tf = 2.5 * p.fwd_flops / statistics.median(b_ms) / 1e9
-
-    # roofline of the dominant kernel (bwd main: 2.5x forward FLOPs per launch), timed live by events
+    # roofline of the dominant kernel (bwd main: 2.5x forward FLOPs per launch), timed live by events around its
+    # launches inside the timed steps
     kmean = float(np.mean(kern_ms))
     achieved = 2.5 * p.fwd_flops / (kmean / 1e3) / 1e12
     kname = f"bwd_kernel<{w.d},{w.dtype}>"
@@ -463,11 +614,18 @@ def run_ours(args):
     # ------------------------------------------------------------------ end to end through the C ABI, host buffers
     e2e = run_e2e(p, stream, args, world) if args.e2e else None
 
-    targets = measure_targets(stream, flush, peak) if (args.targets and rank == 0) else None
-    varlen = measure_varlen(stream, flush, peak) if (args.targets and rank == 0) else None
-    decode = measure_decode(stream, flush, hbm) if (args.targets and rank == 0) else None
-    d256 = measure_d256(stream, flush, peak) if (args.targets and rank == 0) else None
-    cpu = cpu_baseline(p.w) if rank == 0 and world == 1 and args.cpu_baseline else None
+    configs = extra = None
+    if args.extras and rank == 0:
+        configs = {args.workload: measure_config(args.workload, stream, flush, peak, hbm, p=p)}
+    del p
+    torch.cuda.empty_cache()
+    if args.extras and rank == 0:
+        for name in ("tiny", "gpt2", "bert", "lc4k", "lc8k", "lc16k", "bs64k"):
+            if name not in configs:
+                configs[name] = measure_config(name, stream, flush, peak, hbm)
+        extra = {"varlen": measure_varlen(stream, flush, peak), "decode": measure_decode(stream, flush, hbm),
+                 "d256": measure_d256(stream, flush, peak), "standard_vs_tiled": measure_standard(stream, flush)}
+    cpu = cpu_baseline(w) if rank == 0 and world == 1 and args.cpu_baseline else None
 
     if rank == 0:
         line = {
@@ -479,19 +637,21 @@ def run_ours(args):
                        "seq_len": w.N, "parallelism": f"dp{world} (independent heads per rank, no collective)",
                        "l2": "flushed (256 MiB write, untimed) before every timed step",
                        "flop_convention": "fwd 4*d*visible pairs; bwd 2.5x; step 3.5x"},
-            "fwd_tflops": round(fwd_tf, 2), "bwd_tflops": round(bwd_tf, 2),
-            "frac_of_peak": {"step": round(value / world / peak, 4), "fwd": round(fwd_tf / peak, 4),
-                             "bwd": round(bwd_tf / peak, 4), "peak_tflops": peak, "peak_source": peak_src},
+            "frac_of_peak": {"step": round(value / world / peak, 4), "peak_tflops": peak, "peak_source": peak_src,
+                             "datasheet_dense_bf16_tflops": 2250.0,
+                             "step_of_datasheet": round(value / world / 2250.0, 4)},
             "roofline": roofline,
             "e2e": e2e,
             "gpu_launches": 4 * args.steps,
             "clocks": clk.summary(),
-            "targets": targets,
-            "varlen": varlen,
-            "decode": decode,
-            "d256": d256,
+            "configs": configs,
+            "paths": extra,
             "cpu_baseline": cpu,
         }
+        if configs and args.workload in configs:
+            c = configs[args.workload]
+            line["fwd_tflops"], line["bwd_tflops"] = c["fwd_tflops"], c["bwd_tflops"]
+            line["frac_of_peak"].update({"fwd": c["fwd_frac"], "bwd": c["bwd_frac"]})
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
@@ -500,7 +660,7 @@ def run_ours(args):
 
 def run_e2e(p, stream, args, world):
     """Same metric through the public C ABI with host buffers: per step, copy q, k, v, dO from pinned host memory,
-    run fa_fwd + fa_bwd, copy O, LSE, dQ, dK, dV back to pinned host memory; device-timed on the stream."""
+    run the forward and backward, copy O, LSE, dQ, dK, dV back to pinned host memory; device-timed on the stream."""
     import torch
     outs = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (p.o, p.lse, p.dq, p.dk, p.dv)]
     h2d = sum(t.numel() * t.element_size() for t in p.host)
@@ -537,118 +697,126 @@ def run_e2e(p, stream, args, world):
 
 
 # ---------------------------------------------------------------------------------------------- CPU oracle
-def oracle_step(w, heads=None):
-    """One fwd+bwd of the fp64 oracle on the workload (optionally the first `heads` flattened heads).
-    Returns (seconds, algorithmic FLOPs of the part computed)."""
+def host_cpu():
+    """CPU model and core counts of this host."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        avail = len(os.sched_getaffinity(0))
+    except AttributeError:
+        avail = os.cpu_count()
+    return {"model": model, "nproc": avail, "logical_cpus": os.cpu_count()}
+
+
+class OracleRows:
+    """The fp64 oracle on sampled query rows of a workload: per row, the row's forward (O, LSE) and its dQ (which
+    recomputes the row's forward).  Credited with the algorithmic FLOPs of that work: 4*d per visible pair for the
+    forward and 6*d for the dQ share of the backward (recomputed scores, dP, dQ; the backward's full 10*d adds dV and
+    dK), so rate = credited FLOPs / seconds and the full step's extrapolated time = 3.5 * 4*d * all pairs / rate."""
+
+    def __init__(self, w):
+        import oracle
+        from exact_io_aware_48_b200 import inputs
+        oracle.build()
+        self.w = w
+        self.inputs = inputs
+        self.oracle = oracle
+        self.q, self.k, self.v, self.do = (inputs.to_f64(t) for t in w.tensors())
+
+    def run(self, nrows, seed):
+        w = self.w
+        sb, sr = self.inputs.sample_rows(seed, w.B * w.H, w.N, nrows)
+        t0 = time.perf_counter()
+        self.oracle.attn_fwd_rows(self.q, self.k, self.v, w.scale, sb, sr, causal=w.causal)
+        self.oracle.attn_bwd_rows(self.q, self.k, self.v, self.do, w.scale, sb, sr, causal=w.causal)
+        dt = time.perf_counter() - t0
+        return dt, 10.0 * w.d * float(row_visible_keys(w, sr).sum())
+
+
+def cpu_baseline(w, target_s=10.0):
+    """The oracle as it stands on this host's cores, on a bounded sample of the timed workload (sampled query rows,
+    rate extrapolated to the full step), plus the tiny workload's full fwd+bwd on one core and on all cores."""
     import oracle
     from exact_io_aware_48_b200 import inputs
-    q, k, v, do = (inputs.to_f64(t) for t in w.tensors())
-    B, H = w.B, w.H
-    if heads is not None and heads < B * H:
-        sl = lambda x: x.reshape(B * H, w.N, w.d)[:heads].reshape(1, heads, w.N, w.d)
-        q, k, v, do = sl(q), sl(k), sl(v), sl(do)
-        B, H = 1, heads
-    kl = w.key_lens_array()
-    t0 = time.perf_counter()
-    oracle.attn_bwd(q, k, v, do, w.scale, causal=w.causal, key_lens=kl if B == w.B else None)
-    dt = time.perf_counter() - t0
-    return dt, 3.5 * fwd_flops(w.d, visible_pairs(B, H, w.N, w.causal))
-
-
-def cpu_baseline(w):
-    import oracle
     oracle.build()
-    reps, secs, flops = 0, 0.0, 0.0
-    while secs < 10.0 and reps < 20:  # about 10-30 s of CPU work
-        dt, f = oracle_step(w)
+    cores = oracle.num_threads()
+    rows = OracleRows(w)
+    secs, flops, n, nrows = 0.0, 0.0, 0, 256
+    while secs < target_s and n < 64:
+        dt, f = rows.run(nrows, 5000 + n)
         secs += dt
         flops += f
-        reps += 1
-    return {"value": round(flops / secs / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
-            "kind": "oracle",
-            "sample": f"full workload fwd+bwd (fp64 C oracle, OpenMP over heads) x{reps}, {secs:.1f} s"}
+        n += 1
+    rate = flops / secs
+    full_flops = 3.5 * fwd_flops(w.d, visible_pairs(w.B, w.H, w.N, w.causal, w.key_lens_array(), w.block_mask()))
+    tiny = inputs.workloads()["tiny"]
+    tq, tk, tv, tdo = (inputs.to_f64(t) for t in tiny.tensors())
+    tiny_flops = 3.5 * fwd_flops(tiny.d, visible_pairs(tiny.B, tiny.H, tiny.N, tiny.causal))
+
+    def tiny_rate(threads, reps=5):
+        oracle.set_num_threads(threads)
+        t0 = time.perf_counter()
+        for _ in range(reps):
+            oracle.attn_bwd(tq, tk, tv, tdo, tiny.scale, causal=tiny.causal)
+        return reps * tiny_flops / (time.perf_counter() - t0) / 1e12
+
+    tiny_1 = tiny_rate(1)
+    tiny_all = tiny_rate(cores)
+    oracle.set_num_threads(cores)
+    return {"value": round(rate / 1e12, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} x {nrows} seeded query rows of the timed workload: each row's forward and dQ (fp64 C "
+                      f"oracle, OpenMP over rows), {secs:.1f} s; rate extrapolated to the full step",
+            "extrapolated_full_step_s": round(full_flops / rate, 1), "extrapolated": True,
+            "host": host_cpu(),
+            "tiny_full_fwd_bwd": {"workload": WORKLOAD_NAMES["tiny"], "tflops_1_core": round(tiny_1, 6),
+                                  f"tflops_{cores}_cores": round(tiny_all, 6)}}
 
 
 def run_reference(args):
-    import oracle
     from exact_io_aware_48_b200 import inputs
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    oracle.build()
-    w = inputs.workloads()["gpt2"]
-    heads = 24  # each step: a quarter of the workload's heads (bounded sample)
-    for _ in range(args.warmup):
-        oracle_step(w, heads)
+    w = inputs.workloads()[args.workload]
+    rows = OracleRows(w)
+    nrows = 256  # each step: 256 seeded query rows of the workload (bounded sample)
+    for s in range(args.warmup):
+        rows.run(nrows, 9000 + s)
     secs, flops = 0.0, 0.0
-    for _ in range(args.steps):
-        dt, f = oracle_step(w, heads)
+    for s in range(args.steps):
+        dt, f = rows.run(nrows, 9500 + s)
         secs += dt
         flops += f
     val = flops / secs / 1e12
     ms = secs / args.steps * 1e3
-    cores = oracle.num_threads()
+    cores = rows.oracle.num_threads()
     line = {"impl": "reference", "metric": METRIC, "value": round(val, 6), "unit": "TFLOP/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "gpt2-small-shaped causal self-attention fwd+bwd B8 H12 N1024 d64 bf16",
-                       "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": True, "global_batch": w.B,
+            "config": {"workload": WORKLOAD_NAMES.get(w.name, w.name),
+                       "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal, "global_batch": w.B,
                        "seq_len": w.N, "parallelism": "host cores (OpenMP)"},
             "cpu_baseline": {"value": round(val, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                             "sample": f"{heads} of {w.B * w.H} heads per step, fwd+bwd, fp64"},
+                             "sample": f"{nrows} seeded query rows per step: each row's forward and dQ, fp64; rate "
+                                       "extrapolated to the full step", "host": host_cpu()},
             "e2e": {"value": round(val, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
 def run_standard(args):
-    """The slide deck's suggested experiment ("Run it": a toy that materialises the attention matrix against the
-    tiled streaming version): eager PyTorch standard attention -- S = scale*QK^T written to HBM, masked, softmax, P V,
-    backward through autograd (P and dS also materialised) -- timed next to fa_fwd/fa_bwd on the same workload.
-    Prints one JSON line.  Measurement only: nothing here is on the library's path."""
+    """Prints the standard-vs-tiled comparison alone (the default run includes it under paths.standard_vs_tiled)."""
     import torch
-    from exact_io_aware_48_b200 import _lib, inputs
     torch.cuda.set_device(0)
     stream = torch.cuda.Stream()
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
-    w = inputs.workloads()[args.workload]
-    p = Problem(w)
-    q = p.q.detach().clone().requires_grad_(True)
-    k = p.k.detach().clone().requires_grad_(True)
-    v = p.v.detach().clone().requires_grad_(True)
-    mask = torch.ones(w.N, w.N, device="cuda", dtype=torch.bool).tril() if w.causal else None
-
-    def std_fwd(_s=None):
-        s = torch.matmul(q, k.transpose(-1, -2)) * w.scale
-        if mask is not None:
-            s = s.masked_fill(~mask, float("-inf"))
-        return torch.matmul(torch.softmax(s.float(), dim=-1).to(q.dtype), v)
-
-    def std_step(_s=None):
-        o = std_fwd()
-        o.backward(p.do)
-        q.grad = k.grad = v.grad = None
-
-    with torch.cuda.stream(stream):
-        for _ in range(3):
-            std_step()
-            p.step(stream)
-    stream.synchronize()
-    n = max(5, args.steps // 2)
-    res = {}
-    for name, fn in (("standard_fwd", lambda s: std_fwd()), ("standard_fwd_bwd", std_step),
-                     ("tiled_fwd", p.fwd), ("tiled_fwd_bwd", p.step)):
-        with torch.cuda.stream(stream):
-            ms, _ = time_loop(fn, n, stream, flush)
-        res[name] = statistics.median(ms)
-    o_std = std_fwd().detach()
-    p.fwd(stream)
-    stream.synchronize()
-    err = float((o_std.float() - p.o.float()).abs().max())
-    line = {"mode": "standard-attention baseline", "workload": WORKLOAD_NAMES.get(w.name, w.name),
-            "ms": {k2: round(v2, 4) for k2, v2 in res.items()},
-            "speedup_fwd": round(res["standard_fwd"] / res["tiled_fwd"], 2),
-            "speedup_fwd_bwd": round(res["standard_fwd_bwd"] / res["tiled_fwd_bwd"], 2),
-            "max_abs_diff_O": err, "steps": n, "l2": "flushed before every timed call"}
+    line = {"mode": "standard-attention baseline", **measure_standard(stream, flush, reps=max(5, args.steps // 2))}
     print(json.dumps(line), flush=True)
 
 
@@ -660,11 +828,12 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--standard", action="store_true",
                     help="time eager standard (materialising) attention next to the tiled kernels and exit")
-    ap.add_argument("--no-targets", dest="targets", action="store_false")
+    ap.add_argument("--no-extras", "--no-targets", dest="extras", action="store_false",
+                    help="skip the other workloads and paths (configs, paths keys)")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
-    ap.add_argument("--workload", default="gpt2", choices=sorted(WORKLOAD_NAMES),
-                    help="timed workload (default: the GPT-2-small shape; others are for profiling)")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOAD_NAMES),
+                    help="timed workload (default: the 16K long-context causal d128 case; others are for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

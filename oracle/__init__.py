@@ -62,6 +62,7 @@ def _bind(path: str):
     lib.oracle_blockmask_csc.argtypes = [_u8p, ctypes.c_int, _i32p, _i32p]
     lib.oracle_blockmask_csc.restype = ctypes.c_int64
     lib.oracle_num_threads.restype = ctypes.c_int
+    lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
     return lib
 
 
@@ -76,6 +77,11 @@ def _load():
 def num_threads() -> int:
     """OpenMP threads the oracle uses (OMP_NUM_THREADS, else all host cores)."""
     return int(_load().oracle_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Use n OpenMP threads from now on (n >= 1)."""
+    _load().oracle_set_num_threads(int(n))
 
 
 def _f64(a):

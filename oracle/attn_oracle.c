@@ -65,6 +65,15 @@ int oracle_num_threads(void) {
 #endif
 }
 
+/* Threads of the OpenMP regions that follow (the host-baseline timing runs once on one core, once on all). */
+void oracle_set_num_threads(int n) {
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
 /* Is key c visible from query row r of sequence b? */
 static int allowed(const attn_problem *p, int b, int r, int c) {
     if (p->causal && c > r) return 0;
