@@ -41,6 +41,16 @@ namespace fa {
 #define FA_BWD_EXP_FMA_EVERY 0
 #endif
 constexpr int kBwdExpFmaEvery = FA_BWD_EXP_FMA_EVERY;
+// Per-warpgroup register budgets (setmaxnreg): the two recompute warpgroups take FA_BWD_REGS_HIGH registers a
+// thread, the drain warpgroup keeps 128 and the MMA / TMA warpgroup gives up the difference.  Measured on B200: at
+// 136 / 112 the d = 64 kernel uses no local memory (128 for all: a stack frame and spills in the recompute loop) and
+// the GPT-2 shape backward kernel goes from 388 to 403 TFLOP/s; 144 / 96 spills in the MMA / TMA warps.
+#ifndef FA_BWD_SETMAXNREG
+#define FA_BWD_SETMAXNREG 1
+#endif
+#ifndef FA_BWD_REGS_HIGH
+#define FA_BWD_REGS_HIGH 136
+#endif
 
 template <int D>
 struct BwdCfg {
@@ -311,6 +321,11 @@ __global__ void __launch_bounds__(512, 1)
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
+  // Register budgets per warpgroup when FA_BWD_SETMAXNREG is set (launched with 128 each): the recompute
+  // warpgroups hold a tile row of scores, probabilities and gradients, the MMA / TMA warpgroup needs few
+  // (kBwdRegsLow + 2 * kBwdRegsHigh + 128 = 4 x 128).  Each role changes its budget at the top of its own branch.
+  constexpr int kBwdRegsHigh = FA_BWD_REGS_HIGH, kBwdRegsLow = 512 - 128 - 2 * FA_BWD_REGS_HIGH;
+  static_assert(2 * kBwdRegsHigh + 128 + kBwdRegsLow <= 4 * 128, "register split exceeds the launch budget");
 
   // Every role walks the same unit sequence and, per unit, the same Q-tile list; counters that index barrier
   // phases and ring slots run on across units.  Units without a visible Q tile load and compute nothing (the
@@ -321,6 +336,9 @@ __global__ void __launch_bounds__(512, 1)
 
   if (warp == kWarpLoad) {
     // ------------------------------------------------------------------------------------------ TMA producer
+#if FA_BWD_SETMAXNREG
+    ptx::setmaxnreg_dec<kBwdRegsLow>();
+#endif
     if (lane == 0) {
       ptx::prefetch_tensormap(&map_q);
       ptx::prefetch_tensormap(&map_do);
@@ -377,6 +395,9 @@ __global__ void __launch_bounds__(512, 1)
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------------------------------------ MMA issuer
+#if FA_BWD_SETMAXNREG
+    ptx::setmaxnreg_dec<kBwdRegsLow>();
+#endif
     if (lane == 0) {
       constexpr uint32_t id_sq = ptx::idesc_f16(kBF16, false, false, 128, 128);  // S^T, dP^T
       constexpr uint32_t id_dv = ptx::idesc_f16(kBF16, false, true, 128, D);     // dV (A from TMEM), dK
@@ -543,6 +564,9 @@ __global__ void __launch_bounds__(512, 1)
   } else if (warp < kWarpDrain) {
     // ------------------------------------------------------------------------------------------ P^T / dS^T warps
     // Warpgroup g handles queries [64g, 64g+64) of every key row; the 4 warps of a group cover the 128 key rows.
+#if FA_BWD_SETMAXNREG
+    ptx::setmaxnreg_inc<kBwdRegsHigh>();
+#endif
     const int g = warp / 4, quarter = warp % 4;
     const int c = quarter * 32 + lane;  // key row within the tile == TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
@@ -773,6 +797,11 @@ __global__ void __launch_bounds__(512, 1)
     }
     if (lane == 0) ptx::bulk_wait_group<0>();  // all reductions performed before the CTA retires
     __syncwarp();
+  } else {
+    // ------------------------------------------------------------------------------------------ idle warps 14, 15
+#if FA_BWD_SETMAXNREG
+    ptx::setmaxnreg_dec<kBwdRegsLow>();  // every warp of the MMA / TMA warpgroup takes the same budget
+#endif
   }
 
   ptx::tc_fence_before();
@@ -820,52 +849,6 @@ cudaError_t launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   const unsigned blocks = (unsigned)std::min<long long>((total_vec8 + 255) / 256, 148LL * 16);
   bwd_dq_kernel<D, BF><<<blocks, 256, 0, st>>>(a.dq_acc, dq, a.N, Npad, total_vec8, a.cu_q, a.total_q, a.H, a.dl);
   return cudaGetLastError();
-}
-
-inline cudaError_t run_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                           const CUtensorMap& mdo, const CUtensorMap& mdq, const void* o, const void* dout, const float* lse, void* dq,
-                           void* dk, void* dv, int B, int H, int N, int d, float scale, bool causal,
-                           const int32_t* key_lens, const int32_t* col_ptr, const int32_t* row_idx, void* workspace,
-                           bool bf16, uint64_t budget_ns, cudaStream_t st, cudaEvent_t ev_start,
-                           cudaEvent_t ev_stop, const int32_t* cu_q = nullptr, const int32_t* cu_k = nullptr,
-                           int total_q = 0, int total_k = 0, int Nk = 0, long long list_head_stride = 0) {
-  // packed variable-length batches: N / Nk are the longest query / key sequences; dense: Nk = N
-  if (Nk <= 0) Nk = N;
-  const int nT = (N + kTile - 1) / kTile;
-  const int BH = B * H;
-  const size_t npad = (size_t)nT * kTile;
-  auto al = [](size_t x) { return (x + 255) / 256 * 256; };
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  BwdArgs a;
-  a.dk = dk;
-  a.dv = dv;
-  a.dq_acc = reinterpret_cast<float*>(ws);
-  a.lse2 = reinterpret_cast<const float*>(ws + al((size_t)BH * npad * d * 4));
-  a.Dv = reinterpret_cast<const float*>(ws + al((size_t)BH * npad * d * 4) + al((size_t)BH * npad * 4));
-  a.dl = d;
-  a.key_lens = key_lens;
-  a.col_ptr = col_ptr;
-  a.row_idx = row_idx;
-  a.list_head_stride = list_head_stride;
-  a.cu_q = cu_q;
-  a.cu_k = cu_k;
-  a.total_q = total_q;
-  a.total_k = total_k;
-  a.H = H;
-  a.N = N;
-  a.nT = nT;
-  a.Nk = Nk;
-  a.nTk = (Nk + kTile - 1) / kTile;
-  a.BH = BH;
-  a.causal = causal ? 1 : 0;
-  a.scale = scale;
-  a.scale_log2 = scale * 1.4426950408889634f;
-  a.budget_ns = budget_ns;
-  if (d <= 64)  // 32 runs on the 64 kernel
-    return bf16 ? launch_bwd<64, true>(mq, mk, mv, mdo, mdq, o, dout, lse, dq, a, st, ev_start, ev_stop)
-                : launch_bwd<64, false>(mq, mk, mv, mdo, mdq, o, dout, lse, dq, a, st, ev_start, ev_stop);
-  return bf16 ? launch_bwd<128, true>(mq, mk, mv, mdo, mdq, o, dout, lse, dq, a, st, ev_start, ev_stop)
-              : launch_bwd<128, false>(mq, mk, mv, mdo, mdq, o, dout, lse, dq, a, st, ev_start, ev_stop);
 }
 
 }  // namespace fa

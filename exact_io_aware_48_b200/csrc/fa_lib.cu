@@ -13,6 +13,7 @@
 #include "fa_fwd.cuh"
 #include "fa_fwd256.cuh"
 #include "fa_bwd.cuh"
+#include "fa_bwd256.cuh"
 #include "fa_mask.cuh"
 
 namespace {
@@ -49,11 +50,11 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Head dims: 64 and 128 natively; 32 and 96 run on the 64 / 128 kernels, whose TMA boxes are 64 columns wide and
-// zero-fill the columns past the tensor's own, so the extra columns add nothing to any product.
-bool head_dim_ok(int d) { return d == 32 || d == 64 || d == 96 || d == 128; }
-// The forward also runs d = 256 (its own kernel, fa_fwd256.cuh); the backward does not.
-bool fwd_head_dim_ok(int d) { return head_dim_ok(d) || d == 256; }
+// Head dims: 64, 128 and 256 natively; 32 and 96 run on the 64 / 128 kernels, whose TMA boxes are 64 columns wide
+// and zero-fill the columns past the tensor's own, so the extra columns add nothing to any product.  d = 256 has
+// its own forward (fa_fwd256.cuh) and backward (fa_bwd256.cuh) kernels.
+bool head_dim_ok(int d) { return d == 32 || d == 64 || d == 96 || d == 128 || d == 256; }
+bool fwd_head_dim_ok(int d) { return head_dim_ok(d); }
 
 int cuda_fail(cudaError_t e) {
   t_last_error = cudaGetErrorString(e);
@@ -309,9 +310,17 @@ Lists carve_lists(void* ws, int nT) {
 // Tile lists of `heads` masks ([heads][nT][nT]); head h's lists are lists_bytes(nT) bytes after head 0's.
 int launch_lists(const uint8_t* mask, int nT, const Lists& l, cudaStream_t st, int heads = 1) {
   const long long stride = heads > 1 ? (long long)(lists_bytes(nT) / 4) : 0;
-  fa::blockmask_lists_kernel<<<heads, fa::kMaskThreads, 0, st>>>(mask, nT, l.row_ptr, l.col_idx, l.col_ptr,
-                                                                 l.row_idx, stride);
+  const int row_blocks = (nT + fa::kMaskWarps - 1) / fa::kMaskWarps;
+  const int col_blocks = (nT + 32 * fa::kMaskWarps - 1) / (32 * fa::kMaskWarps);
+  const dim3 grid(row_blocks + col_blocks, heads);
+  fa::blockmask_count_kernel<<<grid, fa::kMaskWarps * 32, 0, st>>>(mask, nT, l.row_ptr, l.col_ptr, stride);
   cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  fa::blockmask_scan_kernel<<<heads, fa::kMaskThreads, 0, st>>>(nT, l.row_ptr, l.col_ptr, stride);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
+  fa::blockmask_fill_kernel<<<grid, fa::kMaskWarps * 32, 0, st>>>(mask, nT, l.row_ptr, l.col_idx, l.col_ptr,
+                                                                  l.row_idx, stride);
+  e = cudaGetLastError();
   return e == cudaSuccess ? FA_OK : cuda_fail(e);
 }
 

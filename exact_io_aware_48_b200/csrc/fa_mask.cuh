@@ -5,35 +5,59 @@
 
 namespace fa {
 
-constexpr int kMaskThreads = 1024;
+constexpr int kMaskThreads = 1024;  // threads of the prefix-scan kernel
+constexpr int kMaskWarps = 8;       // warps per CTA of the count and fill kernels
 constexpr int kMaxMaskTiles = 8192;
 
-// One CTA of 1024 threads.  Phase 1 counts kept tiles per row and per column, phase 2 turns the counts into
-// exclusive prefix sums (row_ptr, col_ptr), phase 3 writes each row's columns and each column's rows in
-// ascending order.  Integer only; the result is unique, so it must equal any correct CPU construction exactly.
-// Per-head masks: CTA h reads mask + h*nT*nT and writes lists `head_stride` int32 further on (grid = number of
-// masks; one mask shared by all heads: grid 1, stride 0).
+// Tile lists of a block mask in three launches, integer only (the result is unique, so it must equal any correct
+// CPU construction exactly):
+//   blockmask_count_kernel  kept tiles per row (one warp per row, coalesced byte loads and a warp sum) into
+//                           row_ptr[i+1], and per column (one warp per strip of 32 columns, lane = column, walking
+//                           the rows) into col_ptr[j+1]
+//   blockmask_scan_kernel   in-place prefix sums: row_ptr, col_ptr become the CSR / CSC offsets
+//   blockmask_fill_kernel   each row's kept columns in ascending order (warp ballot compaction) into col_idx, and
+//                           each column's kept rows in ascending order (the strip's lanes walk the rows in order)
+//                           into row_idx
+// The count and fill kernels take ceil(nT/8) CTAs for rows followed by ceil(nT/256) CTAs for column strips; grid.y
+// is the number of masks.  Per-head masks: mask h is at mask + h*nT*nT and its lists `head_stride` int32 further
+// on than head 0's (one mask for all heads: grid.y = 1, stride 0).
+__device__ __forceinline__ int mask_row_blocks(int nT) { return (nT + kMaskWarps - 1) / kMaskWarps; }
+
+__global__ void __launch_bounds__(kMaskWarps * 32)
+    blockmask_count_kernel(const uint8_t* __restrict__ mask, int nT, int32_t* __restrict__ row_ptr,
+                           int32_t* __restrict__ col_ptr, long long head_stride) {
+  mask += (size_t)blockIdx.y * nT * nT;
+  row_ptr += blockIdx.y * head_stride;
+  col_ptr += blockIdx.y * head_stride;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int rb = mask_row_blocks(nT);
+  if ((int)blockIdx.x < rb) {
+    const int i = blockIdx.x * kMaskWarps + warp;
+    if (i >= nT) return;
+    const uint8_t* r = mask + (size_t)i * nT;
+    int c = 0;
+    for (int x = lane; x < nT; x += 32) c += r[x] != 0;
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1) c += __shfl_xor_sync(0xffffffffu, c, m);
+    if (lane == 0) row_ptr[i + 1] = c;
+  } else {
+    const int j = ((blockIdx.x - rb) * kMaskWarps + warp) * 32 + lane;
+    if (j >= nT) return;
+    int c = 0;
+#pragma unroll 8
+    for (int x = 0; x < nT; ++x) c += mask[(size_t)x * nT + j] != 0;
+    col_ptr[j + 1] = c;
+  }
+}
+
+// One CTA per mask: counts at [1, nT] become inclusive prefix sums in place, [0] = 0.
 __global__ void __launch_bounds__(kMaskThreads, 1)
-    blockmask_lists_kernel(const uint8_t* __restrict__ mask, int nT, int32_t* __restrict__ row_ptr,
-                           int32_t* __restrict__ col_idx, int32_t* __restrict__ col_ptr,
-                           int32_t* __restrict__ row_idx, long long head_stride) {
-  mask += (size_t)blockIdx.x * nT * nT;
+    blockmask_scan_kernel(int nT, int32_t* __restrict__ row_ptr, int32_t* __restrict__ col_ptr,
+                          long long head_stride) {
   row_ptr += blockIdx.x * head_stride;
-  col_idx += blockIdx.x * head_stride;
   col_ptr += blockIdx.x * head_stride;
-  row_idx += blockIdx.x * head_stride;
   __shared__ int32_t part_r[kMaskThreads], part_c[kMaskThreads];
   const int tid = threadIdx.x;
-  for (int i = tid; i < nT; i += kMaskThreads) {
-    int cr = 0, cc = 0;
-    for (int x = 0; x < nT; ++x) {
-      cr += mask[(size_t)i * nT + x] != 0;  // row i
-      cc += mask[(size_t)x * nT + i] != 0;  // column i (coalesced across threads)
-    }
-    row_ptr[i + 1] = cr;
-    col_ptr[i + 1] = cc;
-  }
-  __syncthreads();
   // each thread owns a contiguous chunk of the counts
   const int chunk = (nT + kMaskThreads - 1) / kMaskThreads;
   const int lo = tid * chunk, hi = min(lo + chunk, nT);
@@ -52,20 +76,43 @@ __global__ void __launch_bounds__(kMaskThreads, 1)
   }
   int run_r = part_r[tid] - sr, run_c = part_c[tid] - sc;  // exclusive prefix of this chunk
   for (int i = lo; i < hi; ++i) {
-    const int cr = row_ptr[i + 1], cc = col_ptr[i + 1];
-    run_r += cr;
-    run_c += cc;
+    run_r += row_ptr[i + 1];
+    run_c += col_ptr[i + 1];
     row_ptr[i + 1] = run_r;
     col_ptr[i + 1] = run_c;
   }
   if (tid == 0) { row_ptr[0] = 0; col_ptr[0] = 0; }
-  __syncthreads();
-  for (int i = tid; i < nT; i += kMaskThreads) {
-    int pr = row_ptr[i], pc = col_ptr[i];
-    for (int x = 0; x < nT; ++x) {
-      if (mask[(size_t)i * nT + x]) col_idx[pr++] = x;
-      if (mask[(size_t)x * nT + i]) row_idx[pc++] = x;
+}
+
+__global__ void __launch_bounds__(kMaskWarps * 32)
+    blockmask_fill_kernel(const uint8_t* __restrict__ mask, int nT, const int32_t* __restrict__ row_ptr,
+                          int32_t* __restrict__ col_idx, const int32_t* __restrict__ col_ptr,
+                          int32_t* __restrict__ row_idx, long long head_stride) {
+  mask += (size_t)blockIdx.y * nT * nT;
+  row_ptr += blockIdx.y * head_stride;
+  col_idx += blockIdx.y * head_stride;
+  col_ptr += blockIdx.y * head_stride;
+  row_idx += blockIdx.y * head_stride;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int rb = mask_row_blocks(nT);
+  if ((int)blockIdx.x < rb) {
+    const int i = blockIdx.x * kMaskWarps + warp;
+    if (i >= nT) return;
+    const uint8_t* r = mask + (size_t)i * nT;
+    int pos = row_ptr[i];
+    for (int x0 = 0; x0 < nT; x0 += 32) {
+      const bool kept = x0 + lane < nT && r[x0 + lane] != 0;
+      const unsigned bal = __ballot_sync(0xffffffffu, kept);
+      if (kept) col_idx[pos + __popc(bal & ((1u << lane) - 1u))] = x0 + lane;
+      pos += __popc(bal);
     }
+  } else {
+    const int j = ((blockIdx.x - rb) * kMaskWarps + warp) * 32 + lane;
+    if (j >= nT) return;
+    int pos = col_ptr[j];
+#pragma unroll 8
+    for (int x = 0; x < nT; ++x)
+      if (mask[(size_t)x * nT + j]) row_idx[pos++] = x;
   }
 }
 

@@ -224,6 +224,18 @@ __host__ __device__ constexpr uint32_t idesc_f16(bool is_bf16, bool a_mn, bool b
          | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
 }
 
+// ------------------------------------------------------------------------------------------------ registers
+// Per-warpgroup register budget (all four warps of a warpgroup execute the same instruction).  An increase draws
+// on the registers the CTA was launched with, so the warpgroups' budgets must add up to at most that total.
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ------------------------------------------------------------------------------------------------ math
 __device__ __forceinline__ float ex2(float x) {
   float y;

@@ -90,12 +90,13 @@ def test_bwd_and_blocksparse_argument_errors(lib):
     assert _lib.fa_blockmask_lists(A, 8193, A, A, A, A, 0) == _lib.FA_ERR_INVALID_ARG
 
 
-def test_head_dim_256_is_forward_only(lib):
-    # d = 256 has a forward kernel; the backward entry points refuse it before any CUDA call
-    rc = _lib.fa_bwd(A, A, A, A, A, A, A, A, A, 1, 1, 128, 256, 0.0625, 0, None, None, A, 1 << 30, 0, 0)
+def test_head_dims_checked_before_any_cuda_call(lib):
+    # d = 256 runs forward and backward; other head dims are refused before any CUDA call
+    rc = _lib.fa_bwd(A, A, A, A, A, A, A, A, A, 1, 1, 128, 192, 0.0625, 0, None, None, A, 1 << 30, 0, 0)
     assert rc == _lib.FA_ERR_UNSUPPORTED
-    assert _lib.fa_bwd_workspace_size(1, 2, 1024, 256, False) == 0
-    assert _lib.fa_bwd_varlen_workspace_size(1, 2, 1024, 256) == 0
+    assert _lib.fa_bwd_workspace_size(1, 2, 1024, 256, False) >= 2 * 1024 * 256 * 4
+    assert _lib.fa_bwd_varlen_workspace_size(1, 2, 1024, 256) > 0
+    assert _lib.fa_bwd_workspace_size(1, 2, 1024, 192, False) == 0
     assert _lib.fa_fwd_splitkv_workspace_size(1, 2, 1, 4096, 256, 0) > 0
 
 

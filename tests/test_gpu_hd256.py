@@ -1,7 +1,10 @@
-"""Head dim 256 on the GPU (forward only: fwd256_kernel, one Q tile per CTA with two score buffers) vs the fp64
-oracle: dense forward with causal masks, key lengths (0 included), ragged tiles, more units than SMs, shared and
-per-head block masks, a packed variable-length batch and the split-K/V decode path.  Tolerance as for the other
-head dims: O and LSE max-abs <= 1e-2.  The backward refuses d = 256 (FA_ERR_UNSUPPORTED)."""
+"""Head dim 256 on the GPU vs the fp64 oracle.
+
+Forward (fwd256_kernel, one Q tile per CTA with two score buffers): dense with causal masks, key lengths (0
+included), ragged tiles, more units than SMs, shared and per-head block masks, a packed variable-length batch and the
+split-K/V decode path.  Backward (bwd256_kernel, two passes over halves of the head dim, every operand streamed in
+16 KB boxes): the same mask kinds, packed batches and runs of more units than SMs.  Tolerances as for the other head
+dims: O and LSE max-abs <= 1e-2, dQ/dK/dV max-abs <= 5e-2 of the oracle's largest gradient magnitude."""
 import numpy as np
 import pytest
 import torch
@@ -9,7 +12,7 @@ import torch
 import oracle
 import exact_io_aware_48_b200 as fa
 from exact_io_aware_48_b200 import _lib, inputs
-from parity import assert_lse_close, assert_o_close, f64, gpu_fwd, log_errors
+from parity import assert_grad_close, assert_lse_close, assert_o_close, f64, gpu_fwd, gpu_fwd_bwd, log_errors
 
 pytestmark = pytest.mark.gpu
 
@@ -95,8 +98,73 @@ def test_d256_decode(splits):
     log_errors(f"d256 decode splits={splits}", O=eo, LSE=el)
 
 
-def test_d256_backward_is_refused():
-    q, k, v, do = [inputs.gaussian((1, 1, 128, D), 795 + t, "bf16").cuda() for t in range(4)]
-    o, lse = fa.attention_fwd(q, k, v)
-    with pytest.raises(RuntimeError, match="FA_ERR_UNSUPPORTED"):
-        fa.attention_bwd(q, k, v, o, do, lse)
+BWD = [
+    # B, H, N, dtype, causal, key_lens
+    (1, 2, 128, "bf16", False, None),
+    (1, 2, 300, "bf16", True, None),
+    (2, 2, 640, "fp16", False, [640, 200]),
+    (3, 1, 129, "bf16", True, [1, 129, 0]),
+    (2, 8, 1200, "bf16", True, None),          # 320 units (key tile x half x head): several per CTA
+    (2, 16, 256, "fp16", False, [0, 256]),     # runs of units with no visible query
+]
+
+
+@pytest.mark.parametrize("B,H,N,dtype,causal,kl", BWD)
+def test_d256_backward(B, H, N, dtype, causal, kl):
+    q, k, v, do = [inputs.gaussian((B, H, N, D), 720 + N + t, dtype) for t in range(4)]
+    scale = 1.0 / np.sqrt(D)
+    kla = None if kl is None else np.array(kl, np.int32)
+    o, lse, dq, dk, dv = gpu_fwd_bwd(q, k, v, do, causal, scale, key_lens=kla)
+    rq, rk, rv, ro, rl = oracle.attn_bwd(f64(q), f64(k), f64(v), f64(do), scale, causal=causal, key_lens=kla)
+    eo = assert_o_close(o.double().numpy(), ro)
+    el = assert_lse_close(lse.numpy(), rl)
+    e = [assert_grad_close(g.double().numpy(), r, n) for g, r, n in ((dq, rq, "dQ"), (dk, rk, "dK"), (dv, rv, "dV"))]
+    log_errors(f"d256 bwd B{B} H{H} N{N} {dtype} causal={causal} kl={kl}", O=eo, LSE=el, dQ=e[0], dK=e[1], dV=e[2])
+    if kl is not None:  # keys beyond the length get exactly zero gradient
+        for b in range(B):
+            assert torch.all(dk[b, :, kl[b]:] == 0) and torch.all(dv[b, :, kl[b]:] == 0)
+
+
+def test_d256_backward_block_masks():
+    B, H, N = 1, 2, 640
+    q, k, v, do = [inputs.gaussian((B, H, N, D), 740 + t, "bf16") for t in range(4)]
+    nT = 5
+    shared = np.tril(np.ones((nT, nT), np.uint8))
+    shared[3, 1] = 0
+    shared[4, 4] = 0
+    o, lse, dq, dk, dv = gpu_fwd_bwd(q, k, v, do, True, 0.07, block_mask=shared)
+    rq, rk, rv, ro, rl = oracle.attn_bwd(f64(q), f64(k), f64(v), f64(do), 0.07, causal=True, block_mask=shared)
+    for g, r, n in ((dq, rq, "dQ"), (dk, rk, "dK"), (dv, rv, "dV")):
+        assert_grad_close(g.double().numpy(), r, n)
+    heads = np.stack([shared, (np.arange(nT)[:, None] + np.arange(nT)[None, :]) % 2 == 0]).astype(np.uint8)
+    o, lse, dq, dk, dv = gpu_fwd_bwd(q, k, v, do, False, 0.07, block_mask=heads)
+    rq, rk, rv, ro, rl = oracle.attn_bwd_head_masks(f64(q), f64(k), f64(v), f64(do), 0.07, heads)
+    for g, r, n in ((dq, rq, "dQ"), (dk, rk, "dK"), (dv, rv, "dV")):
+        assert_grad_close(g.double().numpy(), r, n)
+
+
+def test_d256_backward_packed_varlen():
+    lens = [200, 1, 129, 384]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    H = 2
+    q, k, v, do = [inputs.gaussian((int(cu[-1]), H, D), 750 + t, "bf16") for t in range(4)]
+    cud = torch.as_tensor(cu).cuda()
+    qd, kd, vd, dod = (t.cuda() for t in (q, k, v, do))
+    o, lse = fa.attention_fwd_varlen(qd, kd, vd, cud, cud, 384, 384, causal=True)
+    dq, dk, dv = fa.attention_bwd_varlen(qd, kd, vd, o, dod, lse, cud, cud, 384, 384, causal=True)
+    assert fa.last_device_status() == 0
+    rq, rk, rv, ro, rl = oracle.attn_bwd_varlen(f64(q), f64(k), f64(v), f64(do), cu, cu, 1.0 / np.sqrt(D),
+                                                causal=True)
+    e = [assert_grad_close(g.cpu().double().numpy(), r, n) for g, r, n in ((dq, rq, "dQ"), (dk, rk, "dK"),
+                                                                           (dv, rv, "dV"))]
+    log_errors("d256 bwd varlen", dQ=e[0], dK=e[1], dV=e[2])
+
+
+def test_d256_backward_repeatable():
+    # every gradient is a sum in a fixed order except dQ (fp32 reductions in L2 in arrival order)
+    q, k, v, do = [inputs.gaussian((1, 4, 900, D), 760 + t, "bf16") for t in range(4)]
+    a = gpu_fwd_bwd(q, k, v, do, True, 0.0625)
+    b = gpu_fwd_bwd(q, k, v, do, True, 0.0625)
+    for x, y in zip(a[:2] + a[3:], b[:2] + b[3:]):
+        assert torch.equal(x, y)
+    assert torch.allclose(a[2].float(), b[2].float(), rtol=0, atol=2e-2 * float(a[2].float().abs().max()))

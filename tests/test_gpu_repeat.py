@@ -1,6 +1,7 @@
 """Repeatability: a race between warps shows up as run-to-run differences.  O, LSE, dK and dV are accumulated in a
-fixed order on chip, so repeated runs on the same inputs must agree bit for bit; dQ is summed across CTAs by L2
-reductions in no fixed order, so it must agree to fp32 rounding."""
+fixed order on chip, so repeated runs on the same inputs must agree bit for bit; dQ is summed across CTAs by fp32 L2
+reductions in no fixed order, so its fp32 sums agree to rounding and its 16-bit output may differ by one unit in the
+last place: at most 2^-7 (bf16) or 2^-10 (fp16) of the largest magnitude."""
 import numpy as np
 import pytest
 import torch
@@ -33,4 +34,5 @@ def test_runs_repeat_exactly(B, H, N, d, dtype, causal, kl):
         for name, a, b in zip(("O", "LSE", "dK", "dV"), (base[0], base[1], base[3], base[4]), (r[0], r[1], r[3], r[4])):
             assert torch.equal(a, b), f"{name} differs between runs"
         scale = float(base[2].float().abs().max())
-        assert float((base[2].float() - r[2].float()).abs().max()) <= 1e-3 * max(scale, 1e-3), "dQ drifts"
+        ulp = 2.0 ** (-7 if dtype == "bf16" else -10)
+        assert float((base[2].float() - r[2].float()).abs().max()) <= ulp * max(scale, 1e-3), "dQ drifts"
