@@ -42,19 +42,12 @@ struct FwdCfg {
 };
 
 // Every kExpFmaEvery-th pair of probabilities is exponentiated on the FMA pipe (see ptx::exp2_fma); 0 = never.
-// FA_FWD_L_ROUNDED = 1 (kept) makes the running denominator l sum the 16-bit rounded probabilities that P V
-// multiplies, so O = sum(P~ V) / sum(P~) stays a convex mix of V rows even when one probability dominates a row;
-// 0 sums the fp32 probabilities before rounding (two instructions fewer per pair, 1-5% faster on B200) but then a
-// dominant probability's rounding error (up to 2^-9 relative) reaches O undivided: 1.7e-2 on a peaked-score test,
-// above the 1e-2 bound.  Measured with l rounded: 1 pair in 16 on the FMA pipe gains 1-5% (GPT-2 shape 286 -> 299
-// TFLOP/s, N = 4096 800 -> 819, N = 16384 1109 -> 1122); 1 in 4 loses 6%.
+// Measured on B200 (same box, interleaved runs): 1 pair in 16 gains 1-5% (GPT-2 shape 286 -> 299 TFLOP/s,
+// N = 4096 800 -> 819, N = 16384 1109 -> 1122); 1 in 8 gains nothing (GPT-2 shape 4% slower) and 1 in 4 loses 6%.
 #ifndef FA_FWD_EXP_FMA_EVERY
 #define FA_FWD_EXP_FMA_EVERY 16
 #endif
 constexpr int kExpFmaEvery = FA_FWD_EXP_FMA_EVERY;
-#ifndef FA_FWD_L_ROUNDED
-#define FA_FWD_L_ROUNDED 1
-#endif
 
 struct FwdArgs {
   void* o;
@@ -440,12 +433,8 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
             const float p0 = emu ? ptx::exp2_fma(x.x) : ptx::ex2(x.x);
             const float p1 = emu ? ptx::exp2_fma(x.y) : ptx::ex2(x.y);
             pk[i] = ptx::pack2<kBF16>(p0, p1);
-#if FA_FWD_L_ROUNDED
             // l sums the rounded P that P V multiplies, so O stays a convex mix of V rows
             lacc[i & 1] = ptx::add2(lacc[i & 1], ptx::unpack2<kBF16>(pk[i]));
-#else
-            lacc[i & 1] = ptx::add2(lacc[i & 1], {p0, p1});
-#endif
           }
           ptx::tmem_st32(tS + h * 32, pk);
         }

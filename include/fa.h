@@ -19,10 +19,9 @@
  *   Pointers    Device pointers, 16-byte aligned, caller-owned; the library never allocates, frees or keeps them.
  *               Scratch that a call needs is passed in as `workspace` (device memory, 256-byte aligned) of at
  *               least the size returned by the matching *_workspace_size query.
- *   Shapes      B >= 1, H >= 1, 1 <= N <= 1048576 (2^20), d in {32, 64, 96, 128} (32 and 96 run on the 64 and 128
- *               kernels with the extra columns zero, at their cost); the forward calls (fa_fwd, fa_fwd_blocksparse,
- *               fa_fwd_blocksparse_heads, fa_fwd_varlen, fa_fwd_splitkv) also take d = 256, the backward calls do
- *               not (FA_ERR_UNSUPPORTED).  B*H*N*d <= 2^34, softmax_scale finite and > 0.
+ *   Shapes      B >= 1, H >= 1, 1 <= N <= 1048576 (2^20), d in {32, 64, 96, 128, 256} (32 and 96 run on the 64
+ *               and 128 kernels with the extra columns zero, at their cost; 256 has its own forward and backward
+ *               kernels), for every call.  B*H*N*d <= 2^34, softmax_scale finite and > 0.
  *   Execution   Asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).  Inputs must stay valid
  *               until the stream reaches the work.
  *   Errors      Argument errors are detected on the host before anything is launched and returned as an
@@ -44,7 +43,7 @@ extern "C" {
 typedef enum {
   FA_OK = 0,
   FA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad shape, scale <= 0, bad dtype */
-  FA_ERR_UNSUPPORTED = 2, /* head dimension other than 32, 64, 96, 128 (or 256 for the forward calls) */
+  FA_ERR_UNSUPPORTED = 2, /* head dimension other than 32, 64, 96, 128, 256 */
   FA_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed (message: fa_last_error_string) */
   FA_ERR_TIMEOUT = 4,     /* a kernel wait ran out of its time budget (device-detected) */
   FA_ERR_WORKSPACE = 5    /* workspace missing, misaligned or smaller than the query says */
@@ -97,7 +96,9 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d, int has_block_mask);
  * dq, dk, dv [B,H,N,d] (fully overwritten).  block_mask may be NULL.  Runs a preprocessing kernel (D = rowsum(dO*O),
  * zeroed dQ accumulator), the main kernel (persistent CTAs, each walking 128-key tiles and, per tile, the visible
  * Q tiles; dK, dV accumulate on chip, dQ partial sums go into the fp32 accumulator in the workspace by bulk
- * reduce-add) and a conversion kernel for dQ.
+ * reduce-add) and a conversion kernel for dQ.  At d = 256 the main kernel makes two passes per 128-key tile, one
+ * per half of the head dimension (each recomputes the scores over the full d and produces that half of dK, dV
+ * and dQ), because one pass's dK and dV would not fit the tensor memory.
  */
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
            void* dq, void* dk, void* dv, int B, int H, int N, int d, float softmax_scale, int causal,
