@@ -40,6 +40,7 @@ WORKLOAD_NAMES = {
     "lc8k": "long-context causal fwd+bwd B1 H16 N8192 d128 bf16",
     "lc16k": "long-context causal fwd+bwd B1 H16 N16384 d128 bf16",
     "bs64k": "block-sparse fwd+bwd B1 H8 N65536 d64 fp16, 128x128 tile mask band4+butterfly+2% random",
+    "lc8k_d256": "long-context causal fwd+bwd at head dim 256 B1 H16 N8192 d256 bf16",
 }
 L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
 # workloads reported with HBM bandwidth next to TFLOP/s (short sequences: near or below the ridge point)
@@ -455,50 +456,11 @@ def measure_decode(stream, flush, hbm_gbs):
             "bytes": nbytes, "gbs": round(gbs, 1), "hbm_frac": round(gbs / hbm_gbs, 4) if hbm_gbs else None}
 
 
-def measure_d256(stream, flush, peak):
-    """Head dim 256 (its own forward and backward kernels): B1 H16 N8192 bf16 causal, the long-context shape at
-    twice the head dim.  TFLOP/s by the algorithmic convention (4*d per visible pair forward, 2.5x backward)."""
-    import torch
-    from exact_io_aware_48_b200 import _lib, inputs
-    B, H, N, d = 1, 16, 8192, 256
-    q, k, v, do = [inputs.gaussian((B, H, N, d), 510 + t, "bf16").cuda() for t in range(4)]
-    o = torch.empty_like(q)
-    lse = torch.empty((B, H, N), device="cuda", dtype=torch.float32)
-    scale = 1.0 / math.sqrt(d)
-
-    def fwd(st):
-        rc = _lib.fa_fwd(q, k, v, o, lse, B, H, N, d, scale, True, None, _lib.FA_BF16, st)
-        if rc:
-            raise RuntimeError(f"fa_fwd: {_lib.fa_status_string(rc)}")
-
-    for _ in range(3):
-        fwd(stream)
-    ms, _ = time_loop(fwd, 10, stream, flush)
-    check_status(_lib, stream, "d = 256 forward")
-    t = statistics.median(ms)
-    ff = 4 * d * B * H * (N * (N + 1) // 2)
-    out = {"workload": f"B{B} H{H} N{N} d{d} bf16 causal", "fwd_ms": round(t, 4), "fwd_tflops": round(ff / t / 1e9, 1),
-           "fwd_frac": round(ff / t / 1e9 / peak, 4) if peak else None}
-    ws_bytes = _lib.fa_bwd_workspace_size(B, H, N, d, False)
-    if ws_bytes:  # the backward takes d = 256
-        ws = torch.empty(ws_bytes, device="cuda", dtype=torch.uint8)
-        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-
-        def bwd(st):
-            rc = _lib.fa_bwd(q, k, v, o, do, lse, dq, dk, dv, B, H, N, d, scale, True, None, None, ws, ws_bytes,
-                             _lib.FA_BF16, st)
-            if rc:
-                raise RuntimeError(f"fa_bwd: {_lib.fa_status_string(rc)}")
-
-        for _ in range(3):
-            bwd(stream)
-        bms, _ = time_loop(bwd, 10, stream, flush)
-        check_status(_lib, stream, "d = 256 backward")
-        tb = statistics.median(bms)
-        out.update({"bwd_ms": round(tb, 4), "bwd_tflops": round(2.5 * ff / tb / 1e9, 1),
-                    "bwd_frac": round(2.5 * ff / tb / 1e9 / peak, 4) if peak else None,
-                    "fwd_bwd_tflops": round(3.5 * ff / (t + tb) / 1e9, 1)})
-    return out
+def measure_d256(stream, flush, peak, hbm):
+    """Head dim 256 (its own forward and backward kernels) on the long-context causal shape at twice the head dim,
+    B1 H16 N8192 bf16, through fa_fwd / fa_bwd.  TFLOP/s by the algorithmic convention (4*d per visible pair
+    forward, 2.5x backward)."""
+    return measure_config("lc8k_d256", stream, flush, peak, hbm)
 
 
 def measure_standard(stream, flush, reps=5):
@@ -624,7 +586,7 @@ def run_ours(args):
             if name not in configs:
                 configs[name] = measure_config(name, stream, flush, peak, hbm)
         extra = {"varlen": measure_varlen(stream, flush, peak), "decode": measure_decode(stream, flush, hbm),
-                 "d256": measure_d256(stream, flush, peak), "standard_vs_tiled": measure_standard(stream, flush)}
+                 "d256": measure_d256(stream, flush, peak, hbm), "standard_vs_tiled": measure_standard(stream, flush)}
     cpu = cpu_baseline(w) if rank == 0 and world == 1 and args.cpu_baseline else None
 
     if rank == 0:

@@ -133,7 +133,8 @@ class Workload:
 
 
 def workloads() -> dict[str, Workload]:
-    """The five workload shapes: tiny, GPT-2-small, BERT-large, long-context causal sweep, block-sparse."""
+    """The five workload shapes: tiny, GPT-2-small, BERT-large, long-context causal sweep, block-sparse; and the
+    long-context shape at head dim 256 for the d = 256 kernels."""
     w = {
         "tiny": Workload("tiny", 1, 2, 256, 64, "bf16", False, 0),
         "gpt2": Workload("gpt2", 8, 12, 1024, 64, "bf16", True, 1),
@@ -142,6 +143,7 @@ def workloads() -> dict[str, Workload]:
         "lc8k": Workload("lc8k", 1, 16, 8192, 128, "bf16", True, 3),
         "lc16k": Workload("lc16k", 1, 16, 16384, 128, "bf16", True, 3),
         "bs64k": Workload("bs64k", 1, 8, 65536, 64, "fp16", False, 4, blocksparse=True),
+        "lc8k_d256": Workload("lc8k_d256", 1, 16, 8192, 256, "bf16", True, 5),
     }
     return w
 

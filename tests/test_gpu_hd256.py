@@ -168,3 +168,24 @@ def test_d256_backward_repeatable():
     for x, y in zip(a[:2] + a[3:], b[:2] + b[3:]):
         assert torch.equal(x, y)
     assert torch.allclose(a[2].float(), b[2].float(), rtol=0, atol=2e-2 * float(a[2].float().abs().max()))
+
+
+def test_d256_workload_sampled():
+    # B1 H16 N8192 d256 causal at full size: O, LSE and dQ of 1024 seeded rows, dK and dV of 128 seeded keys in each
+    # of two seeded heads against the oracle; each tolerance scale is the oracle's largest sampled magnitude
+    from parity import sampled_keys
+    w = inputs.workloads()["lc8k_d256"]
+    q, k, v, do = w.tensors()
+    o, lse, dq, dk, dv = gpu_fwd_bwd(q, k, v, do, w.causal, w.scale)
+    qf, kf, vf, dof = f64(q), f64(k), f64(v), f64(do)
+    sb, sr = inputs.sample_rows(w.seed + 600, w.B * w.H, w.N, 1024)
+    ro, rl = oracle.attn_fwd_rows(qf, kf, vf, w.scale, sb, sr, causal=w.causal)
+    eo = assert_o_close(o.reshape(-1, w.N, D)[sb, sr].double().numpy(), ro)
+    el = assert_lse_close(lse.reshape(-1, w.N)[sb, sr].numpy(), rl)
+    rq = oracle.attn_bwd_rows(qf, kf, vf, dof, w.scale, sb, sr, causal=w.causal)
+    kb, kc = sampled_keys(w.seed + 700, w.B * w.H, w.N, heads=2, per_head=128)
+    rk, rv = oracle.attn_bwd_keys(qf, kf, vf, dof, w.scale, kb, kc, causal=w.causal)
+    e_q = assert_grad_close(dq.reshape(-1, w.N, D)[sb, sr].double().numpy(), rq, "dQ")
+    e_k = assert_grad_close(dk.reshape(-1, w.N, D)[kb, kc].double().numpy(), rk, "dK")
+    e_v = assert_grad_close(dv.reshape(-1, w.N, D)[kb, kc].double().numpy(), rv, "dV")
+    log_errors("d256 lc8k sampled", O=eo, LSE=el, dQ=e_q, dK=e_k, dV=e_v)
