@@ -9,6 +9,13 @@ from exact_io_aware_48_b200 import inputs
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
+def test_recorded_traffic_matches_the_current_sources():
+    # the committed record was taken on the kernel sources as they are now (any kernel edit must retake it)
+    with open(os.path.join(ROOT, "profiles", "kernel_traffic.json")) as f:
+        rec = json.load(f)
+    assert rec["src_hash"] == bench.kernel_src_hash()
+
+
 def test_algorithmic_bwd_bytes_closed_form():
     # GPT-2 shape B8 H12 N1024 d64: Q, K, V, dO read and dK, dV written (6 tensors of B*H*N*d 16-bit values) plus
     # the fp32 LSE2 and D rows of the 128-padded row space
@@ -19,12 +26,12 @@ def test_algorithmic_bwd_bytes_closed_form():
 def test_recorded_traffic_is_gated_by_the_source_hash(monkeypatch):
     with open(os.path.join(ROOT, "profiles", "kernel_traffic.json")) as f:
         rec = json.load(f)
-    e = rec["gpt2"]["bwd_kernel<64,bf16>"]
+    e = rec["lc16k"]["bwd_kernel<128,bf16>"]
     monkeypatch.setattr(bench, "kernel_src_hash", lambda: rec["src_hash"])
-    assert bench.recorded_traffic("gpt2", "bwd_kernel<64,bf16>") == e["read"] + e["write"]
-    assert bench.recorded_traffic("gpt2", "no_such_kernel") is None
+    assert bench.recorded_traffic("lc16k", "bwd_kernel<128,bf16>") == e["read"] + e["write"]
+    assert bench.recorded_traffic("lc16k", "no_such_kernel") is None
     monkeypatch.setattr(bench, "kernel_src_hash", lambda: "0" * 16)
-    assert bench.recorded_traffic("gpt2", "bwd_kernel<64,bf16>") is None
+    assert bench.recorded_traffic("lc16k", "bwd_kernel<128,bf16>") is None
 
 
 def test_peaks_come_from_the_measured_file():
