@@ -574,7 +574,7 @@ def run_ours(args):
                 "traffic": recorded_traffic(w.name, kname), "traffic_unit": "bytes per launch (ncu DRAM read+write)",
                 "algorithmic_bytes": algorithmic_bwd_bytes(w)}
     # ------------------------------------------------------------------ end to end through the C ABI, host buffers
-    e2e = run_e2e(p, stream, args, world) if args.e2e else None
+    e2e = run_e2e(p, stream, args, world, chunks=args.e2e_chunks) if args.e2e else None
 
     configs = extra = None
     if args.extras and rank == 0:
@@ -620,42 +620,132 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def run_e2e(p, stream, args, world):
+def run_e2e(p, stream, args, world, chunks=4):
     """Same metric through the public C ABI with host buffers: per step, copy q, k, v, dO from pinned host memory,
-    run the forward and backward, copy O, LSE, dQ, dK, dV back to pinned host memory; device-timed on the stream."""
+    run the forward and backward, copy O, LSE, dQ, dK, dV back to pinned host memory; device-timed.
+
+    Heads are independent, so a caller with host data can overlap the copies with the compute: the batch is cut
+    into `chunks` groups of batch entries (or of heads when B = 1), each group's inputs go up on one stream, its
+    fa_fwd / fa_bwd calls run on the compute stream as soon as its inputs have landed, and its outputs come back on a
+    third stream while the next group computes.  Every byte of the step still crosses PCIe inside the timed region.
+    The serial form (all inputs, then compute, then all outputs) is timed too and reported beside it."""
     import torch
+    w, L = p.w, p.lib
     outs = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (p.o, p.lse, p.dq, p.dk, p.dv)]
     h2d = sum(t.numel() * t.element_size() for t in p.host)
     d2h = sum(t.numel() * t.element_size() for t in outs)
+    dev_in, dev_out = (p.q, p.k, p.v, p.do), (p.o, p.lse, p.dq, p.dk, p.dv)
+    if w.B >= chunks and w.B % chunks == 0:
+        axis = 0
+    elif w.B == 1 and w.H % chunks == 0:
+        axis = 1
+    else:
+        axis, chunks = 0, 1
+    Bc, Hc = (w.B // chunks, w.H) if axis == 0 else (w.B, w.H // chunks)
 
-    def e2e_step(s):
-        for dst, src in zip((p.q, p.k, p.v, p.do), p.host):
+    def part(t, c):  # group c of a [B, H, ...] tensor: contiguous, 16-byte aligned
+        n = t.shape[axis] // chunks
+        return t.narrow(axis, c * n, n)
+
+    def compute(c, st):
+        q, k, v, do = (part(t, c) for t in dev_in)
+        o, lse, dq, dk, dv = (part(t, c) for t in dev_out)
+        kl = p.kl if (p.kl is None or axis == 1) else p.kl[c * Bc:(c + 1) * Bc]
+        if p.bm is None:
+            rc = L.fa_fwd(q, k, v, o, lse, Bc, Hc, w.N, w.d, w.scale, w.causal, kl, p.dt, st)
+        else:
+            rc = L.fa_fwd_blocksparse(q, k, v, o, lse, Bc, Hc, w.N, w.d, w.scale, w.causal, kl, p.bm, p.fws,
+                                      p.fws_bytes, p.dt, st)
+        if rc:
+            raise RuntimeError(f"forward: {L.fa_status_string(rc)}")
+        rc = L.fa_bwd(q, k, v, o, do, lse, dq, dk, dv, Bc, Hc, w.N, w.d, w.scale, w.causal, kl, p.bm, p.ws,
+                      p.ws_bytes, p.dt, st)
+        if rc:
+            raise RuntimeError(f"fa_bwd: {L.fa_status_string(rc)}")
+
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()
+    state = {"comp": [None] * chunks, "out": [None] * chunks}
+
+    def step():
+        ins = []
+        for c in range(chunks):
+            if state["comp"][c] is not None:
+                s_in.wait_event(state["comp"][c])  # the previous step's compute has read this group's inputs
+            with torch.cuda.stream(s_in):
+                for dst, src in zip(dev_in, p.host):
+                    part(dst, c).copy_(part(src, c), non_blocking=True)
+            e = ev()
+            e.record(s_in)
+            ins.append(e)
+        for c in range(chunks):
+            stream.wait_event(ins[c])
+            if state["out"][c] is not None:
+                stream.wait_event(state["out"][c])  # the previous step's outputs of this group have left
+            compute(c, stream)
+            e = ev()
+            e.record(stream)
+            state["comp"][c] = e
+            s_out.wait_event(e)
+            with torch.cuda.stream(s_out):
+                for dst, src in zip(outs, dev_out):
+                    part(dst, c).copy_(part(src, c), non_blocking=True)
+            e2 = ev()
+            e2.record(s_out)
+            state["out"][c] = e2
+
+    def serial_step(s):
+        for dst, src in zip(dev_in, p.host):
             dst.copy_(src, non_blocking=True)
         p.step(s)
-        for dst, src in zip(outs, (p.o, p.lse, p.dq, p.dk, p.dv)):
+        for dst, src in zip(outs, dev_out):
             dst.copy_(src, non_blocking=True)
 
-    with torch.cuda.stream(stream):
-        for _ in range(2):
-            e2e_step(stream)
-    stream.synchronize()
     n = max(5, args.steps // 4)
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        ev0.record(stream)
+
+    def timed(run):
+        for _ in range(2):
+            run()
+        torch.cuda.synchronize()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record(s_in)
+        s_in.wait_event(ev0)
         for _ in range(n):
-            e2e_step(stream)
-        ev1.record(stream)
-    stream.synchronize()
-    ms = ev0.elapsed_time(ev1) / n
+            run()
+        for s_ in (s_in, stream):
+            e = ev()
+            e.record(s_)
+            s_out.wait_event(e)
+        ev1.record(s_out)
+        torch.cuda.synchronize()
+        return ev0.elapsed_time(ev1) / n
+
+    def serial():
+        with torch.cuda.stream(s_in):
+            serial_step(s_in)
+
+    ms_serial = timed(serial)
+    ref = [t.clone() for t in outs]  # the unchunked step's results
+    ms = timed(step)
+    check_status(L, stream, "end-to-end steps")
+    for name, a, b in zip(("O", "LSE", "dQ", "dK", "dV"), ref, outs):  # chunking must not change the results
+        if name == "dQ":  # fp32 reductions in run-dependent order: one 16-bit unit in the last place at most
+            ok = float((a.float() - b.float()).abs().max()) <= 2.0 ** -7 * max(float(a.float().abs().max()), 1e-3)
+        else:
+            ok = torch.equal(a, b)
+        if not ok:
+            raise RuntimeError(f"end-to-end: {name} of the overlapped steps differs from the unchunked step")
     if world > 1:
         import torch.distributed as dist
-        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
+        t = torch.tensor([ms, ms_serial], device="cuda", dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+        ms, ms_serial = float(t[0].item()), float(t[1].item())
     val = world * 3.5 * p.fwd_flops / (ms / 1e3) / 1e12
     return {"value": round(val, 3), "unit": "TFLOP/s", "ms_per_step": round(ms, 4), "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h}
+            "d2h_bytes_per_step": d2h, "overlap": f"{chunks} groups of {'batch entries' if axis == 0 else 'heads'}, "
+            "copies in, compute and copies out on three streams",
+            "serial_ms_per_step": round(ms_serial, 4),
+            "serial_value": round(world * 3.5 * p.fwd_flops / (ms_serial / 1e3) / 1e12, 3)}
 
 
 # ---------------------------------------------------------------------------------------------- CPU oracle
@@ -794,6 +884,8 @@ def main():
                     help="skip the other workloads and paths (configs, paths keys)")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
+    ap.add_argument("--e2e-chunks", type=int, default=4,
+                    help="groups of batch entries (or heads when B = 1) whose copies overlap the compute in e2e")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOAD_NAMES),
                     help="timed workload (default: the 16K long-context causal d128 case; others are for profiling)")
     args = ap.parse_args()
