@@ -12,17 +12,19 @@
 //     and sends dQ[:, half h] = scale * dS K[:, half h] to the fp32 accumulator.  The two passes together give every
 //     column once; S^T and dP^T are computed twice (29.4 instead of 21 MFLOP of products per tile pair and pass
 //     pair: 5/7 of the work is the algorithmic 2.5x forward).
-//   * Every operand streams through one ring of 16 KB boxes (128 rows x 64 columns, 128-byte swizzle) in exactly
-//     the order the MMA thread consumes them, and each box is released after its single use, so no box is ever
-//     held while later ones wait for its slot.  Per Q tile i of a unit:
-//         S^T  : (K box c, Q box c) for c = 0..3              8 boxes, contraction over d in four steps of 64
+//   * The key tile K_j (four 16 KB boxes of 128 rows x 64 columns) stays resident for the unit: it is the A operand
+//     of every S^T and the B operand of every dQ_h.  Every other operand streams through one ring of 16 KB boxes in
+//     exactly the order the MMA thread consumes them, and each box is released after its single use, so no box is
+//     ever held while later ones wait for its slot.  Per Q tile i of a unit:
+//         S^T  : Q box c for c = 0..3 (A = resident K box c)   4 boxes, contraction over d in four steps of 64
 //         dP^T : (V box c, dO box c) for c = 0..3             8 boxes
 //         dV_h : dO boxes 2h, 2h+1                            2 boxes, one N = 128 operand
-//         dQ_h : K boxes 2h, 2h+1                             2 boxes
+//         dQ_h : (resident K boxes 2h, 2h+1)                  0 boxes
 //         dK_h : Q boxes 2h, 2h+1                             2 boxes
 //     in the MMA order S^T_first, then per i: dP^T_i [P^T_i] dV_i, S^T_{i+1} [dS^T_i] dQ_i, dK_i.  Every pair starts
 //     at an even box position and the ring has an even number of slots, so the two boxes of a pair always sit in
-//     adjacent slots 16 KB apart (the N-chunk stride of their shared-memory descriptor).
+//     adjacent slots 16 KB apart (the N-chunk stride of their shared-memory descriptor).  The next unit's K waits
+//     until every MMA of the current unit has completed.
 //   The LSE2 / D rows of each Q tile come through a separate two-entry ring.
 // TMEM (512 columns): S^T [0,128); dP^T [128,256); dV_h [256,384); dK_h [384,512); P^T (16-bit pairs) over the S^T
 // columns it replaces ([0,32) and [64,96)); dQ_h in the dP^T columns once they have been read.
@@ -36,11 +38,12 @@ struct Bwd256Cfg {
   static constexpr int kHalf = 128;                    // head-dim columns per pass
   static constexpr int kBoxBytes = kTile * 64 * 2;     // 16 KB: 128 rows x 64 columns
   static constexpr int kBoxes = D / 64;                // column boxes of a 128 x 256 tile
-  static constexpr int kNumSlots = 10;                 // even, so a box pair never wraps around the ring
+  static constexpr int kKBytes = 4 * kTile * 64 * 2;   // resident K tile: four boxes
+  static constexpr int kNumSlots = 6;                  // even, so a box pair never wraps around the ring
   static constexpr int kLdSlots = 2;                   // LSE2 / D rows of a Q tile, 1 KB each
   static constexpr int kDsBytes = kTile * kTile * 2;   // dS^T, 128 keys x 128 queries
   static constexpr int kStageBytes = 4 * 4096;         // dQ staging: one 32 x 32 fp32 box per drain warp
-  static constexpr int kSmemBytes = kNumSlots * kBoxBytes + kDsBytes + kStageBytes + kLdSlots * 1024 + 1024;
+  static constexpr int kSmemBytes = kKBytes + kNumSlots * kBoxBytes + kDsBytes + kStageBytes + kLdSlots * 1024 + 1024;
   static constexpr int kThreads = 512;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 384, kColDQ = 128;
@@ -58,14 +61,15 @@ __global__ void __launch_bounds__(512, 1)
   constexpr int NS = C::kNumSlots;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sRing = smem;
+  uint8_t* sK = smem;
+  uint8_t* sRing = sK + C::kKBytes;
   uint8_t* sDS = sRing + NS * C::kBoxBytes;
   uint8_t* sStage = sDS + C::kDsBytes;
   uint8_t* sLd = sStage + C::kStageBytes;
 
   __shared__ __align__(8) uint64_t bar_full[NS], bar_empty[NS], bar_ld_full[C::kLdSlots], bar_ld_empty[C::kLdSlots],
       bar_s, bar_dp, bar_p, bar_ds, bar_dq_full, bar_dq_free, bar_ds_free, bar_dv_done, bar_done, bar_dv_free,
-      bar_dk_free, bar_drain;
+      bar_dk_free, bar_drain, bar_kfull, bar_kfree;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
   volatile int* abortp = &abort_flag;
@@ -98,6 +102,8 @@ __global__ void __launch_bounds__(512, 1)
     ptx::mbar_init(ptx::smem_addr(&bar_dv_free), 128);
     ptx::mbar_init(ptx::smem_addr(&bar_dk_free), 128);
     ptx::mbar_init(ptx::smem_addr(&bar_drain), 1);
+    ptx::mbar_init(ptx::smem_addr(&bar_kfull), 1);
+    ptx::mbar_init(ptx::smem_addr(&bar_kfree), 1);
     abort_flag = 0;
     ptx::fence_barrier_init();
   }
@@ -136,7 +142,7 @@ __global__ void __launch_bounds__(512, 1)
       ptx::prefetch_tensormap(&map_do);
       ptx::prefetch_tensormap(&map_k);
       ptx::prefetch_tensormap(&map_v);
-      int nb = 0, gl = 0;
+      int nb = 0, gl = 0, ku = 0;
       bool ok = true;
       while (ok && us.next(L)) {
         int half;
@@ -172,19 +178,33 @@ __global__ void __launch_bounds__(512, 1)
             if (!box(ma, c, ra, ba) || !box(mb, c, rb, bb)) return false;
           return true;
         };
+        auto qboxes = [&](int row, int base) -> bool {  // the four Q boxes of one S^T (K is resident)
+          for (int c = 0; c < C::kBoxes; ++c)
+            if (!box(&map_q, c, row, base)) return false;
+          return true;
+        };
         auto pair = [&](const CUtensorMap* m, int row, int base) -> bool {
           return box(m, 2 * half, row, base) && box(m, 2 * half + 1, row, base);
         };
         const int krow = u.j * kTile;
         int i, inext;
         bool have = it.next(i);
-        ok = ld_rows(i) && scores(&map_k, krow, u.g.k0, &map_q, i * kTile, u.g.q0);
+        ok = ld_rows(i) && qboxes(i * kTile, u.g.q0);
+        // the resident K tile, once every MMA of the previous unit has completed (the first Q boxes are already
+        // on their way, so the MMA pipe only waits for K itself)
+        if (ok && ku > 0) ok = wait_or_abort(ptx::smem_addr(&bar_kfree), (ku - 1) & 1, args.budget_ns, abortp);
+        if (ok) {
+          const uint32_t bk = ptx::smem_addr(&bar_kfull);
+          ptx::mbar_arrive_expect_tx(bk, C::kKBytes);
+          for (int c = 0; c < C::kBoxes; ++c)
+            tma_rows(ptx::smem_addr(sK + c * C::kBoxBytes), &map_k, c, krow, u.g.k0, u.bh, u.h, packed, bk);
+          ++ku;
+        }
         while (ok && have) {
           const bool have_next = it.next(inext);
           ok = scores(&map_v, krow, u.g.k0, &map_do, i * kTile, u.g.q0) && pair(&map_do, i * kTile, u.g.q0);
-          if (ok && have_next)
-            ok = ld_rows(inext) && scores(&map_k, krow, u.g.k0, &map_q, inext * kTile, u.g.q0);
-          if (ok) ok = pair(&map_k, krow, u.g.k0) && pair(&map_q, i * kTile, u.g.q0);
+          if (ok && have_next) ok = ld_rows(inext) && qboxes(inext * kTile, u.g.q0);
+          if (ok) ok = pair(&map_q, i * kTile, u.g.q0);
           have = have_next;
           i = inext;
         }
@@ -194,6 +214,7 @@ __global__ void __launch_bounds__(512, 1)
         ptx::mbar_wait(ptx::smem_addr(&bar_full[k % NS]), (k / NS) & 1, args.budget_ns);
       for (int k = (gl > C::kLdSlots ? gl - C::kLdSlots : 0); k < gl; ++k)
         ptx::mbar_wait(ptx::smem_addr(&bar_ld_full[k % C::kLdSlots]), (k / C::kLdSlots) & 1, args.budget_ns);
+      if (ku > 0) ptx::mbar_wait(ptx::smem_addr(&bar_kfull), (ku - 1) & 1, args.budget_ns);
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------------------------------------ MMA issuer
@@ -207,6 +228,7 @@ __global__ void __launch_bounds__(512, 1)
       const uint64_t dds_k = ptx::sw128_desc(ptx::smem_addr(sDS), 16, 1024);      // dS^T, K-major (dK)
       const uint64_t dds_mn = ptx::sw128_desc(ptx::smem_addr(sDS), 16384, 1024);  // dS, M-major (dQ)
       const uint64_t ring_k = ptx::sw128_desc(ptx::smem_addr(sRing), 16, 1024);   // a box, K-major
+      const uint64_t k_k = ptx::sw128_desc(ptx::smem_addr(sK), 16, 1024);         // resident K box, K-major
       // a box pair (adjacent slots), M/N-major: 64-element N chunks one slot (16 KB) apart
       const uint64_t ring_mn = ptx::sw128_desc(ptx::smem_addr(sRing), C::kBoxBytes, 1024);
       constexpr auto kstep = [](int kk) { return (uint32_t)((kk / 4) * 16384 + (kk % 4) * 32); };
@@ -234,6 +256,21 @@ __global__ void __launch_bounds__(512, 1)
         ptx::mma_commit(ptx::smem_addr(&bar));
         return true;
       };
+      // S^T = K Q^T over d = 256: A = resident K box c, B = the next ring box (Q box c), both K-major
+      auto scores_k = [&]() -> bool {
+        for (int c = 0; c < C::kBoxes; ++c) {
+          if (!take(nb)) return false;
+          const uint64_t da = ptx::desc_advance(k_k, c * C::kBoxBytes), db = ptx::desc_advance(ring_k, off(nb));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            ptx::mma_ss(tmem + C::kColS, ptx::desc_advance(da, kk * 32), ptx::desc_advance(db, kk * 32), id_sq,
+                        (c > 0 || kk > 0) ? 1u : 0u);
+          release(nb);
+          nb += 1;
+        }
+        ptx::mma_commit(ptx::smem_addr(&bar_s));
+        return true;
+      };
       // dV_h += P^T dO[:, h]  (P^T from TMEM, the dO pair as one N = 128 M/N-major operand)
       auto issue_dv = [&](bool first) -> bool {
         if (!take(nb) || !take(nb + 1)) return false;
@@ -247,19 +284,15 @@ __global__ void __launch_bounds__(512, 1)
         nb += 2;
         return true;
       };
-      // dQ_h = dS K[:, h]  (dS read M-major from the dS^T tile, the K pair as one N = 128 operand)
-      auto issue_dq = [&]() -> bool {
-        if (!take(nb) || !take(nb + 1)) return false;
-        const uint64_t db = ptx::desc_advance(ring_mn, off(nb));
+      // dQ_h = dS K[:, h]  (dS read M-major from the dS^T tile; resident K boxes 2h, 2h+1 as one N = 128 operand)
+      auto issue_dq = [&](int half) {
+        const uint64_t db =
+            ptx::desc_advance(ptx::sw128_desc(ptx::smem_addr(sK), C::kBoxBytes, 1024), 2 * half * C::kBoxBytes);
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)
           ptx::mma_ss(tmem + C::kColDQ, ptx::desc_advance(dds_mn, kk * 2048), ptx::desc_advance(db, kk * 2048), id_dq,
                       kk > 0 ? 1u : 0u);
         ptx::mma_commit(ptx::smem_addr(&bar_dq_full));
-        release(nb);
-        release(nb + 1);
-        nb += 2;
-        return true;
       };
       // dK_h += dS^T Q[:, h]  (dS^T K-major, the Q pair as one N = 128 operand)
       auto issue_dk = [&](bool first) -> bool {
@@ -290,7 +323,9 @@ __global__ void __launch_bounds__(512, 1)
         };
         int i, li = 0;
         bool have = it.next(i);
-        if (!(ok = scores(C::kColS, bar_s))) break;
+        if (!(ok = wait_or_abort(ptx::smem_addr(&bar_kfull), ku & 1, args.budget_ns, abortp))) break;
+        ptx::tc_fence_after();
+        if (!(ok = scores_k())) break;
         while (ok && have) {
           const uint32_t ph = gi & 1, ph_prev = (gi - 1) & 1;
           // dP^T_i lands in the columns that held dQ_{i-1}: wait until the drain warps have read it
@@ -305,10 +340,10 @@ __global__ void __launch_bounds__(512, 1)
           const bool have_next = it.next(inext);
           if (!have_next) ptx::mma_commit(ptx::smem_addr(&bar_dv_done));  // this unit's dV_h is final
           // S^T_{i+1} overwrites P^T_i only after dV_i has read it (MMAs complete in issue order)
-          if (have_next && !(ok = scores(C::kColS, bar_s))) break;
+          if (have_next && !(ok = scores_k())) break;
           if (!(ok = wait_or_abort(ptx::smem_addr(&bar_ds), ph, args.budget_ns, abortp))) break;
           ptx::tc_fence_after();
-          if (!(ok = issue_dq())) break;
+          issue_dq(half);
           if (li == 0 && !(ok = acc_ready(bar_dk_free))) break;
           if (!(ok = issue_dk(li == 0))) break;
           ptx::mma_commit(ptx::smem_addr(&bar_ds_free));
@@ -318,7 +353,8 @@ __global__ void __launch_bounds__(512, 1)
           i = inext;
         }
         if (!ok) break;
-        ptx::mma_commit(ptx::smem_addr(&bar_done));  // dK_h of this unit is final (and every MMA before it)
+        ptx::mma_commit(ptx::smem_addr(&bar_done));   // dK_h of this unit is final (and every MMA before it)
+        ptx::mma_commit(ptx::smem_addr(&bar_kfree));  // the resident K tile is no longer read
         ++ku;
       }
       ptx::mma_commit(ptx::smem_addr(&bar_drain));
