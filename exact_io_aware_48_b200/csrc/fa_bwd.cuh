@@ -7,9 +7,10 @@
 //     dQ = scale * dS K,  dK = scale * dS^T Q.
 //
 // Three launches:
-//   bwd_pre_kernel   D_r = sum_j dO_rj O_rj (fp32) and LSE in base 2 for every row of a 128-padded row space,
-//                    stored as -scale * D_r and -LSE2_r (padded rows and rows with no visible key get -LSE2 = -inf,
-//                    so their recomputed P is exactly 0); zeroes the fp32 dQ accumulator.  HBM-bound.
+//   bwd_pre_kernel   D_r = sum_j dO_rj O_rj (fp32) for every row of a 128-padded row space; stores, per row, the
+//                    fold rows of -LSE_r / scale and -D_r (three 16-bit parts each, see Fold) that the tensor core
+//                    adds to S^T and dP^T (padded rows and rows with no visible key get the masked row, so their
+//                    recomputed P is exactly 0); zeroes the fp32 dQ accumulator.  HBM-bound.
 //   bwd_kernel       persistent, at most one CTA per SM; each CTA walks a share of the units (128-key tile j of
 //                    one (b, h)) and, per unit, loops over the visible 128-row Q tiles i.
 //                    Five tcgen05 GEMMs per (i, j): S^T = K Q^T and dP^T = V dO^T (recompute), dV += P^T dO (P^T read
@@ -56,13 +57,21 @@ template <int D>
 struct BwdCfg {
   static_assert(D == 64 || D == 128, "head dim");
   static constexpr int kTileBytes = kTile * D * 2;       // 128 x D 16-bit tile
-  static constexpr int kSlotBytes = kTileBytes + 1024;   // Q or dO tile, plus 128 LSE2 + 128 D floats (Q slots)
+  static constexpr int kAugBytes = kTile * 16;           // 128 rows x 8 16-bit values: the tile's fold operand
+  static constexpr int kSlotBytes = kTileBytes + kAugBytes;  // Q tile + its LSE fold rows, or dO tile + its D rows
   static constexpr int kSubTiles = D / 64;
-  static constexpr int kNumSlots = D == 128 ? 3 : 6;
+  // Two rings of tile slots: Q tiles in kQSlots, dO tiles in kDoSlots (slots [kQSlots, kNumSlots)).  A dO slot is
+  // freed by dV_i, early in tile i, so with d = 128 even one dO slot loads dO_{i+1} while S^T_{i+1}, dQ_i and dK_i
+  // run; the Q slots are freed by the last MMA of their tile (dK_i), so they need the second slot.
+  static constexpr int kQSlots = D == 128 ? 2 : 3;
+  static constexpr int kDoSlots = D == 128 ? 1 : 3;
+  static constexpr int kNumSlots = kQSlots + kDoSlots;
   static constexpr int kDsBytes = kTile * kTile * 2;      // dS^T, 128 keys x 128 queries
   static constexpr int kStageBytes = 4 * 4096;             // dQ staging: one 32 x 32 fp32 box per drain warp
   static constexpr int kKvBufs = D == 64 ? 2 : 1;           // K/V tile buffers: d = 64 prefetches the next unit's
-  static constexpr int kSmemBytes = kKvBufs * 2 * kTileBytes + kDsBytes + kNumSlots * kSlotBytes + kStageBytes + 1024;
+  static constexpr int kOnesBytes = 2048;  // the fold's constant A operand (one core-matrix pair used, rest zero)
+  static constexpr int kSmemBytes =
+      kKvBufs * 2 * kTileBytes + kDsBytes + kNumSlots * kSlotBytes + kStageBytes + kOnesBytes + 1024;
   static constexpr int kThreads = 512;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
@@ -74,20 +83,22 @@ struct BwdCfg {
   static constexpr uint32_t kPtHalf = kDqOwnCols ? 32 : 64;  // column distance between the two query halves
 };
 
-// Workspace layout: dq_acc [BH][Npad][D] fp32 | nlse2 [BH][Npad] fp32 (-LSE in base 2) | nDv [BH][Npad] fp32
-// (-softmax_scale * D), each 256-B aligned
+// Per-row side data of the backward, in bytes: d <= 128 keeps, per padded row, the two fold rows of 8 16-bit
+// values each (-LSE/scale and -D, split in three; see bwd_pre_kernel); d = 256 keeps -LSE2 and -scale * D as fp32.
+inline size_t bwd_row_side_bytes(int d) { return d <= 128 ? 16 : 4; }
+// Workspace layout: dq_acc [BH][Npad][d] fp32 | LSE side [BH][Npad] | D side [BH][Npad], each 256-B aligned
 inline size_t bwd_workspace_bytes(int BH, int nT, int d) {
   const size_t npad = (size_t)nT * kTile;
   auto al = [](size_t x) { return (x + 255) / 256 * 256; };
-  return al((size_t)BH * npad * d * 4) + 2 * al((size_t)BH * npad * 4);
+  return al((size_t)BH * npad * d * 4) + 2 * al((size_t)BH * npad * bwd_row_side_bytes(d));
 }
 
 struct BwdArgs {
   void* dk;
   void* dv;
   float* dq_acc;
-  const float* lse2;  // -LSE2 per padded row
-  const float* Dv;    // -scale * D per padded row
+  const float* lse2;  // d = 256: -LSE2 per padded row;  d <= 128: the LSE fold rows (16 bytes per padded row)
+  const float* Dv;    // d = 256: -scale * D per padded row;  d <= 128: the D fold rows
   const int32_t* key_lens;
   const int32_t* col_ptr;  // CSC of the block mask (nullptr: dense)
   const int32_t* row_idx;
@@ -149,6 +160,32 @@ struct ColTileIter {
 // 16-byte stores.  Grid-stride over all padded rows of all heads.  Packed variable-length batches (cu_q non-null):
 // O, dO are [total_q, H, d] and LSE [H, total_q]; the padded row space stays per (b, h), rows past the sequence's
 // length get -LSE2 = -inf like padding.
+// The fold (d <= 128).  The per-query terms of the recompute, -LSE_r / scale in the scores and -D_r in dP, are added
+// by the tensor core: one more K = 16 step of S^T = K Q^T (and of dP^T = V dO^T) whose A operand holds the constant
+// kFoldScale in columns 0-2 of every key row and whose B operand holds, for query r, the value w_r = x_r /
+// kFoldScale split into three 16-bit parts (w = hi + mid + lo to about 24 bits) in columns 0-2.  The accumulator
+// then holds S + x_r (fp32), so the P^T / dS^T warps need no per-query operand at all.  kFoldScale = 1 for bf16;
+// 256 for fp16, whose 16-bit range would otherwise end at |x| = 65504 (beyond 256 * 65504 the fp16 fold saturates).
+// Rows with no visible key (padding, fully masked rows) get w = -kFoldMasked: their P is exp2 of a huge negative
+// number, exactly 0.
+template <bool kBF16>
+struct Fold {
+  static constexpr float kScale = kBF16 ? 1.f : 256.f;
+  static constexpr float kMasked = kBF16 ? 0x1p100f : 65504.f;
+  static constexpr float kMax = kBF16 ? 3.0e38f : 65504.f;
+  // 16 bytes: {hi, mid, lo, 0, 0, 0, 0, 0} of x / kScale
+  static __device__ __forceinline__ uint4 row(float x) {
+    const float w = fminf(fmaxf(x * (1.f / kScale), -kMax), kMax);
+    const float hi = ptx::unpack2<kBF16>(ptx::pack2<kBF16>(w, 0.f)).x;
+    const float r1 = w - hi;  // exact: hi is w rounded to fewer significand bits
+    const float mid = ptx::unpack2<kBF16>(ptx::pack2<kBF16>(r1, 0.f)).x;
+    return make_uint4(ptx::pack2<kBF16>(hi, mid), ptx::pack2<kBF16>(r1 - mid, 0.f), 0u, 0u);
+  }
+  static __device__ __forceinline__ uint4 masked_row() {
+    return make_uint4(ptx::pack2<kBF16>(-kMasked, 0.f), 0u, 0u, 0u);
+  }
+};
+
 template <int D, bool kBF16>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const void* __restrict__ o, const void* __restrict__ dout,
                                                       const float* __restrict__ lse, float* __restrict__ dq_acc,
@@ -192,13 +229,16 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const void* __restrict__ o
         acc[2 * l + 1] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
       if (l == 0) {
-        float nl2 = -INFINITY;  // padded row or no visible key: recomputed P = exp2(x - inf) = 0
-        if (valid) {
-          const float lv = lse[cu_q ? (size_t)(bh % H) * total_q + g.q0 + r : (size_t)bh * N + r];
-          if (lv != -INFINITY) nl2 = -lv * 1.4426950408889634f;
+        const float lv = valid ? lse[cu_q ? (size_t)(bh % H) * total_q + g.q0 + r : (size_t)bh * N + r] : -INFINITY;
+        if constexpr (D <= 128) {
+          // the fold rows: -LSE / scale and -D (padded row or no visible key: the masked row, P = 0)
+          reinterpret_cast<uint4*>(lse2)[row] = lv != -INFINITY ? Fold<kBF16>::row(-lv / scale) : Fold<kBF16>::masked_row();
+          reinterpret_cast<uint4*>(Dv)[row] = Fold<kBF16>::row(-dsum);
+        } else {
+          // padded row or no visible key: recomputed P = exp2(x - inf) = 0
+          lse2[row] = lv != -INFINITY ? -lv * 1.4426950408889634f : -INFINITY;
+          Dv[row] = -scale * dsum;
         }
-        lse2[row] = nl2;
-        Dv[row] = -scale * dsum;
       }
     }
   }
@@ -263,12 +303,18 @@ __global__ void __launch_bounds__(512, 1)
                const __grid_constant__ CUtensorMap map_dq, const BwdArgs args) {
   using C = BwdCfg<D>;
   constexpr int NS = C::kNumSlots, KB = C::kKvBufs;
+  // ring position k = 2 t + v of the t-th Q tile processed (v = 0: its Q tile, v = 1: its dO tile)
+  auto pos_slot = [](int k) { return (k & 1) ? C::kQSlots + (k >> 1) % C::kDoSlots : (k >> 1) % C::kQSlots; };
+  auto pos_phase = [](int k) {
+    return (uint32_t)(((k & 1) ? (k >> 1) / C::kDoSlots : (k >> 1) / C::kQSlots) & 1);
+  };
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sKV = smem;                               // KB x (K tile, V tile)
   uint8_t* sDS = smem + KB * 2 * C::kTileBytes;
   uint8_t* sRing = sDS + C::kDsBytes;
   uint8_t* sStage = sRing + NS * C::kSlotBytes;  // 1024-aligned: slot bytes are multiples of 1024
+  uint8_t* sOnes = sStage + C::kStageBytes;
   auto sK = [&](int kb) { return sKV + kb * 2 * C::kTileBytes; };
   auto sV = [&](int kb) { return sKV + kb * 2 * C::kTileBytes + C::kTileBytes; };
 
@@ -316,6 +362,14 @@ __global__ void __launch_bounds__(512, 1)
   if (warp == kWarpMma) {
     ptx::tmem_alloc(ptx::smem_addr(&tmem_base_sh), C::kTmemCols);
     ptx::tmem_relinquish();
+  }
+  // The fold's A operand: kScale in columns 0-2 of the 8 rows of one core matrix (bytes [0,128)), zeros in its
+  // second K chunk (bytes [128,256)); every 8-row group of the 128 key rows reads that same pair (group stride 0).
+  if (threadIdx.x < C::kOnesBytes / 16) {
+    const uint32_t f2 = ptx::pack2<kBF16>(Fold<kBF16>::kScale, Fold<kBF16>::kScale);
+    const uint32_t f1 = ptx::pack2<kBF16>(Fold<kBF16>::kScale, 0.f);
+    *reinterpret_cast<uint4*>(sOnes + threadIdx.x * 16) = threadIdx.x < 8 ? make_uint4(f2, f1, 0u, 0u) : make_uint4(0u, 0u, 0u, 0u);
+    ptx::fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
   }
   ptx::tc_fence_before();
   __syncthreads();
@@ -367,21 +421,19 @@ __global__ void __launch_bounds__(512, 1)
         }
         int i;
         while (ok && it.next(i)) {
-          for (int v = 0; v < 2; ++v) {  // v = 0: Q_i (+ LSE2, D rows), v = 1: dO_i
-            const int s = n % NS;
-            const uint32_t ph = (n / NS) & 1;
+          for (int v = 0; v < 2; ++v) {  // v = 0: Q_i and its LSE fold rows, v = 1: dO_i and its D fold rows
+            const int s = pos_slot(n);
+            const uint32_t ph = pos_phase(n);
             if (!wait_or_abort(ptx::smem_addr(&bar_empty[s]), ph ^ 1, args.budget_ns, abortp)) { ok = false; break; }
             const uint32_t bf = ptx::smem_addr(&bar_full[s]);
             uint8_t* slot = sRing + s * C::kSlotBytes;
-            ptx::mbar_arrive_expect_tx(bf, C::kTileBytes + (v == 0 ? 1024 : 0));
+            ptx::mbar_arrive_expect_tx(bf, C::kTileBytes + C::kAugBytes);
             for (int c = 0; c < C::kSubTiles; ++c)
               tma_rows(ptx::smem_addr(slot + c * 16384), v == 0 ? &map_q : &map_do, c, i * kTile, u.g.q0, u.bh, u.h,
                        packed, bf);
-            if (v == 0) {
-              const size_t row0 = (size_t)u.bh * Npad + (size_t)i * kTile;
-              ptx::bulk_load(ptx::smem_addr(slot + C::kTileBytes), args.lse2 + row0, 512, bf);
-              ptx::bulk_load(ptx::smem_addr(slot + C::kTileBytes + 512), args.Dv + row0, 512, bf);
-            }
+            const size_t row0 = (size_t)u.bh * Npad + (size_t)i * kTile;
+            const uint8_t* side = reinterpret_cast<const uint8_t*>(v == 0 ? args.lse2 : args.Dv) + row0 * 16;
+            ptx::bulk_load(ptx::smem_addr(slot + C::kTileBytes), side, C::kAugBytes, bf);
             ++n;
           }
         }
@@ -390,8 +442,11 @@ __global__ void __launch_bounds__(512, 1)
       // Let every copy this thread issued land before the CTA can exit (immediate in the normal path).
       for (int k = (ku > KB ? ku - KB : 0); k < ku; ++k)
         ptx::mbar_wait(ptx::smem_addr(&bar_kv[k % KB]), (k / KB) & 1, args.budget_ns);
-      for (int k = (n > NS ? n - NS : 0); k < n; ++k)
-        ptx::mbar_wait(ptx::smem_addr(&bar_full[k % NS]), (k / NS) & 1, args.budget_ns);
+      // (the last positions that used each slot: kQSlots Q tiles, kDoSlots dO tiles)
+      for (int k = n - 2 * C::kQSlots; k < n; k += 2)
+        if (k >= 0) ptx::mbar_wait(ptx::smem_addr(&bar_full[pos_slot(k)]), pos_phase(k), args.budget_ns);
+      for (int k = n + 1 - 2 * C::kDoSlots; k < n; k += 2)
+        if (k >= 0) ptx::mbar_wait(ptx::smem_addr(&bar_full[pos_slot(k)]), pos_phase(k), args.budget_ns);
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------------------------------------ MMA issuer
@@ -408,11 +463,15 @@ __global__ void __launch_bounds__(512, 1)
       const uint64_t dds_mn = ptx::sw128_desc(ptx::smem_addr(sDS), 16384, 1024);  // dS, M-major (dQ)
       const uint64_t dring_k = ptx::sw128_desc(ptx::smem_addr(sRing), 16, 1024);
       const uint64_t dring_mn = ptx::sw128_desc(ptx::smem_addr(sRing), 16384, 1024);
-      auto slot_off = [&](int k) { return (uint32_t)((k % NS) * C::kSlotBytes); };
-      auto slot_full = [&](int k) { return ptx::smem_addr(&bar_full[k % NS]); };
-      auto slot_empty = [&](int k) { return ptx::smem_addr(&bar_empty[k % NS]); };
-      auto slot_phase = [&](int k) { return (uint32_t)((k / NS) & 1); };
+      auto slot_off = [&](int k) { return (uint32_t)(pos_slot(k) * C::kSlotBytes); };
+      auto slot_full = [&](int k) { return ptx::smem_addr(&bar_full[pos_slot(k)]); };
+      auto slot_empty = [&](int k) { return ptx::smem_addr(&bar_empty[pos_slot(k)]); };
+      auto slot_phase = [&](int k) { return pos_phase(k); };
       constexpr auto kstep = [](int kk) { return (uint32_t)((kk / 4) * 16384 + (kk % 4) * 32); };
+      // the fold step: A = the constant tile (K chunks 128 B apart, 8-row groups all alike), B = the slot's fold
+      // rows (16 bytes per query row, contiguous; the second K chunk repeats the first, where A holds zeros)
+      const uint64_t d_ones = ptx::plain_desc(ptx::smem_addr(sOnes), 128, 0);
+      const uint64_t d_fold = ptx::plain_desc(ptx::smem_addr(sRing + C::kTileBytes), 0, 128);
       uint64_t dk_k = 0, dk_mn = 0, dv_k = 0;  // K_j (K-major for S^T, M/N-major for dQ), V_j (K-major for dP^T)
       // S^T = K Q^T for the Q tile in ring position kq
       auto issue_s = [&](int kq) -> bool {
@@ -423,6 +482,7 @@ __global__ void __launch_bounds__(512, 1)
         for (int kk = 0; kk < D / 16; ++kk)
           ptx::mma_ss(tmem + C::kColS, ptx::desc_advance(dk_k, kstep(kk)), ptx::desc_advance(dq, kstep(kk)), id_sq,
                       kk > 0 ? 1u : 0u);
+        ptx::mma_ss(tmem + C::kColS, d_ones, ptx::desc_advance(d_fold, slot_off(kq)), id_sq, 1u);  // + (-LSE / scale)
         ptx::mma_commit(ptx::smem_addr(&bar_s));
         return true;
       };
@@ -435,6 +495,7 @@ __global__ void __launch_bounds__(512, 1)
         for (int kk = 0; kk < D / 16; ++kk)
           ptx::mma_ss(tmem + C::kColDP, ptx::desc_advance(dv_k, kstep(kk)), ptx::desc_advance(ddo, kstep(kk)), id_sq,
                       kk > 0 ? 1u : 0u);
+        ptx::mma_ss(tmem + C::kColDP, d_ones, ptx::desc_advance(d_fold, slot_off(ko)), id_sq, 1u);  // + (-D)
         ptx::mma_commit(ptx::smem_addr(&bar_dp));
         return true;
       };
@@ -454,7 +515,7 @@ __global__ void __launch_bounds__(512, 1)
         for (int kk = 0; kk < kTile / 16; ++kk)
           ptx::mma_ss(tmem + C::kColDK, ptx::desc_advance(dds_k, kstep(kk)), ptx::desc_advance(dq, kk * 2048), id_dv,
                       (!first || kk > 0) ? 1u : 0u);
-        ptx::mma_commit(slot_empty(kq));  // Q_i (and its LSE2/D rows) no longer needed
+        ptx::mma_commit(slot_empty(kq));  // Q_i (and its fold rows) no longer needed
       };
       // dQ_i = dS K_j  (dS read M-major from the dS^T tile)
       auto issue_dq = [&]() {
@@ -571,7 +632,7 @@ __global__ void __launch_bounds__(512, 1)
     const int c = quarter * 32 + lane;  // key row within the tile == TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const ptx::f32x2 sl2v{args.scale_log2, args.scale_log2}, sc2{args.scale, args.scale};
-    int n = 0, gi = 0;
+    int gi = 0;
     bool ok = true;
     while (ok && us.next(L)) {
       const BwdUnit u = bwd_unit(L, args);
@@ -582,17 +643,9 @@ __global__ void __launch_bounds__(512, 1)
       const int gc = j * kTile + c;  // key index in the sequence
       int i;
       while (it.next(i)) {
-        const int sq = n % NS;
-        const uint32_t phq = (n / NS) & 1;
-        n += 2;
-        // -LSE2 and -scale*D of this half's 64 queries (16-byte aligned: read four at a time, all lanes alike)
-        const float* nlse2 = reinterpret_cast<const float*>(sRing + sq * C::kSlotBytes + C::kTileBytes) + 64 * g;
-        const float* nDrow = nlse2 + 128;
         const uint32_t ph = gi & 1;
-        // the LSE2/D rows came in by bulk copy with Q_i: observe that copy's barrier before reading them (the slot
-        // cannot be refilled before this iteration's dS^T is published, so the phase is stable)
-        ok = __all_sync(0xffffffffu, wait_or_abort(ptx::smem_addr(&bar_full[sq]), phq, args.budget_ns, abortp));
-        if (ok) ok = __all_sync(0xffffffffu, wait_or_abort(ptx::smem_addr(&bar_s), ph, args.budget_ns, abortp));
+        // S^T arrives with -LSE / scale already added per query column (the fold), dP^T with -D
+        ok = __all_sync(0xffffffffu, wait_or_abort(ptx::smem_addr(&bar_s), ph, args.budget_ns, abortp));
         if (!ok) break;
         ptx::tc_fence_after();
         const bool masked = (causal && i == j) || (j + 1) * kTile > kv_lim;
@@ -608,11 +661,9 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
           for (int v = 0; v < 16; ++v) {
             const int r0 = 32 * h + 2 * v;
-            const float4 nl4 = *reinterpret_cast<const float4*>(nlse2 + (r0 & ~3));
-            const ptx::f32x2 nl = (v & 1) ? ptx::f32x2{nl4.z, nl4.w} : ptx::f32x2{nl4.x, nl4.y};
             const bool emu = kBwdExpFmaEvery > 0 && v % (kBwdExpFmaEvery > 0 ? kBwdExpFmaEvery : 1) == 0;
-            const ptx::f32x2 x =
-                ptx::fma2({__uint_as_float(sr[2 * v]), __uint_as_float(sr[2 * v + 1])}, sl2v, nl);  // S*scale - LSE
+            // (S - LSE / scale) * scale * log2(e) = log2 P
+            const ptx::f32x2 x = ptx::mul2({__uint_as_float(sr[2 * v]), __uint_as_float(sr[2 * v + 1])}, sl2v);
             float p0 = emu ? ptx::exp2_fma(x.x) : ptx::ex2(x.x);
             float p1 = emu ? ptx::exp2_fma(x.y) : ptx::ex2(x.y);
             if (masked) {
@@ -651,12 +702,8 @@ __global__ void __launch_bounds__(512, 1)
           uint32_t o[16];
 #pragma unroll
           for (int v = 0; v < 16; ++v) {
-            const int r0 = 32 * h + 2 * v;
-            const float4 nd4 = *reinterpret_cast<const float4*>(nDrow + (r0 & ~3));
-            const ptx::f32x2 nd = (v & 1) ? ptx::f32x2{nd4.z, nd4.w} : ptx::f32x2{nd4.x, nd4.y};
-            // dS = P * (dP - D) * scale = P * (dP * scale + (-scale * D)), P as the 16-bit values dV used
-            const ptx::f32x2 t =
-                ptx::fma2({__uint_as_float(dr[2 * v]), __uint_as_float(dr[2 * v + 1])}, sc2, nd);
+            // dS = P * (dP - D) * scale, P as the 16-bit values dV used (dP - D from the fold)
+            const ptx::f32x2 t = ptx::mul2({__uint_as_float(dr[2 * v]), __uint_as_float(dr[2 * v + 1])}, sc2);
             const ptx::f32x2 ds = ptx::mul2(ptx::unpack2<kBF16>(pk[16 * h + v]), t);
             o[v] = ptx::pack2<kBF16>(ds.x, ds.y);
           }

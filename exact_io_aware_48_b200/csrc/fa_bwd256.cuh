@@ -632,8 +632,9 @@ inline cudaError_t run_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const C
   a.dk = dk;
   a.dv = dv;
   a.dq_acc = reinterpret_cast<float*>(ws);
+  const size_t side = al((size_t)BH * npad * bwd_row_side_bytes(d));
   a.lse2 = reinterpret_cast<const float*>(ws + al((size_t)BH * npad * d * 4));
-  a.Dv = reinterpret_cast<const float*>(ws + al((size_t)BH * npad * d * 4) + al((size_t)BH * npad * 4));
+  a.Dv = reinterpret_cast<const float*>(ws + al((size_t)BH * npad * d * 4) + side);
   a.dl = d;
   a.key_lens = key_lens;
   a.col_ptr = col_ptr;

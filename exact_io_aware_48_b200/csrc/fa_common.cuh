@@ -20,6 +20,9 @@ __device__ int g_device_status = 0;
 
 __device__ __forceinline__ void record_error(int code) { atomicCAS(&g_device_status, 0, code); }
 
+#ifndef FA_WAIT_HINT_NS
+#define FA_WAIT_HINT_NS 0
+#endif
 // Bounded wait used by every pipeline role.  Gives up when the CTA's abort flag is raised by another role, or
 // after `budget_ns` (then it records FA_ERR_TIMEOUT in the status word and raises the abort flag itself).
 __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, uint64_t budget_ns,
@@ -27,9 +30,13 @@ __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, uin
   if (ptx::mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = ptx::globaltimer_ns();
   while (true) {
+#if FA_WAIT_HINT_NS
+    if (ptx::mbar_try_wait_sleep(bar, parity, FA_WAIT_HINT_NS)) return true;
+#else
 #pragma unroll 1
     for (int i = 0; i < 16; ++i)
       if (ptx::mbar_try_wait(bar, parity)) return true;
+#endif
     if (*abort_flag) return false;
     if (ptx::globaltimer_ns() - t0 > budget_ns) {
       record_error(kDevTimeout);
