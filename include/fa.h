@@ -87,7 +87,7 @@ int fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* o, flo
                        int d, float softmax_scale, int causal, const int32_t* key_lens, const uint8_t* block_mask,
                        void* workspace, size_t workspace_bytes, int dtype, void* stream);
 
-/* Bytes of workspace fa_bwd needs (fp32 dQ accumulator, per-row LSE/D in base 2, tile lists if masked). */
+/* Bytes of workspace fa_bwd needs (fp32 dQ accumulator, per-row LSE and D terms, tile lists if masked). */
 size_t fa_bwd_workspace_size(int B, int H, int N, int d, int has_block_mask);
 
 /*

@@ -10,7 +10,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def test_recorded_traffic_matches_the_current_sources():
-    # the committed record was taken on the kernel sources as they are now (any kernel edit must retake it)
+    # the committed record was taken on the recorded kernels' sources as they are now (editing them means retaking it)
     with open(os.path.join(ROOT, "profiles", "kernel_traffic.json")) as f:
         rec = json.load(f)
     assert rec["src_hash"] == bench.kernel_src_hash()
