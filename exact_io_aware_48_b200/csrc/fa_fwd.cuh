@@ -264,7 +264,10 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
       // Issue the pending P V of the previous visible tile for tile t (waits for its P).  The first P V of a unit
       // overwrites O_t, so it also waits until the epilogue has read the previous unit's O_t.
       bool v_ready = false;
-      auto flush_pv = [&](int t) -> bool {
+      // `k_wait` (a K slot's barrier and phase, bar 0 = none) is waited for together with this P V's own waits, so
+      // the MMA thread stops once rather than again before the next S: on sm_100a each wait of the issuing thread
+      // lets its queued MMAs drain first.
+      auto flush_pv = [&](int t, uint32_t k_bar = 0, uint32_t k_phase = 0) -> bool {
         if (!(pend_flags & (1 << t))) return true;
         if (!wait_or_abort(ptx::smem_addr(&bar_p[t]), p_phase[t], args.budget_ns, abortp)) return false;
         p_phase[t] ^= 1;
@@ -272,6 +275,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
           if (!wait_or_abort(ptx::smem_addr(&bar_full[pend_slot]), pend_phase, args.budget_ns, abortp)) return false;
           v_ready = true;
         }
+        if (k_bar != 0 && !wait_or_abort(k_bar, k_phase, args.budget_ns, abortp)) return false;
         if (pv_count[t] == 0 && ku > 0 &&
             !wait_or_abort(ptx::smem_addr(&bar_o_free[t]), (ku - 1) & 1, args.budget_ns, abortp))
           return false;
@@ -296,10 +300,19 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
           const int sV = n % NS;
           const uint32_t phV = (n / NS) & 1;
           ++n;
+          // K_j is waited for inside the first P V's waits when there is one before the first S
           bool k_ready = false;
+          const int t_first = (fl & 1) ? 0 : 1;  // the first tile that sees K_j
 #pragma unroll
           for (int t = 0; t < 2; ++t) {
-            if (ok) ok = flush_pv(t);
+            if (ok) {
+              if (t == t_first && !k_ready && (pend_flags & (1 << t))) {
+                ok = flush_pv(t, ptx::smem_addr(&bar_full[sK]), phK);
+                k_ready = ok;
+              } else {
+                ok = flush_pv(t);
+              }
+            }
             if (ok && (fl & (1 << t))) {
               if (!k_ready) {
                 ok = wait_or_abort(ptx::smem_addr(&bar_full[sK]), phK, args.budget_ns, abortp);
