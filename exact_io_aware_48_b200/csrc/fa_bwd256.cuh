@@ -238,12 +238,22 @@ __global__ void __launch_bounds__(512, 1)
         ptx::tc_fence_after();
         return true;
       };
+      // boxes k .. k+count-1, all waited for before any of their MMAs is issued: on sm_100a each wait of the
+      // issuing thread lets its queued MMAs drain first, so the waits of a group of MMAs are made back to back
+      auto take_n = [&](int k, int count) -> bool {
+        for (int i = 0; i < count; ++i)
+          if (!wait_or_abort(ptx::smem_addr(&bar_full[(k + i) % NS]), ((k + i) / NS) & 1, args.budget_ns, abortp))
+            return false;
+        ptx::tc_fence_after();
+        return true;
+      };
       auto release = [&](int k) { ptx::mma_commit(ptx::smem_addr(&bar_empty[k % NS])); };
       auto off = [&](int k) { return (uint32_t)((k % NS) * C::kBoxBytes); };
       // S^T = K Q^T or dP^T = V dO^T over d = 256: four (A box, B box) pairs, both K-major
+      // (two chunks, four boxes, per group: the ring holds six)
       auto scores = [&](uint32_t col, uint64_t& bar) -> bool {
         for (int c = 0; c < C::kBoxes; ++c) {
-          if (!take(nb) || !take(nb + 1)) return false;
+          if ((c & 1) == 0 && !take_n(nb, 4)) return false;
           const uint64_t da = ptx::desc_advance(ring_k, off(nb)), db = ptx::desc_advance(ring_k, off(nb + 1));
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
@@ -258,8 +268,8 @@ __global__ void __launch_bounds__(512, 1)
       };
       // S^T = K Q^T over d = 256: A = resident K box c, B = the next ring box (Q box c), both K-major
       auto scores_k = [&]() -> bool {
+        if (!take_n(nb, C::kBoxes)) return false;
         for (int c = 0; c < C::kBoxes; ++c) {
-          if (!take(nb)) return false;
           const uint64_t da = ptx::desc_advance(k_k, c * C::kBoxBytes), db = ptx::desc_advance(ring_k, off(nb));
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
@@ -295,8 +305,8 @@ __global__ void __launch_bounds__(512, 1)
         ptx::mma_commit(ptx::smem_addr(&bar_dq_full));
       };
       // dK_h += dS^T Q[:, h]  (dS^T K-major, the Q pair as one N = 128 operand)
-      auto issue_dk = [&](bool first) -> bool {
-        if (!take(nb) || !take(nb + 1)) return false;
+      // (the caller has taken the pair, together with the dS^T wait)
+      auto issue_dk = [&](bool first) {
         const uint64_t db = ptx::desc_advance(ring_mn, off(nb));
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)
@@ -305,7 +315,6 @@ __global__ void __launch_bounds__(512, 1)
         release(nb);
         release(nb + 1);
         nb += 2;
-        return true;
       };
       int gi = 0, ku = 0;  // Q tiles and non-empty units processed so far
       bool ok = true;
@@ -341,11 +350,13 @@ __global__ void __launch_bounds__(512, 1)
           if (!have_next) ptx::mma_commit(ptx::smem_addr(&bar_dv_done));  // this unit's dV_h is final
           // S^T_{i+1} overwrites P^T_i only after dV_i has read it (MMAs complete in issue order)
           if (have_next && !(ok = scores_k())) break;
+          // dS^T_i, dK_h's Q pair and (first tile) the dK accumulator: all waited for before dQ_i and dK_i
           if (!(ok = wait_or_abort(ptx::smem_addr(&bar_ds), ph, args.budget_ns, abortp))) break;
+          if (!(ok = take_n(nb, 2))) break;
+          if (li == 0 && !(ok = acc_ready(bar_dk_free))) break;
           ptx::tc_fence_after();
           issue_dq(half);
-          if (li == 0 && !(ok = acc_ready(bar_dk_free))) break;
-          if (!(ok = issue_dk(li == 0))) break;
+          issue_dk(li == 0);
           ptx::mma_commit(ptx::smem_addr(&bar_ds_free));
           ++gi;
           ++li;
