@@ -236,11 +236,15 @@ __global__ void __launch_bounds__(Fwd256Cfg::kThreads, 1)
       int n = 0;           // ring chunks consumed (same order as issued by the TMA warp)
       int gs = 0, nq = 0;  // S steps issued, Q tiles used
       bool ok = true;
-      auto chunk = [&](int& s) -> bool {
-        s = n % NS;
-        const uint32_t ph = (n / NS) & 1;
-        ++n;
-        if (!wait_or_abort(ptx::smem_addr(&bar_full[s]), ph, args.budget_ns, abortp)) return false;
+      // the next kChunks ring chunks (one K or V tile), all waited for before any of their MMAs is issued: on
+      // sm_100a each wait of the issuing thread lets its queued MMAs drain first
+      auto chunks = [&](int (&slots)[C::kChunks]) -> bool {
+        for (int c = 0; c < C::kChunks; ++c) {
+          slots[c] = n % NS;
+          const uint32_t ph = (n / NS) & 1;
+          ++n;
+          if (!wait_or_abort(ptx::smem_addr(&bar_full[slots[c]]), ph, args.budget_ns, abortp)) return false;
+        }
         ptx::tc_fence_after();
         return true;
       };
@@ -257,9 +261,10 @@ __global__ void __launch_bounds__(Fwd256Cfg::kThreads, 1)
           ++nq;
         }
         const uint32_t d_s = tmem + (gs & 1) * 128;
+        int slots[C::kChunks];
+        if (!chunks(slots)) return false;
         for (int c = 0; c < C::kChunks; ++c) {
-          int s;
-          if (!chunk(s)) return false;
+          const int s = slots[c];
           const uint64_t a = ptx::desc_advance(dq0, c * 16384);
           const uint64_t b = ptx::desc_advance(dk0, s * C::kChunkBytes);
 #pragma unroll
@@ -299,9 +304,10 @@ __global__ void __launch_bounds__(Fwd256Cfg::kThreads, 1)
             break;
           ptx::tc_fence_after();
           const uint32_t p_col = tmem + (gp & 1) * 128;
-          for (int kc = 0; kc < C::kChunks && ok; ++kc) {
-            int s;
-            if (!(ok = chunk(s))) break;
+          int slots[C::kChunks];
+          if (!(ok = chunks(slots))) break;
+          for (int kc = 0; kc < C::kChunks; ++kc) {
+            const int s = slots[kc];
             const uint64_t b = ptx::desc_advance(dv0, s * C::kChunkBytes);
 #pragma unroll
             for (int k2 = 0; k2 < 2; ++k2)  // 16 keys each; P packs two keys per column
