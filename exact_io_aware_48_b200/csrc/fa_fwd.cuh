@@ -300,13 +300,14 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
           const int sV = n % NS;
           const uint32_t phV = (n / NS) & 1;
           ++n;
-          // K_j is waited for inside the first P V's waits when there is one before the first S
+          // K_j is waited for inside the first P V's waits when there is one before the first S (two-tile kernel;
+          // measured slower in the one-tile kernel, whose K/V loads have less lead)
           bool k_ready = false;
           const int t_first = (fl & 1) ? 0 : 1;  // the first tile that sees K_j
 #pragma unroll
           for (int t = 0; t < 2; ++t) {
             if (ok) {
-              if (t == t_first && !k_ready && (pend_flags & (1 << t))) {
+              if (kTiles == 2 && t == t_first && !k_ready && (pend_flags & (1 << t))) {
                 ok = flush_pv(t, ptx::smem_addr(&bar_full[sK]), phK);
                 k_ready = ok;
               } else {
