@@ -726,7 +726,16 @@ def run_e2e(p, stream, args, world, chunks=4):
         with torch.cuda.stream(s_in):
             serial_step(s_in)
 
+    def copies():  # the step's PCIe traffic alone, both directions at once: the bound for the overlapped step
+        with torch.cuda.stream(s_in):
+            for dst, src in zip(dev_in, p.host):
+                dst.copy_(src, non_blocking=True)
+        with torch.cuda.stream(s_out):
+            for dst, src in zip(outs, dev_out):
+                dst.copy_(src, non_blocking=True)
+
     ms_serial = timed(serial)
+    ms_copies = timed(copies)
     ref = [t.clone() for t in outs]  # the unchunked step's results
     ms = timed(step)
     check_status(L, stream, "end-to-end steps")
@@ -739,15 +748,18 @@ def run_e2e(p, stream, args, world, chunks=4):
             raise RuntimeError(f"end-to-end: {name} of the overlapped steps differs from the unchunked step")
     if world > 1:
         import torch.distributed as dist
-        t = torch.tensor([ms, ms_serial], device="cuda", dtype=torch.float64)
+        t = torch.tensor([ms, ms_serial, ms_copies], device="cuda", dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, ms_serial = float(t[0].item()), float(t[1].item())
+        ms, ms_serial, ms_copies = float(t[0].item()), float(t[1].item()), float(t[2].item())
     val = world * 3.5 * p.fwd_flops / (ms / 1e3) / 1e12
     return {"value": round(val, 3), "unit": "TFLOP/s", "ms_per_step": round(ms, 4), "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "overlap": f"{chunks} groups of {'batch entries' if axis == 0 else 'heads'}, "
             "copies in, compute and copies out on three streams",
             "serial_ms_per_step": round(ms_serial, 4),
-            "serial_value": round(world * 3.5 * p.fwd_flops / (ms_serial / 1e3) / 1e12, 3)}
+            "serial_value": round(world * 3.5 * p.fwd_flops / (ms_serial / 1e3) / 1e12, 3),
+            "copies_only_ms_per_step": round(ms_copies, 4),
+            "copies_only_gbs": {"h2d": round(h2d / (ms_copies / 1e3) / 1e9, 1),
+                                "d2h": round(d2h / (ms_copies / 1e3) / 1e9, 1)}}
 
 
 # ---------------------------------------------------------------------------------------------- CPU oracle
