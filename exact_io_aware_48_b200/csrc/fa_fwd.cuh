@@ -140,7 +140,11 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
   uint8_t* sQ = smem;
   uint8_t* sKV = smem + C::kQBytes;
 
-  __shared__ __align__(8) uint64_t bar_q, bar_q_free, bar_full[NS], bar_empty[NS], bar_s[2], bar_p[2], bar_o[2],
+  // bar_sd[g % NSD]: every MMA of K/V step g (its S, and the previous step's P V) has completed.  K_g's slot was
+  // last read in step g - NSD and V_g's slot in step g - NSD + 1 (V is read by the next step's P V), so the producer
+  // waits for those; one commit per step releases both of a step's slots.
+  constexpr int NSD = NS / 2;
+  __shared__ __align__(8) uint64_t bar_q, bar_q_free, bar_full[NS], bar_sd[NSD], bar_s[2], bar_p[2], bar_o[2],
       bar_o_free[2], bar_drain;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
@@ -155,10 +159,8 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
   if (threadIdx.x == 0) {
     ptx::mbar_init(ptx::smem_addr(&bar_q), 1);
     ptx::mbar_init(ptx::smem_addr(&bar_q_free), 1);
-    for (int s = 0; s < NS; ++s) {
-      ptx::mbar_init(ptx::smem_addr(&bar_full[s]), 1);
-      ptx::mbar_init(ptx::smem_addr(&bar_empty[s]), 1);
-    }
+    for (int s = 0; s < NS; ++s) ptx::mbar_init(ptx::smem_addr(&bar_full[s]), 1);
+    for (int s = 0; s < NSD; ++s) ptx::mbar_init(ptx::smem_addr(&bar_sd[s]), 1);
     for (int t = 0; t < 2; ++t) {
       ptx::mbar_init(ptx::smem_addr(&bar_s[t]), 1);
       ptx::mbar_init(ptx::smem_addr(&bar_p[t]), 128);
@@ -191,7 +193,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
       ptx::prefetch_tensormap(&map_k);
       ptx::prefetch_tensormap(&map_v);
       const uint32_t bq = ptx::smem_addr(&bar_q);
-      int n = 0, ku = 0, j, fl;
+      int n = 0, g = 0, ku = 0, j, fl;  // g: K/V steps loaded
       bool ok = true;
       while (ok && us.next(L)) {
         const FwdUnit u = fwd_unit<kMode>(L, args, kTiles);
@@ -207,8 +209,11 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
         while (ok && it.next(j, fl)) {
           for (int kv = 0; kv < 2; ++kv) {
             const int s = n % NS;
-            const uint32_t ph = (n / NS) & 1;
-            if (!wait_or_abort(ptx::smem_addr(&bar_empty[s]), ph ^ 1, args.budget_ns, abortp)) { ok = false; break; }
+            const int x = g - NSD + kv;  // the step that last read this slot
+            if (x >= 0 && !wait_or_abort(ptx::smem_addr(&bar_sd[x % NSD]), (x / NSD) & 1, args.budget_ns, abortp)) {
+              ok = false;
+              break;
+            }
             const uint32_t bf = ptx::smem_addr(&bar_full[s]);
             ptx::mbar_arrive_expect_tx(bf, C::kSlotBytes);
             const CUtensorMap* map = kv == 0 ? &map_k : &map_v;
@@ -217,6 +222,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
                        packed, bf);
             ++n;
           }
+          ++g;
         }
         ++ku;
       }
@@ -235,7 +241,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
       const uint64_t dkv_k = ptx::sw128_desc(ptx::smem_addr(sKV), 16, 1024);     // K tiles, K-major
       const uint64_t dkv_mn = ptx::sw128_desc(ptx::smem_addr(sKV), 16384, 1024); // V tiles, M/N-major
       bool ok = true;
-      int n = 0, ku = 0, j, fl;
+      int n = 0, g = 0, ku = 0, j, fl;  // g: K/V steps issued
       int pend_slot = 0, pend_flags = 0;
       uint32_t pend_phase = 0;
       uint32_t p_phase[2] = {0, 0};
@@ -327,8 +333,8 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
             }
           }
           if (!ok) break;
-          if (pend_flags) ptx::mma_commit(ptx::smem_addr(&bar_empty[pend_slot]));  // previous V consumed
-          ptx::mma_commit(ptx::smem_addr(&bar_empty[sK]));                          // this K consumed
+          ptx::mma_commit(ptx::smem_addr(&bar_sd[g % NSD]));  // this K and the previous V consumed
+          ++g;
           pend_slot = sV;
           pend_phase = phV;
           pend_flags = fl;
@@ -340,7 +346,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
         for (int t = 0; t < 2; ++t)
           if (ok) ok = flush_pv(t);
         if (!ok) break;
-        if (pend_flags) ptx::mma_commit(ptx::smem_addr(&bar_empty[pend_slot]));
+        // (this unit's last V is released by the next step's commit)
         // A tile that had no P V in this unit did not wait for the previous unit's epilogue; wait now, or two
         // back-to-back empty units would complete two phases of bar_o before its softmax warps look (ABA).
         for (int t = 0; t < kTiles && ok; ++t)
