@@ -11,9 +11,12 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libfa.so")
+RELEASE_LIB_PATH = os.path.join(_HERE, "libfa.so")
+DEBUG_LIB_PATH = os.path.join(_HERE, "libfa_debug.so")  # FA_DEBUG=1 build: device-side index checks
+# FA_LIB_PATH (a debug knob) selects another build of the same library, e.g. DEBUG_LIB_PATH
+LIB_PATH = os.environ.get("FA_LIB_PATH") or RELEASE_LIB_PATH
 
-FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT, FA_ERR_WORKSPACE = range(6)
+FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT, FA_ERR_WORKSPACE, FA_ERR_BOUNDS = range(7)
 FA_BF16, FA_FP16 = 0, 1
 
 # C signatures, exactly as declared in include/fa.h
@@ -33,6 +36,9 @@ SIGNATURES = {
     "fa_selftest_wait_timeout": ([_U64, _P], _I),
     "fa_set_kernel_events": ([_I, _P, _P], _I),
     "fa_selftest_exp2": ([_P, _P, _P, _I, _P], _I),
+    "fa_debug_build": ([], _I),
+    "fa_last_bounds_site": ([_P], _I),
+    "fa_selftest_bounds": ([_P], _I),
     "fa_set_fwd_tiles_per_cta": ([_I], _I),
     "fa_bwd_noalloc": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P, _P, _I, _P], _I),
     "fa_fwd_varlen": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P], _I),
@@ -166,6 +172,18 @@ def fa_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, softmax_scale,
 
 def fa_selftest_exp2(x, out_fma, out_mufu, n, stream=None) -> int:
     return load().fa_selftest_exp2(_ptr(x), _ptr(out_fma), _ptr(out_mufu), n, _stream(stream))
+
+
+def fa_debug_build() -> int:
+    return load().fa_debug_build()
+
+
+def fa_last_bounds_site(stream=None) -> int:
+    return load().fa_last_bounds_site(_stream(stream))
+
+
+def fa_selftest_bounds(stream=None) -> int:
+    return load().fa_selftest_bounds(_stream(stream))
 
 
 def fa_set_fwd_tiles_per_cta(tiles) -> int:

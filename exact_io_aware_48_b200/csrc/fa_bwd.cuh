@@ -208,7 +208,9 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const void* __restrict__ o
     const size_t prow = cu_q ? (size_t)(g.q0 + r) * H + (size_t)(bh % H) : (size_t)bh * N + r;  // row of O, dO
     float dsum = 0.f;
     const bool col_ok = l * 8 < dl;  // lanes past the head dim (32 / 96 on the 64 / 128 kernels) hold nothing
-    if (in && valid && col_ok) {
+    const size_t o_rows = cu_q ? (size_t)total_q * H : (size_t)(rows / Npad) * N;  // rows of O, dO (entries of LSE)
+    (void)o_rows;
+    if (in && valid && col_ok && in_bounds(prow < o_rows, kSiteBwdPre)) {
       const size_t off = prow * dl + (size_t)l * 8;
       const uint4 a = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(o) + off);
       const uint4 c = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(dout) + off);
@@ -229,7 +231,8 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const void* __restrict__ o
         acc[2 * l + 1] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
       if (l == 0) {
-        const float lv = valid ? lse[cu_q ? (size_t)(bh % H) * total_q + g.q0 + r : (size_t)bh * N + r] : -INFINITY;
+        const size_t li = cu_q ? (size_t)(bh % H) * total_q + g.q0 + r : (size_t)bh * N + r;
+        const float lv = valid && in_bounds(li < o_rows, kSiteBwdPre) ? lse[li] : -INFINITY;
         if constexpr (D <= 128) {
           // the fold rows: -LSE / scale and -D (padded row or no visible key: the masked row, P = 0)
           reinterpret_cast<uint4*>(lse2)[row] = lv != -INFINITY ? Fold<kBF16>::row(-lv / scale) : Fold<kBF16>::masked_row();
@@ -264,6 +267,13 @@ __global__ void __launch_bounds__(256) bwd_dq_kernel(const float* __restrict__ d
       if (r >= g.lq) continue;
       out_e = ((size_t)(g.q0 + r) * H + (size_t)(bh % H)) * dl + c;
     }
+    // extents checked in FA_DEBUG builds: rows of the fp32 accumulator ([BH][Npad]) and elements of dQ
+    const long long rows_v = total_vec8 * 8 / dl;  // dense: BH * N; packed: BH * Npad
+    const size_t acc_rows = cu_q ? (size_t)rows_v : (size_t)(rows_v / N) * Npad;
+    const size_t out_elems = cu_q ? (size_t)total_q * H * dl : (size_t)total_vec8 * 8;
+    if (!in_bounds((size_t)bh * Npad + r < acc_rows && out_e + 8 <= out_elems, kSiteBwdDqConv)) continue;
+    (void)acc_rows;
+    (void)out_elems;
     const float4* src = reinterpret_cast<const float4*>(dq_acc + ((size_t)bh * Npad + r) * dl + c);
     const float4 a = src[0], b = src[1];
     uint4 out;
@@ -427,13 +437,15 @@ __global__ void __launch_bounds__(512, 1)
             if (!wait_or_abort(ptx::smem_addr(&bar_empty[s]), ph ^ 1, args.budget_ns, abortp)) { ok = false; break; }
             const uint32_t bf = ptx::smem_addr(&bar_full[s]);
             uint8_t* slot = sRing + s * C::kSlotBytes;
-            ptx::mbar_arrive_expect_tx(bf, C::kTileBytes + C::kAugBytes);
+            const size_t row0 = (size_t)u.bh * Npad + (size_t)i * kTile;
+            // the 128 fold rows lie inside the [BH][Npad] side arrays (a skipped load is left out of the byte count)
+            const bool side_ok = in_bounds(row0 + kTile <= (size_t)args.BH * Npad, kSiteBwdSide);
+            ptx::mbar_arrive_expect_tx(bf, C::kTileBytes + (side_ok ? C::kAugBytes : 0));
             for (int c = 0; c < C::kSubTiles; ++c)
               tma_rows(ptx::smem_addr(slot + c * 16384), v == 0 ? &map_q : &map_do, c, i * kTile, u.g.q0, u.bh, u.h,
                        packed, bf);
-            const size_t row0 = (size_t)u.bh * Npad + (size_t)i * kTile;
             const uint8_t* side = reinterpret_cast<const uint8_t*>(v == 0 ? args.lse2 : args.Dv) + row0 * 16;
-            ptx::bulk_load(ptx::smem_addr(slot + C::kTileBytes), side, C::kAugBytes, bf);
+            if (side_ok) ptx::bulk_load(ptx::smem_addr(slot + C::kTileBytes), side, C::kAugBytes, bf);
             ++n;
           }
         }
@@ -746,6 +758,8 @@ __global__ void __launch_bounds__(512, 1)
       // dense: every row of the head (keys past a key length get zero); packed: the sequence's own keys only
       const bool row_ok = packed ? gc < u.g.lk : gc < args.N;
       const size_t krow = packed ? (size_t)(u.g.k0 + gc) * args.H + u.h : (size_t)u.bh * args.N + gc;
+      const size_t kv_rows = packed ? (size_t)args.total_k * args.H : (size_t)args.BH * args.N;  // rows of dK, dV
+      (void)kv_rows;
       // dV (is_dk false) or dK of this unit: read out of TMEM chunk by chunk, release the columns to the next unit
       // after the last read, store 16-bit; a unit with no visible query writes zeros
       auto epilogue = [&](bool is_dk) {
@@ -768,7 +782,7 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
           for (int v = 0; v < 16; ++v)
             pkd[v] = ptx::pack2<kBF16>(__uint_as_float(r[2 * v]), __uint_as_float(r[2 * v + 1]));
-          if (row_ok && cc * 32 < args.dl) {
+          if (row_ok && cc * 32 < args.dl && in_bounds(krow < kv_rows, kSiteBwdKV)) {
             uint4* dst = reinterpret_cast<uint4*>(row + cc * 64);
 #pragma unroll
             for (int v = 0; v < 4; ++v)
@@ -800,7 +814,9 @@ __global__ void __launch_bounds__(512, 1)
           ptx::fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            ptx::tma_reduce_add_2d(&map_dq, col, row0, stage_addr);
+            // the 32 x 32 box lies inside the [BH * Npad][dl] accumulator
+            if (in_bounds(row0 >= 0 && (size_t)row0 + 32 <= (size_t)args.BH * Npad && col + 32 <= args.dl, kSiteBwdDq))
+              ptx::tma_reduce_add_2d(&map_dq, col, row0, stage_addr);
             ptx::bulk_commit_group();
           }
         };

@@ -166,10 +166,14 @@ __global__ void __launch_bounds__(512, 1)
           if (!wait_or_abort(ptx::smem_addr(&bar_ld_empty[s]), ((gl / C::kLdSlots) & 1) ^ 1, args.budget_ns, abortp))
             return false;
           const uint32_t bf = ptx::smem_addr(&bar_ld_full[s]);
-          ptx::mbar_arrive_expect_tx(bf, 1024);
           const size_t row0 = (size_t)u.bh * Npad + (size_t)i * kTile;
-          ptx::bulk_load(ptx::smem_addr(sLd + s * 1024), args.lse2 + row0, 512, bf);
-          ptx::bulk_load(ptx::smem_addr(sLd + s * 1024 + 512), args.Dv + row0, 512, bf);
+          // the 128 rows lie inside the [BH][Npad] arrays (a skipped load is left out of the byte count)
+          const bool side_ok = in_bounds(row0 + kTile <= (size_t)args.BH * Npad, kSiteBwdSide);
+          ptx::mbar_arrive_expect_tx(bf, side_ok ? 1024 : 0);
+          if (side_ok) {
+            ptx::bulk_load(ptx::smem_addr(sLd + s * 1024), args.lse2 + row0, 512, bf);
+            ptx::bulk_load(ptx::smem_addr(sLd + s * 1024 + 512), args.Dv + row0, 512, bf);
+          }
           ++gl;
           return true;
         };
@@ -487,6 +491,8 @@ __global__ void __launch_bounds__(512, 1)
       const int gc = u.j * kTile + wq * 32 + lane;
       const bool row_ok = packed ? gc < u.g.lk : gc < args.N;
       const size_t krow = packed ? (size_t)(u.g.k0 + gc) * args.H + u.h : (size_t)u.bh * args.N + gc;
+      const size_t kv_rows = packed ? (size_t)args.total_k * args.H : (size_t)args.BH * args.N;  // rows of dK, dV
+      (void)kv_rows;
       auto epilogue = [&](bool is_dk) {
         uint8_t* row = reinterpret_cast<uint8_t*>(is_dk ? args.dk : args.dv) + krow * args.dl * 2 + half * C::kHalf * 2;
 #pragma unroll 1
@@ -507,7 +513,7 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
           for (int v = 0; v < 16; ++v)
             pkd[v] = ptx::pack2<kBF16>(__uint_as_float(r[2 * v]), __uint_as_float(r[2 * v + 1]));
-          if (row_ok) {
+          if (row_ok && in_bounds(krow < kv_rows, kSiteBwdKV)) {
             uint4* dst = reinterpret_cast<uint4*>(row + cc * 64);
 #pragma unroll
             for (int v = 0; v < 4; ++v)
@@ -538,7 +544,10 @@ __global__ void __launch_bounds__(512, 1)
           ptx::fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            ptx::tma_reduce_add_2d(&map_dq, col0 + col, row0, stage_addr);
+            // the 32 x 32 box lies inside the [BH * Npad][dl] accumulator
+            if (in_bounds(row0 >= 0 && (size_t)row0 + 32 <= (size_t)args.BH * Npad && col0 + col + 32 <= args.dl,
+                          kSiteBwdDq))
+              ptx::tma_reduce_add_2d(&map_dq, col0 + col, row0, stage_addr);
             ptx::bulk_commit_group();
           }
         };

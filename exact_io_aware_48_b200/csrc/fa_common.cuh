@@ -13,12 +13,50 @@ namespace fa {
 
 constexpr int kTile = 128;  // rows of a Q tile and keys of a K/V tile
 
-enum DeviceError : int { kDevOk = 0, kDevTimeout = 4 };
+enum DeviceError : int { kDevOk = 0, kDevTimeout = 4, kDevBounds = 6 };
 
 // One status word per device; the first error wins.  Read and cleared by fa_last_device_status().
 __device__ int g_device_status = 0;
 
 __device__ __forceinline__ void record_error(int code) { atomicCAS(&g_device_status, 0, code); }
+
+// ------------------------------------------------------------------------------------------------ debug checks
+// FA_DEBUG builds (libfa_debug.so) check every index the kernels compute for a global-memory access against the
+// extent of the buffer it addresses.  A failed check records kDevBounds in the status word and the site code
+// below in g_bounds_site (first failure wins), and the caller skips the access, so the kernel neither faults nor
+// traps.  Release builds compile the checks away (in_bounds is constant true).
+#ifndef FA_DEBUG
+#define FA_DEBUG 0
+#endif
+enum BoundsSite : int {
+  kSiteFwdO = 1,         // forward O row store
+  kSiteFwdLse = 2,       // forward LSE store
+  kSiteSplitPart = 3,    // split-K/V partial O / LSE store
+  kSiteCombine = 4,      // split-K/V combine O / LSE store
+  kSiteFwd256 = 5,       // d = 256 forward O / LSE store
+  kSiteBwdSide = 11,     // backward per-row fold / side data load
+  kSiteBwdDq = 12,       // backward dQ partial-sum reduce box
+  kSiteBwdKV = 13,       // backward dK / dV row store
+  kSiteBwdPre = 14,      // backward preprocess row
+  kSiteBwdDqConv = 15,   // dQ conversion row
+  kSiteMaskList = 21,    // block-mask list entry
+  kSiteSelftest = 99,    // fa_selftest_bounds
+};
+__device__ int g_bounds_site = 0;
+
+__device__ __forceinline__ bool in_bounds(bool ok, int site) {
+#if FA_DEBUG
+  if (!ok) {
+    record_error(kDevBounds);
+    atomicCAS(&g_bounds_site, 0, site);
+  }
+  return ok;
+#else
+  (void)ok;
+  (void)site;
+  return true;
+#endif
+}
 
 #ifndef FA_WAIT_HINT_NS
 #define FA_WAIT_HINT_NS 0

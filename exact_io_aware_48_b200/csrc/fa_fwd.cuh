@@ -499,6 +499,11 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
       if constexpr (split) prow = ((size_t)u.split * args.BH + u.bh) * (size_t)(args.nT * kTile) + grow;
       const size_t orow_idx = packed ? (size_t)(u.g.q0 + grow) * args.H + u.h : (size_t)u.bh * args.N + grow;
       uint8_t* orow = reinterpret_cast<uint8_t*>(args.o) + orow_idx * args.dl * 2;
+      // extents checked in FA_DEBUG builds: rows of O (and entries of LSE), rows of the split partials
+      const size_t o_rows = packed ? (size_t)args.total_q * args.H : (size_t)args.BH * args.N;
+      const size_t part_rows = (size_t)args.nsplit * args.BH * args.nT * kTile;
+      (void)o_rows;
+      (void)part_rows;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t orr[32];
@@ -509,7 +514,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
           ptx::mbar_arrive(ptx::smem_addr(&bar_o_free[t]));
         }
         if constexpr (split) {
-          if (row_ok) {
+          if (row_ok && in_bounds(prow < part_rows, kSiteSplitPart)) {
             float4* dst = reinterpret_cast<float4*>(args.o_part + prow * D + c * 32);
 #pragma unroll
             for (int v = 0; v < 8; ++v) {
@@ -527,7 +532,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
             const float bb = nonempty ? __uint_as_float(orr[2 * i + 1]) * inv : 0.0f;
             pk[i] = ptx::pack2<kBF16>(a, bb);
           }
-          if (row_ok && c * 32 < args.dl) {
+          if (row_ok && c * 32 < args.dl && in_bounds(orow_idx < o_rows, kSiteFwdO)) {
             uint4* dst = reinterpret_cast<uint4*>(orow + c * 64);
 #pragma unroll
             for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
@@ -537,10 +542,10 @@ __global__ void __launch_bounds__(FwdCfg<D, kTiles>::kThreads, 3 - kTiles)
       if (row_ok) {
         const float lse_v = nonempty ? (m_ref + __log2f(l_sum)) * 0.69314718055994530942f : -INFINITY;
         if constexpr (split) {
-          args.lse_part[prow] = lse_v;
+          if (in_bounds(prow < part_rows, kSiteSplitPart)) args.lse_part[prow] = lse_v;
         } else {
           const size_t li = packed ? (size_t)u.h * args.total_q + u.g.q0 + grow : (size_t)u.bh * args.N + grow;
-          args.lse[li] = lse_v;
+          if (in_bounds(li < o_rows, kSiteFwdLse)) args.lse[li] = lse_v;
         }
       }
       ++ku;

@@ -16,6 +16,9 @@
 #include "fa_bwd256.cuh"
 #include "fa_mask.cuh"
 
+// The device error codes are the fa_status values the host returns for them.
+static_assert(fa::kDevTimeout == FA_ERR_TIMEOUT && fa::kDevBounds == FA_ERR_BOUNDS, "device error codes");
+
 namespace {
 
 constexpr int kVersion = 10300;  // 1.3.0: head dims 32 and 96, per-head block masks
@@ -421,6 +424,7 @@ const char* fa_status_string(int s) {
     case FA_ERR_CUDA: return "FA_ERR_CUDA";
     case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
     case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE";
+    case FA_ERR_BOUNDS: return "FA_ERR_BOUNDS";
     default: return "FA_UNKNOWN_STATUS";
   }
 }
@@ -708,6 +712,28 @@ int fa_set_fwd_tiles_per_cta(int tiles) {
   if (tiles < 0 || tiles > 2) return FA_ERR_INVALID_ARG;
   g_fwd_tiles.store(tiles);
   return FA_OK;
+}
+
+int fa_debug_build(void) { return FA_DEBUG ? 1 : 0; }
+
+int fa_last_bounds_site(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return -cuda_fail(e);
+  int v = 0;
+  e = cudaMemcpyFromSymbol(&v, fa::g_bounds_site, sizeof(int));
+  if (e != cudaSuccess) return -cuda_fail(e);
+  if (v != 0) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(fa::g_bounds_site, &zero, sizeof(int));
+    if (e != cudaSuccess) return -cuda_fail(e);
+  }
+  return v;
+}
+
+int fa_selftest_bounds(void* stream) {
+  fa::selftest_bounds_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>();
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? FA_OK : cuda_fail(e);
 }
 
 int fa_selftest_exp2(const float* x, float* out_fma, float* out_mufu, int n, void* stream) {

@@ -103,7 +103,8 @@ __global__ void __launch_bounds__(kMaskWarps * 32)
     for (int x0 = 0; x0 < nT; x0 += 32) {
       const bool kept = x0 + lane < nT && r[x0 + lane] != 0;
       const unsigned bal = __ballot_sync(0xffffffffu, kept);
-      if (kept) col_idx[pos + __popc(bal & ((1u << lane) - 1u))] = x0 + lane;
+      const long long e = pos + __popc(bal & ((1u << lane) - 1u));  // a list holds at most nT * nT entries
+      if (kept && in_bounds(e < (long long)nT * nT, kSiteMaskList)) col_idx[e] = x0 + lane;
       pos += __popc(bal);
     }
   } else {
@@ -112,8 +113,20 @@ __global__ void __launch_bounds__(kMaskWarps * 32)
     int pos = col_ptr[j];
 #pragma unroll 8
     for (int x = 0; x < nT; ++x)
-      if (mask[(size_t)x * nT + j]) row_idx[pos++] = x;
+      if (mask[(size_t)x * nT + j]) {
+        if (in_bounds(pos < (long long)nT * nT, kSiteMaskList)) row_idx[pos] = x;
+        ++pos;
+      }
   }
+}
+
+// Debug-check self-test: one thread stores to indices 0..4 of a 4-entry array through in_bounds.  In an FA_DEBUG
+// build the last index fails its check, which records kDevBounds and kSiteSelftest and skips that store; no access
+// outside the array is made in either build.
+__device__ int g_selftest_bounds_buf[4];
+__global__ void selftest_bounds_kernel() {
+  for (int i = 0; i <= 4; ++i)
+    if (in_bounds(i < 4, kSiteSelftest)) g_selftest_bounds_buf[i & 3] = i;
 }
 
 // Waits on an mbarrier that nothing arrives on; the bounded wait must give up, record FA_ERR_TIMEOUT and return.

@@ -26,8 +26,12 @@
  *               until the stream reaches the work.
  *   Errors      Argument errors are detected on the host before anything is launched and returned as an
  *               fa_status; launch failures return FA_ERR_CUDA.  Errors found by the kernels while running (a
- *               pipeline wait that exceeded its time budget) are recorded in a per-device status word and
- *               returned by fa_last_device_status().  Non-finite inputs are not checked; they propagate.
+ *               pipeline wait that exceeded its time budget; in the debug build also a failed index check) are
+ *               recorded in a per-device status word and returned by fa_last_device_status().  Non-finite inputs
+ *               are not checked; they propagate.
+ *   Debug build libfa_debug.so (same entry points, compiled with FA_DEBUG=1) checks every index its kernels
+ *               compute for a global-memory access against the extent of the buffer it addresses; a failed check
+ *               skips that access and records FA_ERR_BOUNDS plus a site code (fa_last_bounds_site).
  *   Threads     Calls may come from several host threads; each call only reads library state that is set once.
  */
 #ifndef FA_H_
@@ -46,7 +50,8 @@ typedef enum {
   FA_ERR_UNSUPPORTED = 2, /* head dimension other than 32, 64, 96, 128, 256 */
   FA_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed (message: fa_last_error_string) */
   FA_ERR_TIMEOUT = 4,     /* a kernel wait ran out of its time budget (device-detected) */
-  FA_ERR_WORKSPACE = 5    /* workspace missing, misaligned or smaller than the query says */
+  FA_ERR_WORKSPACE = 5,   /* workspace missing, misaligned or smaller than the query says */
+  FA_ERR_BOUNDS = 6       /* debug build only: a kernel's index check failed and the access was skipped */
 } fa_status;
 
 typedef enum { FA_BF16 = 0, FA_FP16 = 1 } fa_dtype;
@@ -219,6 +224,26 @@ int fa_set_fwd_tiles_per_cta(int tiles);
  * pointers, caller-owned).  Used by the tests to bound the polynomial's relative error.
  */
 int fa_selftest_exp2(const float* x, float* out_fma, float* out_mufu, int n, void* stream);
+
+/* 1 if this library is the debug build (index checks compiled in), else 0. */
+int fa_debug_build(void);
+
+/*
+ * Synchronises `stream`, then returns and clears the site code of the first failed index check since the last
+ * query (0 if none; always 0 in the release build).  Sites: 1 forward O row, 2 forward LSE, 3 split-K/V partials,
+ * 4 split-K/V combine, 5 d = 256 forward O / LSE, 11 backward per-row side data, 12 backward dQ reduce box,
+ * 13 backward dK / dV row, 14 backward preprocess row, 15 dQ conversion, 21 block-mask list entry, 99 self-test.
+ * A negative value is an FA_ERR_CUDA from the synchronisation or the read.
+ */
+int fa_last_bounds_site(void* stream);
+
+/*
+ * Self-test of the index checks: one thread stores to a 4-entry device array through the check, at indices 0..4.
+ * In the debug build the last one fails its check: FA_ERR_BOUNDS is recorded (fa_last_device_status) with site 99
+ * (fa_last_bounds_site) and that store is skipped.  In the release build the checks are compiled out and nothing
+ * is recorded.  No access outside the array is made in either build.
+ */
+int fa_selftest_bounds(void* stream);
 
 /* Size of the fixed device scratch array behind fa_bwd_noalloc: 32 MiB of device memory on every GPU whose context
  * loads the array's module, held until that context is destroyed (normally process exit).  With lazy module loading
