@@ -4,7 +4,10 @@ oracle at the tolerances of the main parity tests; after each case the device st
 must be clear (no index check failed on valid inputs).  Finally the bounds self-test must be caught: status
 FA_ERR_BOUNDS, site 99.  Prints one JSON object on the last line of stdout.
 
-    FA_LIB_PATH=.../libfa_debug.so python tests/debug_cases.py
+    FA_LIB_PATH=.../libfa_debug.so python tests/debug_cases.py [--full]
+
+With --full it instead runs one forward + backward of every benchmark workload at full size through the debug
+library and checks only that no index check failed.
 """
 import json
 import os
@@ -81,8 +84,29 @@ def decode(out):
     out["decode"]["err"] = [assert_o_close(o.cpu().double().numpy(), ro), assert_lse_close(lse.cpu().numpy(), rl)]
 
 
+def full_size(out):
+    """One forward + backward of every benchmark workload (full size): only the status words are checked here;
+    the values at these sizes are compared with the oracle by the sampled parity tests."""
+    import bench
+    st = torch.cuda.Stream()
+    for name, w in inputs.workloads().items():
+        p = bench.Problem(w)
+        p.step(st)
+        st.synchronize()
+        clear("full_" + name, out)
+        del p
+        torch.cuda.empty_cache()
+
+
 def main():
     torch.cuda.set_device(0)
+    if "--full" in sys.argv:
+        out = {"debug_build": _lib.fa_debug_build()}
+        assert out["debug_build"] == 1, "FA_LIB_PATH must select libfa_debug.so"
+        clear("start", out)
+        full_size(out)
+        print(json.dumps(out))
+        return
     out = {"debug_build": _lib.fa_debug_build(), "lib": os.path.basename(_lib.LIB_PATH)}
     assert out["debug_build"] == 1, "FA_LIB_PATH must select libfa_debug.so"
     clear("start", out)

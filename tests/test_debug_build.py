@@ -62,3 +62,17 @@ def test_debug_build_parity_and_bounds_selftest():
     assert len(cases) == 7
     for k in cases:
         assert res[k]["status"] == 0 and res[k]["site"] == 0, k
+
+
+@pytest.mark.gpu
+def test_debug_build_full_size_workloads_pass_every_index_check():
+    env = dict(os.environ, FA_LIB_PATH=_lib.DEBUG_LIB_PATH)
+    r = subprocess.run([sys.executable, os.path.join(HERE, "debug_cases.py"), "--full"], env=env,
+                       capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
+    res = json.loads(r.stdout.strip().splitlines()[-1])
+    full = [k for k in res if k.startswith("full_")]
+    assert len(full) >= 8
+    for k in full:
+        assert res[k] == {"status": 0, "site": 0}, k
+
