@@ -551,20 +551,21 @@ __global__ void __launch_bounds__(512, 1)
             ptx::bulk_commit_group();
           }
         };
+        // at most two 32-column chunks in registers at a time (three spilled at this kernel's register budget)
         uint32_t ra[32], rb[32];
         ptx::tmem_ld32(tmem + lane_base + C::kColDQ, ra);
         ptx::tmem_ld32(tmem + lane_base + C::kColDQ + 32, rb);
         ptx::tmem_ld_wait();
         reduce_box(ra, 0);
-        uint32_t rc[32], rd[32];
-        ptx::tmem_ld32(tmem + lane_base + C::kColDQ + 64, rc);
-        ptx::tmem_ld32(tmem + lane_base + C::kColDQ + 96, rd);
+        ptx::tmem_ld32(tmem + lane_base + C::kColDQ + 64, ra);
+        ptx::tmem_ld_wait();
+        reduce_box(rb, 32);
+        ptx::tmem_ld32(tmem + lane_base + C::kColDQ + 96, rb);
         ptx::tmem_ld_wait();
         ptx::tc_fence_before();
         ptx::mbar_arrive(ptx::smem_addr(&bar_dq_free));  // the next dP^T may overwrite these columns
-        reduce_box(rb, 32);
-        reduce_box(rc, 64);
-        reduce_box(rd, 96);
+        reduce_box(ra, 64);
+        reduce_box(rb, 96);
         ++gi;
       }
       if (!ok) break;
