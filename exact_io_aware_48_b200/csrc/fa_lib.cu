@@ -17,7 +17,8 @@
 #include "fa_mask.cuh"
 
 // The device error codes are the fa_status values the host returns for them.
-static_assert(fa::kDevTimeout == FA_ERR_TIMEOUT && fa::kDevBounds == FA_ERR_BOUNDS, "device error codes");
+static_assert((int)fa::kDevTimeout == (int)FA_ERR_TIMEOUT && (int)fa::kDevBounds == (int)FA_ERR_BOUNDS,
+              "device error codes");
 
 namespace {
 
