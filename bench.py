@@ -313,7 +313,7 @@ def check_status(lib, stream, where):
         raise RuntimeError(f"{where}: device status {lib.fa_status_string(status)}")
 
 
-def measure_config(name, stream, flush, peak, hbm, p=None, reps=10):
+def measure_config(name, stream, flush, peak, hbm, p=None, reps=20):
     """Forward and backward of one workload, each timed alone (median of `reps` calls, L2 flushed before each):
     call-level ms and TFLOP/s, the main kernels' own ms (events around their launches), fractions of the dense bf16
     peak, and HBM GB/s by algorithmic bytes for the short-sequence workloads.  Block-sparse: TFLOP/s count kept-tile
@@ -324,7 +324,7 @@ def measure_config(name, stream, flush, peak, hbm, p=None, reps=10):
     own = p is None
     if own:
         p = Problem(w)
-    for _ in range(3):
+    for _ in range(5):  # warm-up steps
         p.step(stream)
     f_ms, fk = time_loop(p.fwd, reps, stream, flush, (_lib.FA_KERNEL_FWD, _lib))
     b_ms, bk = time_loop(p.bwd, reps, stream, flush, (_lib.FA_KERNEL_BWD_MAIN, _lib))
@@ -405,15 +405,15 @@ def measure_varlen(stream, flush, peak):
     for _ in range(3):
         fwd(stream)
         bwd(stream)
-    f_ms, _ = time_loop(fwd, 10, stream, flush)
-    b_ms, _ = time_loop(bwd, 10, stream, flush)
+    f_ms, _ = time_loop(fwd, 20, stream, flush)
+    b_ms, _ = time_loop(bwd, 20, stream, flush)
     f, b = statistics.median(f_ms), statistics.median(b_ms)
     check_status(_lib, stream, "packed-batch kernels")
     padded = Problem(w)  # the same shape padded to N with key lengths
     for _ in range(3):
         padded.step(stream)
-    pf_ms, _ = time_loop(padded.fwd, 10, stream, flush)
-    pb_ms, _ = time_loop(padded.bwd, 10, stream, flush)
+    pf_ms, _ = time_loop(padded.fwd, 20, stream, flush)
+    pb_ms, _ = time_loop(padded.bwd, 20, stream, flush)
     pf, pb = statistics.median(pf_ms), statistics.median(pb_ms)
     out = {"workload": f"packed BERT-large shape B{B} H{H} d{d} bf16, lengths U[128,512], total {total} tokens",
            "fwd_ms": round(f, 4), "bwd_ms": round(b, 4),
