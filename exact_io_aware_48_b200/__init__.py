@@ -13,7 +13,7 @@ from . import _lib
 from ._lib import (FA_BF16, FA_FP16, FA_OK, FA_ERR_CUDA, FA_ERR_INVALID_ARG, FA_ERR_TIMEOUT, FA_ERR_UNSUPPORTED,
                    FA_ERR_WORKSPACE)
 
-__all__ = ["attention_fwd", "attention_bwd", "attention_fwd_varlen", "attention_bwd_varlen",
+__all__ = ["attention", "attention_fwd", "attention_bwd", "attention_fwd_varlen", "attention_bwd_varlen",
            "attention_fwd_splitkv", "blockmask_lists", "FAError", "FA_BF16", "FA_FP16"]
 
 
@@ -93,6 +93,45 @@ def attention_bwd(q, k, v, o, dout, lse, causal=False, softmax_scale=None, key_l
     _check(_lib.fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, causal, key_lens, block_mask, ws,
                        ws_bytes, _dtype_code(q), stream), "fa_bwd")
     return dq, dk, dv
+
+
+_AUTOGRAD_FN = None
+
+
+def _autograd_fn():
+    """torch.autograd.Function over attention_fwd / attention_bwd (built on first use, so importing this package
+    does not import torch)."""
+    global _AUTOGRAD_FN
+    if _AUTOGRAD_FN is None:
+        import torch
+
+        class _Attention(torch.autograd.Function):
+            @staticmethod
+            def forward(ctx, q, k, v, causal, softmax_scale, key_lens, block_mask):
+                o, lse = attention_fwd(q, k, v, causal=causal, softmax_scale=softmax_scale, key_lens=key_lens,
+                                       block_mask=block_mask)
+                ctx.save_for_backward(q, k, v, o, lse)
+                ctx.args = (causal, softmax_scale, key_lens, block_mask)
+                return o
+
+            @staticmethod
+            def backward(ctx, dout):
+                q, k, v, o, lse = ctx.saved_tensors
+                causal, softmax_scale, key_lens, block_mask = ctx.args
+                dq, dk, dv = attention_bwd(q, k, v, o, dout.contiguous(), lse, causal=causal,
+                                           softmax_scale=softmax_scale, key_lens=key_lens, block_mask=block_mask)
+                return dq, dk, dv, None, None, None, None
+
+        _AUTOGRAD_FN = _Attention
+    return _AUTOGRAD_FN
+
+
+def attention(q, k, v, causal=False, softmax_scale=None, key_lens=None, block_mask=None):
+    """O = exact attention of [B, H, N, d] CUDA tensors (bf16 or fp16), differentiable through torch autograd: the
+    forward saves O and the per-row logsumexp, and the backward of the graph calls the library's backward (the
+    score and probability tiles are recomputed, never stored).  Arguments as for attention_fwd; q, k, v must be
+    contiguous."""
+    return _autograd_fn().apply(q, k, v, causal, softmax_scale, key_lens, block_mask)
 
 
 def blockmask_lists(mask, stream=None):
