@@ -13,7 +13,7 @@ from . import _lib
 from ._lib import (FA_BF16, FA_FP16, FA_OK, FA_ERR_CUDA, FA_ERR_INVALID_ARG, FA_ERR_TIMEOUT, FA_ERR_UNSUPPORTED,
                    FA_ERR_WORKSPACE)
 
-__all__ = ["attention", "attention_fwd", "attention_bwd", "attention_fwd_varlen", "attention_bwd_varlen",
+__all__ = ["attention", "attention_varlen", "attention_fwd", "attention_bwd", "attention_fwd_varlen", "attention_bwd_varlen",
            "attention_fwd_splitkv", "blockmask_lists", "FAError", "FA_BF16", "FA_FP16"]
 
 
@@ -99,8 +99,8 @@ _AUTOGRAD_FN = None
 
 
 def _autograd_fn():
-    """torch.autograd.Function over attention_fwd / attention_bwd (built on first use, so importing this package
-    does not import torch)."""
+    """torch.autograd.Functions over attention_fwd / attention_bwd and their packed variants (built on first use, so
+    importing this package does not import torch)."""
     global _AUTOGRAD_FN
     if _AUTOGRAD_FN is None:
         import torch
@@ -122,7 +122,24 @@ def _autograd_fn():
                                            softmax_scale=softmax_scale, key_lens=key_lens, block_mask=block_mask)
                 return dq, dk, dv, None, None, None, None
 
-        _AUTOGRAD_FN = _Attention
+        class _AttentionVarlen(torch.autograd.Function):
+            @staticmethod
+            def forward(ctx, q, k, v, cu_q, cu_k, max_q, max_k, causal, softmax_scale):
+                o, lse = attention_fwd_varlen(q, k, v, cu_q, cu_k, max_q, max_k, causal=causal,
+                                              softmax_scale=softmax_scale)
+                ctx.save_for_backward(q, k, v, o, lse, cu_q, cu_k)
+                ctx.args = (max_q, max_k, causal, softmax_scale)
+                return o
+
+            @staticmethod
+            def backward(ctx, dout):
+                q, k, v, o, lse, cu_q, cu_k = ctx.saved_tensors
+                max_q, max_k, causal, softmax_scale = ctx.args
+                dq, dk, dv = attention_bwd_varlen(q, k, v, o, dout.contiguous(), lse, cu_q, cu_k, max_q, max_k,
+                                                  causal=causal, softmax_scale=softmax_scale)
+                return dq, dk, dv, None, None, None, None, None, None
+
+        _AUTOGRAD_FN = (_Attention, _AttentionVarlen)
     return _AUTOGRAD_FN
 
 
@@ -131,7 +148,15 @@ def attention(q, k, v, causal=False, softmax_scale=None, key_lens=None, block_ma
     forward saves O and the per-row logsumexp, and the backward of the graph calls the library's backward (the
     score and probability tiles are recomputed, never stored).  Arguments as for attention_fwd; q, k, v must be
     contiguous."""
-    return _autograd_fn().apply(q, k, v, causal, softmax_scale, key_lens, block_mask)
+    return _autograd_fn()[0].apply(q, k, v, causal, softmax_scale, key_lens, block_mask)
+
+
+def attention_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, causal=False,
+                     softmax_scale=None):
+    """O of a packed variable-length batch (arguments as for attention_fwd_varlen), differentiable through torch
+    autograd like attention()."""
+    return _autograd_fn()[1].apply(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, causal,
+                                   softmax_scale)
 
 
 def blockmask_lists(mask, stream=None):

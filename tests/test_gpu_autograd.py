@@ -55,3 +55,23 @@ def test_autograd_matches_direct_backward_and_oracle(B, H, N, d, dtype, causal, 
     assert_o_close(o.detach().cpu().double().numpy(), ro)
     for got, ref, name in ((q.grad, rq, "dQ"), (k.grad, rk, "dK"), (v.grad, rv, "dV")):
         assert_grad_close(got.cpu().double().numpy(), ref, name)
+
+
+def test_autograd_varlen_matches_oracle():
+    lens = [130, 1, 257]
+    cq = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    H, d, total = 2, 64, int(cq[-1])
+    q, k, v = [inputs.gaussian((total, H, d), 620 + t, "bf16").cuda().requires_grad_() for t in range(3)]
+    g = inputs.gaussian((total, H, d), 630, "bf16").cuda().float()
+    cqd = torch.as_tensor(cq).cuda()
+    o = fa.attention_varlen(q, k, v, cqd, cqd, max(lens), max(lens), causal=True)
+    (o.float() * g).sum().backward()
+    assert fa.last_device_status() == 0
+    do = g.to(o.dtype)
+    scale = 1.0 / math.sqrt(d)
+    rq, rk, rv, ro, _ = oracle.attn_bwd_varlen(f64(q.detach().cpu()), f64(k.detach().cpu()), f64(v.detach().cpu()),
+                                               f64(do.cpu()), cq, cq, scale, causal=True)
+    assert_o_close(o.detach().cpu().double().numpy(), ro)
+    for got, ref, name in ((q.grad, rq, "dQ"), (k.grad, rk, "dK"), (v.grad, rv, "dV")):
+        assert_grad_close(got.cpu().double().numpy(), ref, name)
+
